@@ -1,0 +1,77 @@
+// Shared host/device helpers of the fg library (status handling, fp16 bit helpers,
+// 4-bit code expansion).  Nothing here allocates device memory.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include "../../include/fg.h"
+
+namespace fg {
+
+// ------------------------------------------------------------------ host-side errors
+void set_error(const char* fmt, ...);
+int fail(int status, const char* fmt, ...);
+int cuda_fail(cudaError_t e, const char* what);
+
+#define FG_CHECK_CUDA(expr)                               \
+  do {                                                    \
+    cudaError_t _e = (expr);                              \
+    if (_e != cudaSuccess) return ::fg::cuda_fail(_e, #expr); \
+  } while (0)
+
+#define FG_CHECK_LAUNCH(what)                               \
+  do {                                                      \
+    cudaError_t _e = cudaGetLastError();                    \
+    if (_e != cudaSuccess) return ::fg::cuda_fail(_e, what); \
+  } while (0)
+
+#define FG_TRY(expr)                 \
+  do {                               \
+    int _s = (expr);                 \
+    if (_s != FG_OK) return _s;      \
+  } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int num_sms();
+
+// Kernel classes for fg_profile_* (same numbering as the header).
+enum ProfKind { PROF_GEMM = 0, PROF_DECODE_ATTN = 1, PROF_PREFILL_ATTN = 2, PROF_QUANT = 3,
+                PROF_OTHER = 4, PROF_NKINDS = 5 };
+// RAII pair of events around a launch when profiling is on.
+struct ProfScope {
+  int slot;
+  cudaStream_t s;
+  ProfScope(int kind, cudaStream_t s, double flops, double bytes);
+  ~ProfScope();
+};
+
+// ------------------------------------------------------------------ device helpers
+__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+// Eight 4-bit codes of one 32-bit word (element i in bits 4i..4i+3) expanded to the
+// exact fp16 values mn + code*s, one rounding each (fma.rn.f16x2 rounds the exact
+// a*b+c once).  (1024 + code) is built by OR-ing the code into the mantissa of 1024.0
+// (0x6400) and 1024 is then subtracted exactly.  Output pairs in element order:
+// out[j] = {x[2j], x[2j+1]}.
+__device__ __forceinline__ void dequant8(uint32_t w, __half2 s2, __half2 mn2, uint32_t out[4]) {
+  const uint32_t MAGIC = 0x64006400u;  // {1024.0, 1024.0}
+  const __half2 K1024 = u32_as_h2(MAGIC);
+  // even elements of bytes 0..3 at nibble positions 0,2,4,6 ; odd at 1,3,5,7
+  // pair j = {elem 2j, elem 2j+1} = {nibble 2j, nibble 2j+1} of w.
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t byte = (w >> (8 * j)) & 0xFFu;
+    uint32_t lohi = (byte & 0x0Fu) | ((byte & 0xF0u) << 12);  // lo -> bits 0..3, hi -> 16..19
+    __half2 h = u32_as_h2(lohi | MAGIC);
+    __half2 q = __hsub2(h, K1024);
+    out[j] = h2_as_u32(__hfma2(q, s2, mn2));
+  }
+}
+
+}  // namespace fg

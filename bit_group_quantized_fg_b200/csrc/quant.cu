@@ -1,0 +1,372 @@
+// K1 quantize/pack (weights and KV append) and K2 dequantize.
+//
+// Definition ("FlexGen" README mirror, key features "Extreme Compression": weights and
+// attention cache to 4 bits; group-wise asymmetric min-max with fp16 {min, scale} per
+// group of G consecutive elements), per group:
+//   mn = min, mx = max (zero extremes as +0); s = fp16(fp32(mx - mn) / 15);
+//   code = clamp(rint(fp32(x - mn) / s), 0, 15), every code 0 when s == 0.
+// All fp32 steps use explicitly rounded intrinsics (__fsub_rn/__fdiv_rn), so no FMA
+// contraction or reciprocal approximation can change a code.
+//
+// Layout of a row-grouped (axis=1) tensor: 16-byte chunks of 8 fp16 values; one thread
+// owns one chunk, G/8 adjacent lanes own one group and combine min/max with xor
+// shuffles.  A chunk's 8 codes form one 32-bit word (element i in bits 4i..4i+3, i.e.
+// byte j = code(2j) | code(2j+1) << 4).  Loads are 128-bit and read-only cached; the
+// loop is grid-stride over tiles of blockDim*U chunks with all U loads issued first.
+#include <algorithm>
+
+#include "fg_common.cuh"
+
+namespace fg {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+struct GroupQ {
+  uint32_t word;  // 8 packed codes
+  __half2 params; // {mn, s}
+};
+
+// Quantize the 8 values of `v` as part of a group spread over TPG adjacent lanes.
+// Every lane of the warp must call this (shuffles use the full mask).
+template <int TPG>
+__device__ __forceinline__ GroupQ quantize_chunk(uint4 v) {
+  float x[8];
+  {
+    const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 f = __half22float2(h[j]);
+      x[2 * j] = f.x;
+      x[2 * j + 1] = f.y;
+    }
+  }
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    mn = fminf(mn, x[i]);
+    mx = fmaxf(mx, x[i]);
+  }
+#pragma unroll
+  for (int o = 1; o < TPG; o <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  mn = __fadd_rn(mn, 0.0f);  // -0 -> +0
+  mx = __fadd_rn(mx, 0.0f);
+  const float d = __fsub_rn(mx, mn);
+  const __half s16 = __float2half_rn(__fdiv_rn(d, 15.0f));
+  const float sf = __half2float(s16);
+  const bool zero = (sf == 0.0f);
+  const float den = zero ? 1.0f : sf;
+  uint32_t word = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int q = __float2int_rn(__fdiv_rn(__fsub_rn(x[i], mn), den));
+    q = q < 0 ? 0 : (q > 15 ? 15 : q);
+    if (zero) q = 0;
+    word |= uint32_t(q) << (4 * i);
+  }
+  GroupQ r;
+  r.word = word;
+  r.params = __halves2half2(__float2half_rn(mn), s16);
+  return r;
+}
+
+// ------------------------------------------------------------------ K1, axis = 1
+template <int G>
+__global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const uint4* __restrict__ x,
+                                                                 int64_t n_chunks,
+                                                                 uint32_t* __restrict__ codes,
+                                                                 __half2* __restrict__ params) {
+  constexpr int TPG = G / 8;
+  const int64_t tile = int64_t(kThreads) * kUnroll;
+  for (int64_t base = int64_t(blockIdx.x) * tile; base < n_chunks; base += int64_t(gridDim.x) * tile) {
+    uint4 v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t c = base + u * kThreads + threadIdx.x;
+      v[u] = c < n_chunks ? ld_nc_v4(x + c) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t c = base + u * kThreads + threadIdx.x;
+      GroupQ q = quantize_chunk<TPG>(v[u]);
+      if (c < n_chunks) {
+        codes[c] = q.word;
+        if ((threadIdx.x % TPG) == 0) params[c / TPG] = q.params;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ KV append
+// Rows r = b*T + t of k (blockIdx.y == 0) or v (== 1); h valid values per row.
+// Group g of head `hd`-slice lands at cache position len + t.
+template <int G>
+__global__ void __launch_bounds__(kThreads) kv_append_kernel(
+    const __half* __restrict__ k, const __half* __restrict__ v, int64_t row_stride, int T, int h,
+    int hd, int cap, int pos0, int64_t n_chunks, uint32_t* __restrict__ kc, uint32_t* __restrict__ vc,
+    __half2* __restrict__ kp, __half2* __restrict__ vp) {
+  constexpr int TPG = G / 8;
+  const __half* src = blockIdx.y == 0 ? k : v;
+  uint32_t* dc = blockIdx.y == 0 ? kc : vc;
+  __half2* dp = blockIdx.y == 0 ? kp : vp;
+  const int chunks_per_row = h / 8;
+  const int nh = h / hd;
+  const int64_t tile = int64_t(kThreads) * kUnroll;
+  for (int64_t base = int64_t(blockIdx.x) * tile; base < n_chunks; base += int64_t(gridDim.x) * tile) {
+    uint4 val[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t c = base + u * kThreads + threadIdx.x;
+      if (c < n_chunks) {
+        const int64_t row = c / chunks_per_row;
+        const int cc = int(c - row * chunks_per_row);
+        val[u] = ld_nc_v4(src + row * row_stride + cc * 8);
+      } else {
+        val[u] = make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t c = base + u * kThreads + threadIdx.x;
+      GroupQ q = quantize_chunk<TPG>(val[u]);
+      if (c < n_chunks) {
+        const int64_t row = c / chunks_per_row;
+        const int cc = int(c - row * chunks_per_row);
+        const int64_t b = row / T;
+        const int t = int(row - b * T);
+        const int d = cc * 8;
+        const int head = d / hd;
+        const int dh = d - head * hd;
+        const int64_t slot = (b * nh + head) * int64_t(cap) + (pos0 + t);
+        dc[slot * (hd / 8) + dh / 8] = q.word;
+        if ((threadIdx.x % TPG) == 0) dp[slot * (hd / G) + dh / G] = q.params;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ K1, axis = 0
+// One thread per (column pair, row group); min/max down the G rows of its two columns.
+__global__ void __launch_bounds__(kThreads) quantize_cols_kernel(const __half2* __restrict__ x,
+                                                                 int64_t rows, int64_t cols, int G,
+                                                                 uint8_t* __restrict__ codes,
+                                                                 __half2* __restrict__ params) {
+  const int64_t pairs = cols / 2;
+  const int64_t p = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (p >= pairs) return;
+  for (int64_t rg = blockIdx.y; rg < rows / G; rg += gridDim.y) {
+    const __half2* col = x + rg * G * pairs + p;
+    float mn0 = INFINITY, mx0 = -INFINITY, mn1 = INFINITY, mx1 = -INFINITY;
+    for (int r = 0; r < G; ++r) {
+      float2 f = __half22float2(col[int64_t(r) * pairs]);
+      mn0 = fminf(mn0, f.x);
+      mx0 = fmaxf(mx0, f.x);
+      mn1 = fminf(mn1, f.y);
+      mx1 = fmaxf(mx1, f.y);
+    }
+    mn0 = __fadd_rn(mn0, 0.0f);
+    mx0 = __fadd_rn(mx0, 0.0f);
+    mn1 = __fadd_rn(mn1, 0.0f);
+    mx1 = __fadd_rn(mx1, 0.0f);
+    const __half s0 = __float2half_rn(__fdiv_rn(__fsub_rn(mx0, mn0), 15.0f));
+    const __half s1 = __float2half_rn(__fdiv_rn(__fsub_rn(mx1, mn1), 15.0f));
+    const float sf0 = __half2float(s0), sf1 = __half2float(s1);
+    const float d0 = sf0 == 0.0f ? 1.0f : sf0, d1 = sf1 == 0.0f ? 1.0f : sf1;
+    params[rg * cols + 2 * p] = __halves2half2(__float2half_rn(mn0), s0);
+    params[rg * cols + 2 * p + 1] = __halves2half2(__float2half_rn(mn1), s1);
+    for (int r = 0; r < G; ++r) {
+      float2 f = __half22float2(col[int64_t(r) * pairs]);
+      int q0 = __float2int_rn(__fdiv_rn(__fsub_rn(f.x, mn0), d0));
+      int q1 = __float2int_rn(__fdiv_rn(__fsub_rn(f.y, mn1), d1));
+      q0 = q0 < 0 ? 0 : (q0 > 15 ? 15 : q0);
+      q1 = q1 < 0 ? 0 : (q1 > 15 ? 15 : q1);
+      if (sf0 == 0.0f) q0 = 0;
+      if (sf1 == 0.0f) q1 = 0;
+      codes[(rg * G + r) * pairs + p] = uint8_t(q0 | (q1 << 4));
+    }
+  }
+}
+
+// ------------------------------------------------------------------ K2 dequantize
+// axis = 1: one thread per code word (8 elements, one group's params).
+template <int G>
+__global__ void __launch_bounds__(kThreads) dequant_rows_kernel(const uint32_t* __restrict__ codes,
+                                                                const __half2* __restrict__ params,
+                                                                int64_t n_words,
+                                                                uint4* __restrict__ out) {
+  constexpr int WPG = G / 8;
+  const int64_t tile = int64_t(kThreads) * kUnroll;
+  for (int64_t base = int64_t(blockIdx.x) * tile; base < n_words; base += int64_t(gridDim.x) * tile) {
+    uint32_t w[kUnroll];
+    __half2 p[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t c = base + u * kThreads + threadIdx.x;
+      w[u] = c < n_words ? __ldg(codes + c) : 0u;
+      p[u] = c < n_words ? __ldg(params + c / WPG) : __half2();
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t c = base + u * kThreads + threadIdx.x;
+      if (c < n_words) {
+        uint32_t o[4];
+        dequant8(w[u], __high2half2(p[u]), __low2half2(p[u]), o);
+        out[c] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+  }
+}
+
+// axis = 0: one thread per code word; the 8 columns have their own params.
+__global__ void __launch_bounds__(kThreads) dequant_cols_kernel(const uint32_t* __restrict__ codes,
+                                                                const __half2* __restrict__ params,
+                                                                int64_t rows, int64_t cols, int G,
+                                                                uint4* __restrict__ out) {
+  const int64_t words_per_row = cols / 8;
+  const int64_t n_words = rows * words_per_row;
+  for (int64_t c = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; c < n_words;
+       c += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = c / words_per_row;
+    const int64_t col0 = (c - r * words_per_row) * 8;
+    const uint32_t w = __ldg(codes + c);
+    const __half2* pr = params + (r / G) * cols + col0;
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      __half2 pa = __ldg(pr + 2 * j), pb = __ldg(pr + 2 * j + 1);
+      const __half2 s2 = __halves2half2(__high2half(pa), __high2half(pb));
+      const __half2 m2 = __halves2half2(__low2half(pa), __low2half(pb));
+      uint32_t pair[4];
+      dequant8((w >> (8 * j)) & 0xFFu, s2, m2, pair);  // only pair[0] is used
+      o[j] = pair[0];
+    }
+    out[c] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+int grid_for(int64_t units, int64_t per_block) {
+  int64_t blocks = (units + per_block - 1) / per_block;
+  const int64_t cap = int64_t(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return int(blocks);
+}
+
+int check_qargs(const void* a, const void* b, const void* c, int64_t rows, int64_t cols, int group,
+                int axis) {
+  if (!a || !b || !c) return fail(FG_ERR_INVALID_ARG, "null pointer");
+  if (rows < 0 || cols < 0) return fail(FG_ERR_SHAPE, "negative size");
+  if (group != 32 && group != 64 && group != 128)
+    return fail(FG_ERR_SHAPE, "group must be 32, 64 or 128 (got %d)", group);
+  if (axis != 0 && axis != 1) return fail(FG_ERR_INVALID_ARG, "axis must be 0 or 1");
+  if (cols % 8) return fail(FG_ERR_SHAPE, "cols must be a multiple of 8");
+  if (axis == 1 && cols % group) return fail(FG_ERR_SHAPE, "cols %% group != 0");
+  if (axis == 0 && rows % group) return fail(FG_ERR_SHAPE, "rows %% group != 0");
+  if (rows > 0 && cols > 0 && rows > (int64_t(1) << 34) / cols)
+    return fail(FG_ERR_SHAPE, "tensor larger than 2^34 elements");
+  if (!aligned16(a) || !aligned16(b) || !aligned16(c)) return fail(FG_ERR_ALIGN, "pointers must be 16-byte aligned");
+  return FG_OK;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ host entry points
+int quantize_pack_impl(const void* x, int64_t rows, int64_t cols, int group, int axis,
+                       uint8_t* codes, void* params, cudaStream_t s) {
+  FG_TRY(check_qargs(x, codes, params, rows, cols, group, axis));
+  const int64_t n = rows * cols;
+  if (n == 0) return FG_OK;
+  ProfScope ps(PROF_QUANT, s, 0.0, double(n) * (2.0 + 0.5 + 4.0 / group));
+  if (axis == 1) {
+    const int64_t chunks = n / 8;
+    const int grid = grid_for(chunks, int64_t(kThreads) * kUnroll);
+    auto* xin = reinterpret_cast<const uint4*>(x);
+    auto* cw = reinterpret_cast<uint32_t*>(codes);
+    auto* pw = reinterpret_cast<__half2*>(params);
+    if (group == 32) quantize_rows_kernel<32><<<grid, kThreads, 0, s>>>(xin, chunks, cw, pw);
+    else if (group == 64) quantize_rows_kernel<64><<<grid, kThreads, 0, s>>>(xin, chunks, cw, pw);
+    else quantize_rows_kernel<128><<<grid, kThreads, 0, s>>>(xin, chunks, cw, pw);
+  } else {
+    const int64_t pairs = cols / 2;
+    dim3 grid(unsigned((pairs + kThreads - 1) / kThreads),
+              unsigned(std::min<int64_t>(rows / group, 65535)));
+    quantize_cols_kernel<<<grid, kThreads, 0, s>>>(reinterpret_cast<const __half2*>(x), rows, cols,
+                                                   group, codes, reinterpret_cast<__half2*>(params));
+  }
+  FG_CHECK_LAUNCH("quantize kernel");
+  return FG_OK;
+}
+
+int dequantize_impl(const uint8_t* codes, const void* params, int64_t rows, int64_t cols, int group,
+                    int axis, void* out, cudaStream_t s) {
+  FG_TRY(check_qargs(codes, params, out, rows, cols, group, axis));
+  const int64_t n = rows * cols;
+  if (n == 0) return FG_OK;
+  ProfScope ps(PROF_QUANT, s, 0.0, double(n) * (2.0 + 0.5 + 4.0 / group));
+  const int64_t words = n / 8;
+  auto* cw = reinterpret_cast<const uint32_t*>(codes);
+  auto* pw = reinterpret_cast<const __half2*>(params);
+  auto* o = reinterpret_cast<uint4*>(out);
+  if (axis == 1) {
+    const int grid = grid_for(words, int64_t(kThreads) * kUnroll);
+    if (group == 32) dequant_rows_kernel<32><<<grid, kThreads, 0, s>>>(cw, pw, words, o);
+    else if (group == 64) dequant_rows_kernel<64><<<grid, kThreads, 0, s>>>(cw, pw, words, o);
+    else dequant_rows_kernel<128><<<grid, kThreads, 0, s>>>(cw, pw, words, o);
+  } else {
+    const int grid = grid_for(words, kThreads);
+    dequant_cols_kernel<<<grid, kThreads, 0, s>>>(cw, pw, rows, cols, group, o);
+  }
+  FG_CHECK_LAUNCH("dequantize kernel");
+  return FG_OK;
+}
+
+int kv_append_impl(fg_kv_cache* c, const void* k, const void* v, int64_t row_stride, int n_tokens,
+                   cudaStream_t s) {
+  if (!c || !k || !v) return fail(FG_ERR_INVALID_ARG, "null pointer");
+  if (!c->k_codes || !c->v_codes || !c->k_params || !c->v_params)
+    return fail(FG_ERR_INVALID_ARG, "cache buffers not set");
+  const int hd = c->head_dim, G = c->group;
+  if (G != 32 && G != 64 && G != 128) return fail(FG_ERR_SHAPE, "cache group must be 32, 64 or 128");
+  if (hd <= 0 || hd % G || hd % 8) return fail(FG_ERR_SHAPE, "group must divide head_dim");
+  if (c->B <= 0 || c->n_heads <= 0 || n_tokens < 0) return fail(FG_ERR_SHAPE, "bad cache shape");
+  const int h = c->n_heads * hd;
+  if (row_stride < h || row_stride % 8) return fail(FG_ERR_ALIGN, "row_stride must be >= h and a multiple of 8");
+  if (c->len < 0 || int64_t(c->len) + n_tokens > c->capacity)
+    return fail(FG_ERR_CAPACITY, "KV cache capacity %d exceeded (len %d + %d)", c->capacity, c->len, n_tokens);
+  if (!aligned16(k) || !aligned16(v) || !aligned16(c->k_codes) || !aligned16(c->v_codes) ||
+      !aligned16(c->k_params) || !aligned16(c->v_params))
+    return fail(FG_ERR_ALIGN, "pointers must be 16-byte aligned");
+  if (n_tokens == 0) return FG_OK;
+  const int64_t chunks = int64_t(c->B) * n_tokens * (h / 8);
+  ProfScope ps(PROF_QUANT, s, 0.0, double(chunks) * 8 * 2 * (2.0 + 0.5 + 4.0 / G));
+  dim3 grid(unsigned(grid_for(chunks, int64_t(kThreads) * kUnroll)), 2);
+  auto* K = reinterpret_cast<const __half*>(k);
+  auto* V = reinterpret_cast<const __half*>(v);
+  auto* kc = reinterpret_cast<uint32_t*>(c->k_codes);
+  auto* vc = reinterpret_cast<uint32_t*>(c->v_codes);
+  auto* kp = reinterpret_cast<__half2*>(c->k_params);
+  auto* vp = reinterpret_cast<__half2*>(c->v_params);
+  if (G == 32)
+    kv_append_kernel<32><<<grid, kThreads, 0, s>>>(K, V, row_stride, n_tokens, h, hd, c->capacity, c->len, chunks, kc, vc, kp, vp);
+  else if (G == 64)
+    kv_append_kernel<64><<<grid, kThreads, 0, s>>>(K, V, row_stride, n_tokens, h, hd, c->capacity, c->len, chunks, kc, vc, kp, vp);
+  else
+    kv_append_kernel<128><<<grid, kThreads, 0, s>>>(K, V, row_stride, n_tokens, h, hd, c->capacity, c->len, chunks, kc, vc, kp, vp);
+  FG_CHECK_LAUNCH("kv append kernel");
+  c->len += n_tokens;
+  return FG_OK;
+}
+
+}  // namespace fg

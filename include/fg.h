@@ -1,0 +1,213 @@
+/*
+ * fg.h - C ABI of the 4-bit group-wise compressed decode path (B200, sm_100a).
+ *
+ * What the path computes comes from the FlexGen pages: weights and the attention (KV)
+ * cache are compressed to 4 bits ("FlexGen" README mirror, key features, "Extreme
+ * Compression"; arXiv 2303.06865 record, abstract), OPT-shaped models are generated with
+ * input length 512 and output length 32, and throughput is generated tokens divided by
+ * (prompt time + generation time) ("FlexGen" README mirror, benchmark table notes).
+ * The quantizer details the pages leave open (group size/axis, rounding, layout) are
+ * stated at each call below.
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library never
+ *    allocates or frees device memory (scratch comes from a caller-provided workspace).
+ *  - fp16 means IEEE binary16 ("half"); half2 params are {min, scale} pairs, min first.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ *    default stream), except fg_generate, which synchronizes to fill its timing record.
+ *  - Arguments are validated on the host before any launch; on failure nothing is
+ *    launched and a negative fg_status is returned.  fg_last_error() gives a
+ *    thread-local message for the last failure.  Launch failures return FG_ERR_CUDA.
+ *  - Pointers must be 16-byte aligned unless stated otherwise (FG_ERR_ALIGN).
+ */
+#ifndef FG_H
+#define FG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FG_OK = 0,
+  FG_ERR_INVALID_ARG = -1, /* null pointer, bad enum value                        */
+  FG_ERR_SHAPE = -2,       /* sizes inconsistent, group does not divide the axis  */
+  FG_ERR_ALIGN = -3,       /* pointer or stride not aligned as required          */
+  FG_ERR_CAPACITY = -4,    /* KV cache would overflow its capacity                */
+  FG_ERR_CUDA = -5,        /* a CUDA runtime/driver call or a launch failed        */
+  FG_ERR_UNSUPPORTED = -6, /* valid but not implemented (e.g. head_dim > 256)     */
+  FG_ERR_WORKSPACE = -7    /* workspace missing or smaller than required          */
+} fg_status;
+
+const char* fg_status_string(int status); /* static string for a status code */
+const char* fg_last_error(void);           /* thread-local detail of the last error */
+int fg_version(void);                      /* library version (major*10000+minor*100+patch) */
+
+/* ------------------------------------------------------------------------------------
+ * Quantize / pack (compression of a weight or KV tensor to 4 bits).
+ *
+ * Source: "FlexGen" README mirror, key features ("Extreme Compression": parameters and
+ * attention cache down to 4 bits) and the out-of-memory tips (weight compression saves
+ * about 70 % of weight memory: 4 bits + 2 fp16 per 64 elements = 71.9 %).
+ * Definition (readings where the pages are silent), per group of `group` consecutive
+ * elements along `axis`:
+ *   mn = min, mx = max (a zero extreme is stored as +0)
+ *   s  = fp16( fp32(mx - mn) / 15 )          fp32 subtract, fp32 IEEE divide, RNE to fp16
+ *   code = clamp( rint( fp32(x - mn) / s ), 0, 15 )   fp32 ops, half-to-even; s==0 -> 0
+ * Layout:
+ *   x      fp16 [rows][cols], row-major, 16-byte aligned.
+ *   codes  uint8 [rows][cols/2]: byte j of a row = code(col 2j) | code(col 2j+1) << 4.
+ *   params half2 {mn, s}: axis=1 -> [rows][cols/group]; axis=0 -> [rows/group][cols].
+ * group in {32, 64, 128}; axis=1 needs cols % group == 0, axis=0 needs rows % group == 0;
+ * cols must be a multiple of 8.  Sizes up to 2^34 elements (64-bit indexing).
+ * Non-finite inputs give unspecified codes.
+ * ---------------------------------------------------------------------------------- */
+int fg_quantize_pack(const void* x, int64_t rows, int64_t cols, int group, int axis,
+                     uint8_t* codes, void* params, void* stream);
+
+/* Dequantize: out = fp16(mn + code * s) with ONE rounding of the exact value.
+ * Same layouts and preconditions as fg_quantize_pack; out is fp16 [rows][cols]. */
+int fg_dequantize(const uint8_t* codes, const void* params, int64_t rows, int64_t cols,
+                  int group, int axis, void* out, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * Model state.
+ * ---------------------------------------------------------------------------------- */
+
+/* A linear layer Y = X W + b whose weight W [K][N] (math convention, N contiguous) is
+ * stored 4-bit with groups of `group` along N (the output channel):
+ *   codes  uint8 [K][N/2], params half2 [K][N/group], bias fp16 [N] (may be NULL).
+ * This is exactly fg_quantize_pack(W, K, N, group, axis=1). */
+typedef struct {
+  const uint8_t* codes;
+  const void* params;
+  const void* bias;
+  int K, N, group;
+} fg_qlinear;
+
+/* One OPT decoder block (pre-LayerNorm, MHA, ReLU FFN).  qkv: [h][3h] with output
+ * columns q | k | v; out: [h][h]; fc1: [h][F]; fc2: [F][h].  LayerNorm params fp16 [h]. */
+typedef struct {
+  const void *ln1_g, *ln1_b, *ln2_g, *ln2_b;
+  fg_qlinear qkv, out, fc1, fc2;
+} fg_layer;
+
+/* 4-bit KV cache of one layer ("FlexGen" README mirror: attention cache compressed to 4
+ * bits).  Each token's K (and V) row of h = n_heads*head_dim values is quantized in
+ * groups of `group` along the hidden dimension (group divides head_dim):
+ *   k_codes/v_codes   uint8 [B][n_heads][capacity][head_dim/2]
+ *   k_params/v_params half2 [B][n_heads][capacity][head_dim/group]
+ * `len` positions are filled, the same for every sequence; the calls below that append
+ * advance it on success. */
+typedef struct {
+  uint8_t *k_codes, *v_codes;
+  void *k_params, *v_params;
+  int B, n_heads, head_dim, group, capacity;
+  int len;
+} fg_kv_cache;
+
+typedef struct {
+  int n_layers, hidden, n_heads, head_dim, ffn, vocab, max_pos, group;
+  const void* embed;     /* fp16 [vocab][hidden], also the (tied) LM head      */
+  const void* pos_embed; /* fp16 [max_pos][hidden] learned positions           */
+  const void *lnf_g, *lnf_b;
+  const fg_layer* layers; /* HOST array of n_layers layers                      */
+} fg_model;
+
+typedef struct {
+  float prefill_ms, decode_ms; /* device time of the prompt pass and of the decode steps */
+  int64_t tokens;              /* generated tokens (B * gen_len)                          */
+  double tok_per_s;            /* tokens / (prefill + decode) seconds                     */
+} fg_timing;
+
+/* ------------------------------------------------------------------------------------
+ * Steps of the path (each one launch or a few), exposed for tests and benchmarks.
+ * ---------------------------------------------------------------------------------- */
+
+/* Append n_tokens tokens per sequence to the cache at positions len..len+n_tokens-1 and
+ * advance len.  k, v: fp16 rows, row (b*n_tokens + t) at k + row*row_stride (elements),
+ * h valid values per row; row_stride % 8 == 0.  FG_ERR_CAPACITY if it would overflow. */
+int fg_kv_append(fg_kv_cache* cache, const void* k, const void* v, int64_t row_stride,
+                 int n_tokens, void* stream);
+
+/* Dequant-fused GEMM on the tensor cores: Y[M][N] = [relu](X[M][K] W_hat + b) [+ R].
+ * X fp16 [M][K] (row stride K), R fp16 [M][N] or NULL, Y fp16 [M][N].  W_hat is the
+ * fg_dequantize of the weight (exact fp16), products accumulate in fp32.
+ * K % 64 == 0, N % 128 == 0, group in {32, 64, 128}.  `workspace` may be NULL when
+ * fg_qgemm_workspace_bytes(M, N, K) is 0. */
+size_t fg_qgemm_workspace_bytes(int64_t M, int N, int K);
+int fg_qgemm(const void* X, int64_t M, const fg_qlinear* W, const void* R, int relu, void* Y,
+             void* workspace, size_t ws_bytes, void* stream);
+
+/* Decode attention over a 4-bit cache: for each sequence b and head j,
+ * out = softmax(q K^T / sqrt(hd)) V over positions 0..cache->len-1, with K and V the
+ * dequantized cache values (mn + code*s) and an fp32 softmax.  q: fp16, row b at
+ * q + b*q_stride (elements); out fp16 [B][h].  Split over the context with partial
+ * (max, sum, acc) triples in the workspace (fg_decode_attention_workspace_bytes). */
+size_t fg_decode_attention_workspace_bytes(int B, int n_heads, int head_dim, int ctx);
+int fg_decode_attention(const void* q, int64_t q_stride, const fg_kv_cache* cache, void* out,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* Causal prefill attention on unquantized fp16 projections: qkv fp16 [B*L][3h]
+ * (q | k | v), out fp16 [B*L][h].  "FlexGen" README mirror: prompt processing time is
+ * part of the throughput metric. */
+int fg_prefill_attention(const void* qkv, int B, int L, int n_heads, int head_dim, void* out,
+                         void* stream);
+
+/* LayerNorm over rows: y = (x - mean)/sqrt(var + 1e-5) * g + b, fp32 statistics, fp16 in/out. */
+int fg_layernorm(const void* x, int64_t rows, int cols, const void* g, const void* b, void* y,
+                 void* stream);
+
+/* x[b*T + t] = fp16(E[ids[b*T+t]] + P[pos0 + t]) (one rounding). ids int32 [B][T]. */
+int fg_embed(const int32_t* ids, int B, int T, int pos0, const void* E, const void* P,
+             int hidden, void* out, void* stream);
+
+/* Tied LM head + greedy argmax: tokens[b] = argmax_v (x[b] . E[v]) over v < vocab, ties to
+ * the lowest id; x fp16 [B][hidden] (already final-LayerNormed); logits fp32 [B][vocab]
+ * are written when `logits` is not NULL.  Needs fg_lm_head_workspace_bytes. */
+size_t fg_lm_head_workspace_bytes(int B, int vocab);
+int fg_lm_head_argmax(const void* x, int B, int hidden, const void* E, int vocab, float* logits,
+                      int32_t* tokens, void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * Layers and generation.
+ * ---------------------------------------------------------------------------------- */
+
+/* One decoder block for one new token per sequence: x_out = block(x_in), both fp16 [B][h].
+ * Appends the token's K/V at cache->len (then attends over 0..len) and advances len.
+ * workspace >= fg_decode_layer_workspace_bytes(h, ffn, n_heads, B, cache->capacity). */
+size_t fg_decode_layer_workspace_bytes(int hidden, int ffn, int n_heads, int B, int capacity);
+int fg_decode_layer(const fg_layer* layer, fg_kv_cache* cache, const void* x_in, void* x_out,
+                    int B, void* workspace, size_t ws_bytes, void* stream);
+
+/* One decoder block over a whole prompt: x fp16 [B*L][h] in place; writes cache positions
+ * 0..L-1 (cache->len must be 0) and sets len = L.
+ * workspace >= fg_prefill_layer_workspace_bytes(h, ffn, B, L). */
+size_t fg_prefill_layer_workspace_bytes(int hidden, int ffn, int B, int L);
+int fg_prefill_layer(const fg_layer* layer, fg_kv_cache* cache, void* x, int B, int L,
+                     void* workspace, size_t ws_bytes, void* stream);
+
+/* Greedy generation ("FlexGen" README mirror, benchmark notes): prefill over the prompt
+ * (B x L ids, device int32) yields token 1, then gen_len-1 decode steps; out_ids device
+ * int32 [B][gen_len].  caches: HOST array of n_layers caches (len reset to 0 here),
+ * capacity >= L + gen_len.  Timing uses CUDA events on `stream`; this call synchronizes.
+ * workspace >= fg_workspace_bytes(model, B, L, gen_len). */
+size_t fg_workspace_bytes(const fg_model* model, int B, int L, int gen_len);
+int fg_generate(const fg_model* model, const int32_t* prompt_ids, int B, int L, int gen_len,
+                int32_t* out_ids, fg_kv_cache* caches, void* workspace, size_t ws_bytes,
+                fg_timing* timing, void* stream);
+
+/* Per-kernel device timing of the library's own launches (CUDA events on the launching
+ * stream).  kind: 0 = dequant GEMM, 1 = decode attention, 2 = prefill attention,
+ * 3 = quantize/append, 4 = other.  Enabling adds one event pair per launch. */
+int fg_profile_enable(int on);
+int fg_profile_read(int kind, double* total_ms, int64_t* launches, double* flops,
+                    double* bytes);
+int fg_profile_reset(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FG_H */

@@ -25,12 +25,12 @@ oracle takes where they are silent are listed in the module docstrings of
 from .quant import (quantize_groups, dequantize_groups, pack_nibbles, unpack_nibbles,
                     quantize_pack, dequantize, storage_bytes)
 from .decoder import (layernorm, qlinear, linear_fp16, prefill_attention, decode_attention,
-                      kv_append, cache_dequant, decode_layer, prefill_layer, generate, embed,
+                      kv_append, cache_dequant, cache_values, decode_layer, prefill_layer, generate, embed,
                       lm_head_argmax, QLinear, QLayer, KVCache, Model)
 
 __all__ = [
     "quantize_groups", "dequantize_groups", "pack_nibbles", "unpack_nibbles",
     "quantize_pack", "dequantize", "storage_bytes", "layernorm", "qlinear", "linear_fp16",
-    "prefill_attention", "decode_attention", "kv_append", "cache_dequant", "decode_layer",
+    "prefill_attention", "decode_attention", "kv_append", "cache_dequant", "cache_values", "decode_layer",
     "prefill_layer", "generate", "embed", "lm_head_argmax", "QLinear", "QLayer", "KVCache", "Model",
 ]

@@ -19,7 +19,9 @@ LM head).  Readings taken where the pages are silent:
 * Attention scale 1/sqrt(hd).  Prefill attention uses this pass's unquantized fp16 K/V;
   every token's K and V is then appended to the 4-bit cache in groups of g along the
   hidden dimension (g divides hd).  A decode step appends the new token first and then
-  attends over all cached positions 0..len (the new one included), dequantized.
+  attends over all cached positions 0..len (the new one included).  Decode attention
+  consumes the value each code stands for, mn + code*s, exactly (no second rounding to
+  fp16); the softmax and the weighted sum are float64 here, fp32 on the GPU.
 * Embedding x = fp16(E[id] + P[pos]) (one rounding), positions 0..L-1 for the prompt and
   L+j-1 for the j-th generated token; no position offset.
 * LM head logits = LN_f(x) @ E^T with the tied fp16 embedding (not quantized); greedy
@@ -157,10 +159,27 @@ def kv_append(cache: KVCache, k16: np.ndarray, v16: np.ndarray, pos: int) -> Non
 
 
 def cache_dequant(cache: KVCache, which: str, b: int, head: int, S: int) -> np.ndarray:
-    """Dequantized K or V of one (sequence, head) for positions 0..S-1, fp16 [S, hd]."""
+    """Dequantized K or V of one (sequence, head) for positions 0..S-1, fp16 [S, hd]
+    (the storage form, as fg_dequantize would write it)."""
     codes = (cache.k_codes if which == "k" else cache.v_codes)[b, head, :S]
     params = (cache.k_params if which == "k" else cache.v_params)[b, head, :S]
     return dequantize(codes, params.reshape(-1, 2), S, cache.head_dim, cache.group, 1)
+
+
+def cache_values(cache: KVCache, which: str, b: int, head: int, S: int) -> np.ndarray:
+    """Exact values mn + code*s of one (sequence, head), positions 0..S-1, float64 [S, hd].
+
+    This is what attention consumes: the value the 4-bit code stands for, without a
+    second rounding to fp16 (the product and sum are exact in float64)."""
+    codes = (cache.k_codes if which == "k" else cache.v_codes)[b, head, :S]
+    params = (cache.k_params if which == "k" else cache.v_params)[b, head, :S].astype(np.float64)
+    g = cache.group
+    q = np.empty((S, cache.head_dim), np.float64)
+    q[:, 0::2] = codes & 0x0F
+    q[:, 1::2] = codes >> 4
+    mn = np.repeat(params[..., 0], g, axis=1)
+    sc = np.repeat(params[..., 1], g, axis=1)
+    return mn + q * sc
 
 
 def _softmax_rows(s: np.ndarray) -> np.ndarray:
@@ -198,8 +217,8 @@ def decode_attention(q16: np.ndarray, cache: KVCache, S: int) -> np.ndarray:
     for b in range(B):
         for j in range(nh):
             c = slice(j * hd, (j + 1) * hd)
-            K = _f64(cache_dequant(cache, "k", b, j, S))
-            V = _f64(cache_dequant(cache, "v", b, j, S))
+            K = cache_values(cache, "k", b, j, S)
+            V = cache_values(cache, "v", b, j, S)
             p = _softmax_rows((K @ q[b, c]) * scale)
             out[b, c] = p @ V
     return out.astype(np.float16)
