@@ -1,0 +1,503 @@
+// C ABI of the library (include/fg.h): argument checks, workspace carving, per-kernel
+// profiling, and the decoder-layer / generation orchestration over the kernels.
+//
+// Generation follows the "FlexGen" README mirror's benchmark notes: a prompt pass over
+// input length L yields the first token, then gen_len-1 decode steps; throughput =
+// generated tokens / (prompt time + generation time), both measured with CUDA events.
+#include <cstdarg>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "fg_common.cuh"
+
+namespace fg {
+
+// implemented in the kernel files
+int quantize_pack_impl(const void*, int64_t, int64_t, int, int, uint8_t*, void*, cudaStream_t);
+int dequantize_impl(const uint8_t*, const void*, int64_t, int64_t, int, int, void*, cudaStream_t);
+int kv_append_impl(fg_kv_cache*, const void*, const void*, int64_t, int, cudaStream_t);
+size_t decode_attention_ws_bytes(int, int, int, int);
+int decode_attention_impl(const void*, int64_t, const fg_kv_cache*, void*, void*, size_t, cudaStream_t);
+int prefill_attention_impl(const void*, int, int, int, int, void*, cudaStream_t);
+int layernorm_impl(const void*, int64_t, int, const void*, const void*, void*, cudaStream_t);
+int embed_impl(const int32_t*, int64_t, int, int, int, const void*, const void*, int, void*, cudaStream_t);
+int argmax_impl(const float*, int, int, int32_t*, int64_t, cudaStream_t);
+size_t qgemm_ws_bytes(int64_t, int, int);
+int gemm_impl(int, const void*, int64_t, int, int, const void*, const void*, int, const void*, const void*, int,
+              void*, bool, void*, size_t, cudaStream_t);
+int read_device_error(int*);
+
+// ---------------------------------------------------------------- errors
+static thread_local char g_err[512] = "";
+
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+}
+
+int fail(int status, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return status;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  snprintf(g_err, sizeof(g_err), "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+  return FG_ERR_CUDA;
+}
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cached[dev] = v;
+  }
+  return cached[dev];
+}
+
+// ---------------------------------------------------------------- profiling
+namespace {
+struct ProfRec {
+  int kind;
+  cudaEvent_t a, b;
+  double flops, bytes;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof_pending;
+double g_prof_ms[PROF_NKINDS] = {0};
+int64_t g_prof_n[PROF_NKINDS] = {0};
+double g_prof_flops[PROF_NKINDS] = {0};
+double g_prof_bytes[PROF_NKINDS] = {0};
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+void collect_locked() {
+  for (auto& r : g_prof_pending) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) {
+      g_prof_ms[r.kind] += ms;
+      g_prof_n[r.kind] += 1;
+      g_prof_flops[r.kind] += r.flops;
+      g_prof_bytes[r.kind] += r.bytes;
+    }
+    g_event_pool.push_back(r.a);
+    g_event_pool.push_back(r.b);
+  }
+  g_prof_pending.clear();
+}
+}  // namespace
+
+ProfScope::ProfScope(int kind, cudaStream_t st, double flops, double bytes) : slot(-1), s(st) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (!g_prof_on) return;
+  ProfRec r{kind, take_event(), take_event(), flops, bytes};
+  cudaEventRecord(r.a, s);
+  g_prof_pending.push_back(r);
+  slot = int(g_prof_pending.size()) - 1;
+}
+
+ProfScope::~ProfScope() {
+  if (slot < 0) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (slot < int(g_prof_pending.size())) cudaEventRecord(g_prof_pending[slot].b, s);
+}
+
+// ---------------------------------------------------------------- workspace carving
+namespace {
+struct Carver {
+  uint8_t* p;
+  size_t used = 0, cap;
+  Carver(void* base, size_t c) : p(reinterpret_cast<uint8_t*>(base)), cap(c) {}
+  void* take(size_t bytes) {
+    used = (used + 255) & ~size_t(255);
+    void* r = p ? p + used : nullptr;
+    used += bytes;
+    return r;
+  }
+  bool ok() const { return used <= cap; }
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int check_qlinear(const fg_qlinear& w, int K, int N, const char* name) {
+  if (!w.codes || !w.params) return fail(FG_ERR_INVALID_ARG, "%s: null weight", name);
+  if (w.K != K || w.N != N) return fail(FG_ERR_SHAPE, "%s: weight is %dx%d, expected %dx%d", name, w.K, w.N, K, N);
+  return FG_OK;
+}
+
+int check_layer(const fg_layer* L, int h, int* ffn) {
+  if (!L) return fail(FG_ERR_INVALID_ARG, "null layer");
+  if (!L->ln1_g || !L->ln1_b || !L->ln2_g || !L->ln2_b) return fail(FG_ERR_INVALID_ARG, "null LayerNorm params");
+  const int F = L->fc1.N;
+  FG_TRY(check_qlinear(L->qkv, h, 3 * h, "qkv"));
+  FG_TRY(check_qlinear(L->out, h, h, "out"));
+  FG_TRY(check_qlinear(L->fc1, h, F, "fc1"));
+  FG_TRY(check_qlinear(L->fc2, F, h, "fc2"));
+  *ffn = F;
+  return FG_OK;
+}
+
+int qlinear_run(const void* X, int64_t M, const fg_qlinear& w, const void* R, int relu, void* Y, void* ws,
+                size_t wsb, cudaStream_t s) {
+  return gemm_impl(0, X, M, w.N, w.K, w.codes, w.params, w.group, w.bias, R, relu, Y, false, ws, wsb, s);
+}
+
+size_t gemm_ws_for_layer(int64_t M, int h, int F) {
+  size_t m = qgemm_ws_bytes(M, 3 * h, h);
+  m = std::max(m, qgemm_ws_bytes(M, h, h));
+  m = std::max(m, qgemm_ws_bytes(M, F, h));
+  m = std::max(m, qgemm_ws_bytes(M, h, F));
+  return m;
+}
+
+size_t decode_ws(int h, int F, int nh, int B, int cap) {
+  size_t t = 0;
+  t += align256(size_t(B) * h * 2) * 4;        // h1, att, x1, h2
+  t += align256(size_t(B) * 3 * h * 2);        // qkv
+  t += align256(size_t(B) * F * 2);            // f
+  t += align256(gemm_ws_for_layer(B, h, F));   // split-K partials
+  t += align256(decode_attention_ws_bytes(B, nh, h / nh, cap));
+  return t + 256;
+}
+
+size_t prefill_ws(int h, int F, int B, int L) {
+  const size_t BL = size_t(B) * L;
+  size_t t = 0;
+  t += align256(BL * h * 2) * 3;     // h1/h2, att, x1
+  t += align256(BL * 3 * h * 2);     // qkv
+  t += align256(BL * F * 2);         // f
+  t += align256(gemm_ws_for_layer(int64_t(BL), h, F));
+  return t + 256;
+}
+}  // namespace
+
+int decode_layer_impl(const fg_layer* layer, fg_kv_cache* cache, const void* x_in, void* x_out, int B, void* ws,
+                      size_t ws_bytes, cudaStream_t s) {
+  if (!cache || !x_in || !x_out) return fail(FG_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || B != cache->B) return fail(FG_ERR_SHAPE, "B must equal the cache batch");
+  const int h = cache->n_heads * cache->head_dim;
+  int F = 0;
+  FG_TRY(check_layer(layer, h, &F));
+  if (cache->len + 1 > cache->capacity) return fail(FG_ERR_CAPACITY, "KV cache full (capacity %d)", cache->capacity);
+  const size_t need = decode_ws(h, F, cache->n_heads, B, cache->capacity);
+  if (!ws || ws_bytes < need) return fail(FG_ERR_WORKSPACE, "decode layer needs %zu workspace bytes", need);
+  Carver c(ws, ws_bytes);
+  void* h1 = c.take(size_t(B) * h * 2);
+  void* att = c.take(size_t(B) * h * 2);
+  void* x1 = c.take(size_t(B) * h * 2);
+  void* h2 = c.take(size_t(B) * h * 2);
+  void* qkv = c.take(size_t(B) * 3 * h * 2);
+  void* f = c.take(size_t(B) * F * 2);
+  const size_t gws_b = gemm_ws_for_layer(B, h, F);
+  void* gws = c.take(gws_b);
+  const size_t aws_b = decode_attention_ws_bytes(B, cache->n_heads, cache->head_dim, cache->capacity);
+  void* aws = c.take(aws_b);
+  auto* qkvh = reinterpret_cast<__half*>(qkv);
+
+  FG_TRY(layernorm_impl(x_in, B, h, layer->ln1_g, layer->ln1_b, h1, s));
+  FG_TRY(qlinear_run(h1, B, layer->qkv, nullptr, 0, qkv, gws, gws_b, s));
+  FG_TRY(kv_append_impl(cache, qkvh + h, qkvh + 2 * h, 3 * int64_t(h), 1, s));
+  FG_TRY(decode_attention_impl(qkv, 3 * int64_t(h), cache, att, aws, aws_b, s));
+  FG_TRY(qlinear_run(att, B, layer->out, x_in, 0, x1, gws, gws_b, s));
+  FG_TRY(layernorm_impl(x1, B, h, layer->ln2_g, layer->ln2_b, h2, s));
+  FG_TRY(qlinear_run(h2, B, layer->fc1, nullptr, 1, f, gws, gws_b, s));
+  FG_TRY(qlinear_run(f, B, layer->fc2, x1, 0, x_out, gws, gws_b, s));
+  return FG_OK;
+}
+
+int prefill_layer_impl(const fg_layer* layer, fg_kv_cache* cache, void* x, int B, int L, void* ws, size_t ws_bytes,
+                       cudaStream_t s) {
+  if (!cache || !x) return fail(FG_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || L <= 0 || B != cache->B) return fail(FG_ERR_SHAPE, "B must equal the cache batch and L > 0");
+  if (cache->len != 0) return fail(FG_ERR_INVALID_ARG, "prefill needs an empty cache (len 0)");
+  if (L > cache->capacity) return fail(FG_ERR_CAPACITY, "prompt longer than the cache capacity");
+  const int h = cache->n_heads * cache->head_dim;
+  int F = 0;
+  FG_TRY(check_layer(layer, h, &F));
+  const size_t need = prefill_ws(h, F, B, L);
+  if (!ws || ws_bytes < need) return fail(FG_ERR_WORKSPACE, "prefill layer needs %zu workspace bytes", need);
+  const int64_t BL = int64_t(B) * L;
+  Carver c(ws, ws_bytes);
+  void* hn = c.take(size_t(BL) * h * 2);
+  void* att = c.take(size_t(BL) * h * 2);
+  void* x1 = c.take(size_t(BL) * h * 2);
+  void* qkv = c.take(size_t(BL) * 3 * h * 2);
+  void* f = c.take(size_t(BL) * F * 2);
+  const size_t gws_b = gemm_ws_for_layer(BL, h, F);
+  void* gws = c.take(gws_b);
+  auto* qkvh = reinterpret_cast<__half*>(qkv);
+
+  FG_TRY(layernorm_impl(x, BL, h, layer->ln1_g, layer->ln1_b, hn, s));
+  FG_TRY(qlinear_run(hn, BL, layer->qkv, nullptr, 0, qkv, gws, gws_b, s));
+  FG_TRY(kv_append_impl(cache, qkvh + h, qkvh + 2 * h, 3 * int64_t(h), L, s));
+  FG_TRY(prefill_attention_impl(qkv, B, L, cache->n_heads, cache->head_dim, att, s));
+  FG_TRY(qlinear_run(att, BL, layer->out, x, 0, x1, gws, gws_b, s));
+  FG_TRY(layernorm_impl(x1, BL, h, layer->ln2_g, layer->ln2_b, hn, s));
+  FG_TRY(qlinear_run(hn, BL, layer->fc1, nullptr, 1, f, gws, gws_b, s));
+  FG_TRY(qlinear_run(f, BL, layer->fc2, x1, 0, x, gws, gws_b, s));
+  return FG_OK;
+}
+
+namespace {
+size_t lm_ws(int B, int V) { return align256(size_t(B) * V * 4) + 256; }
+
+int lm_head_impl(const void* x, int B, int hidden, const void* E, int V, float* logits, int32_t* tokens,
+                 int64_t tok_stride, void* ws, size_t wsb, cudaStream_t s) {
+  if (!x || !E || !tokens) return fail(FG_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || V <= 0 || hidden <= 0 || hidden % 64) return fail(FG_ERR_SHAPE, "bad LM head shape");
+  float* lg = logits;
+  if (!lg) {
+    if (!ws || wsb < lm_ws(B, V)) return fail(FG_ERR_WORKSPACE, "LM head needs %zu workspace bytes", lm_ws(B, V));
+    lg = reinterpret_cast<float*>(ws);
+  }
+  if (!aligned16(lg)) return fail(FG_ERR_ALIGN, "logits must be 16-byte aligned");
+  FG_TRY(gemm_impl(2, x, B, V, hidden, E, nullptr, 0, nullptr, nullptr, 0, lg, true, nullptr, 0, s));
+  return argmax_impl(lg, B, V, tokens, tok_stride, s);
+}
+
+size_t generate_ws(const fg_model* m, int B, int L, int T) {
+  const int h = m->hidden, F = m->ffn;
+  size_t t = 0;
+  t += align256(size_t(B) * L * h * 2);                 // x (prompt hidden states)
+  t += align256(size_t(B) * h * 2) * 2;                 // decode x, final LN out
+  size_t layer = std::max(prefill_ws(h, F, B, L), decode_ws(h, F, m->n_heads, B, L + T));
+  t += align256(layer);
+  t += lm_ws(B, m->vocab);
+  return t + 256;
+}
+}  // namespace
+
+int generate_impl(const fg_model* m, const int32_t* ids, int B, int L, int T, int32_t* out, fg_kv_cache* caches,
+                  void* ws, size_t wsb, fg_timing* timing, cudaStream_t s) {
+  if (!m || !ids || !out || !caches) return fail(FG_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || L <= 0 || T <= 0) return fail(FG_ERR_SHAPE, "B, L and gen_len must be positive");
+  if (!m->embed || !m->pos_embed || !m->lnf_g || !m->lnf_b || !m->layers)
+    return fail(FG_ERR_INVALID_ARG, "model tensors not set");
+  if (m->hidden != m->n_heads * m->head_dim) return fail(FG_ERR_SHAPE, "hidden != n_heads * head_dim");
+  if (L + T - 1 > m->max_pos) return fail(FG_ERR_SHAPE, "L + gen_len - 1 exceeds max_pos");
+  const int h = m->hidden;
+  for (int l = 0; l < m->n_layers; ++l) {
+    fg_kv_cache& c = caches[l];
+    if (c.B != B || c.n_heads != m->n_heads || c.head_dim != m->head_dim)
+      return fail(FG_ERR_SHAPE, "cache %d shape does not match the model", l);
+    if (c.capacity < L + T) return fail(FG_ERR_CAPACITY, "cache %d capacity %d < L + gen_len", l, c.capacity);
+  }
+  const size_t need = generate_ws(m, B, L, T);
+  if (!ws || wsb < need) return fail(FG_ERR_WORKSPACE, "generate needs %zu workspace bytes", need);
+  Carver c(ws, wsb);
+  void* x = c.take(size_t(B) * L * h * 2);
+  void* xd = c.take(size_t(B) * h * 2);
+  void* xn = c.take(size_t(B) * h * 2);
+  const size_t layer_b = std::max(prefill_ws(h, m->ffn, B, L), decode_ws(h, m->ffn, m->n_heads, B, L + T));
+  void* lws = c.take(layer_b);
+  void* lgw = c.take(lm_ws(B, m->vocab));
+
+  cudaEvent_t e0, e1, e2;
+  FG_CHECK_CUDA(cudaEventCreate(&e0));
+  FG_CHECK_CUDA(cudaEventCreate(&e1));
+  FG_CHECK_CUDA(cudaEventCreate(&e2));
+  int st = FG_OK;
+  do {
+    for (int l = 0; l < m->n_layers; ++l) caches[l].len = 0;
+    if ((st = cudaEventRecord(e0, s)) != cudaSuccess) { st = cuda_fail(cudaError_t(st), "event"); break; }
+    if ((st = embed_impl(ids, B, L, L, 0, m->embed, m->pos_embed, h, x, s)) != FG_OK) break;
+    for (int l = 0; l < m->n_layers && st == FG_OK; ++l)
+      st = prefill_layer_impl(&m->layers[l], &caches[l], x, B, L, lws, layer_b, s);
+    if (st != FG_OK) break;
+    // hidden state of each sequence's last prompt position
+    if (cudaMemcpy2DAsync(xd, size_t(h) * 2, reinterpret_cast<uint8_t*>(x) + size_t(L - 1) * h * 2,
+                          size_t(L) * h * 2, size_t(h) * 2, B, cudaMemcpyDeviceToDevice, s) != cudaSuccess) {
+      st = cuda_fail(cudaGetLastError(), "gather last positions");
+      break;
+    }
+    if ((st = layernorm_impl(xd, B, h, m->lnf_g, m->lnf_b, xn, s)) != FG_OK) break;
+    if ((st = lm_head_impl(xn, B, h, m->embed, m->vocab, nullptr, out, T, lgw, lm_ws(B, m->vocab), s)) != FG_OK) break;
+    cudaEventRecord(e1, s);
+    for (int j = 1; j < T && st == FG_OK; ++j) {
+      // token j-1 sits at position L + j - 1
+      st = embed_impl(out + (j - 1), B, 1, T, L + j - 1, m->embed, m->pos_embed, h, xd, s);
+      for (int l = 0; l < m->n_layers && st == FG_OK; ++l)
+        st = decode_layer_impl(&m->layers[l], &caches[l], xd, xd, B, lws, layer_b, s);
+      if (st == FG_OK) st = layernorm_impl(xd, B, h, m->lnf_g, m->lnf_b, xn, s);
+      if (st == FG_OK) st = lm_head_impl(xn, B, h, m->embed, m->vocab, nullptr, out + j, T, lgw, lm_ws(B, m->vocab), s);
+    }
+    if (st != FG_OK) break;
+    cudaEventRecord(e2, s);
+    cudaError_t ce = cudaEventSynchronize(e2);
+    if (ce != cudaSuccess) { st = cuda_fail(ce, "generate"); break; }
+    int derr = 0;
+    if (read_device_error(&derr) == FG_OK && derr != 0) {
+      st = fail(FG_ERR_CUDA, "a device-side wait timed out (code %d)", derr);
+      break;
+    }
+    float pm = 0.f, dm = 0.f;
+    cudaEventElapsedTime(&pm, e0, e1);
+    cudaEventElapsedTime(&dm, e1, e2);
+    if (timing) {
+      timing->prefill_ms = pm;
+      timing->decode_ms = dm;
+      timing->tokens = int64_t(B) * T;
+      timing->tok_per_s = double(B) * T / ((double(pm) + double(dm)) * 1e-3);
+    }
+  } while (false);
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  cudaEventDestroy(e2);
+  return st;
+}
+
+}  // namespace fg
+
+// ==================================================================== extern "C"
+using namespace fg;
+
+extern "C" {
+
+const char* fg_status_string(int status) {
+  switch (status) {
+    case FG_OK: return "ok";
+    case FG_ERR_INVALID_ARG: return "invalid argument";
+    case FG_ERR_SHAPE: return "shape error";
+    case FG_ERR_ALIGN: return "alignment error";
+    case FG_ERR_CAPACITY: return "KV cache capacity exceeded";
+    case FG_ERR_CUDA: return "CUDA error";
+    case FG_ERR_UNSUPPORTED: return "unsupported configuration";
+    case FG_ERR_WORKSPACE: return "workspace too small";
+    default: return "unknown status";
+  }
+}
+
+const char* fg_last_error(void) { return g_err; }
+int fg_version(void) { return 100; }
+
+int fg_quantize_pack(const void* x, int64_t rows, int64_t cols, int group, int axis, uint8_t* codes, void* params,
+                     void* stream) {
+  return quantize_pack_impl(x, rows, cols, group, axis, codes, params, as_stream(stream));
+}
+
+int fg_dequantize(const uint8_t* codes, const void* params, int64_t rows, int64_t cols, int group, int axis,
+                  void* out, void* stream) {
+  return dequantize_impl(codes, params, rows, cols, group, axis, out, as_stream(stream));
+}
+
+int fg_kv_append(fg_kv_cache* cache, const void* k, const void* v, int64_t row_stride, int n_tokens, void* stream) {
+  return kv_append_impl(cache, k, v, row_stride, n_tokens, as_stream(stream));
+}
+
+size_t fg_qgemm_workspace_bytes(int64_t M, int N, int K) { return qgemm_ws_bytes(M, N, K); }
+
+int fg_qgemm(const void* X, int64_t M, const fg_qlinear* W, const void* R, int relu, void* Y, void* workspace,
+             size_t ws_bytes, void* stream) {
+  if (!W) return fail(FG_ERR_INVALID_ARG, "null weight");
+  return qlinear_run(X, M, *W, R, relu, Y, workspace, ws_bytes, as_stream(stream));
+}
+
+size_t fg_decode_attention_workspace_bytes(int B, int n_heads, int head_dim, int ctx) {
+  return decode_attention_ws_bytes(B, n_heads, head_dim, ctx);
+}
+
+int fg_decode_attention(const void* q, int64_t q_stride, const fg_kv_cache* cache, void* out, void* workspace,
+                        size_t ws_bytes, void* stream) {
+  return decode_attention_impl(q, q_stride, cache, out, workspace, ws_bytes, as_stream(stream));
+}
+
+int fg_prefill_attention(const void* qkv, int B, int L, int n_heads, int head_dim, void* out, void* stream) {
+  return prefill_attention_impl(qkv, B, L, n_heads, head_dim, out, as_stream(stream));
+}
+
+int fg_layernorm(const void* x, int64_t rows, int cols, const void* g, const void* b, void* y, void* stream) {
+  return layernorm_impl(x, rows, cols, g, b, y, as_stream(stream));
+}
+
+int fg_embed(const int32_t* ids, int B, int T, int pos0, const void* E, const void* P, int hidden, void* out,
+             void* stream) {
+  return embed_impl(ids, B, T, T, pos0, E, P, hidden, out, as_stream(stream));
+}
+
+size_t fg_lm_head_workspace_bytes(int B, int vocab) { return lm_ws(B, vocab); }
+
+int fg_lm_head_argmax(const void* x, int B, int hidden, const void* E, int vocab, float* logits, int32_t* tokens,
+                      void* workspace, size_t ws_bytes, void* stream) {
+  return lm_head_impl(x, B, hidden, E, vocab, logits, tokens, 1, workspace, ws_bytes, as_stream(stream));
+}
+
+size_t fg_decode_layer_workspace_bytes(int hidden, int ffn, int n_heads, int B, int capacity) {
+  if (hidden <= 0 || ffn <= 0 || n_heads <= 0 || B <= 0 || capacity <= 0) return 0;
+  return decode_ws(hidden, ffn, n_heads, B, capacity);
+}
+
+int fg_decode_layer(const fg_layer* layer, fg_kv_cache* cache, const void* x_in, void* x_out, int B, void* workspace,
+                    size_t ws_bytes, void* stream) {
+  return decode_layer_impl(layer, cache, x_in, x_out, B, workspace, ws_bytes, as_stream(stream));
+}
+
+size_t fg_prefill_layer_workspace_bytes(int hidden, int ffn, int B, int L) {
+  if (hidden <= 0 || ffn <= 0 || B <= 0 || L <= 0) return 0;
+  return prefill_ws(hidden, ffn, B, L);
+}
+
+int fg_prefill_layer(const fg_layer* layer, fg_kv_cache* cache, void* x, int B, int L, void* workspace,
+                     size_t ws_bytes, void* stream) {
+  return prefill_layer_impl(layer, cache, x, B, L, workspace, ws_bytes, as_stream(stream));
+}
+
+size_t fg_workspace_bytes(const fg_model* model, int B, int L, int gen_len) {
+  if (!model || B <= 0 || L <= 0 || gen_len <= 0) return 0;
+  return generate_ws(model, B, L, gen_len);
+}
+
+int fg_generate(const fg_model* model, const int32_t* prompt_ids, int B, int L, int gen_len, int32_t* out_ids,
+                fg_kv_cache* caches, void* workspace, size_t ws_bytes, fg_timing* timing, void* stream) {
+  return generate_impl(model, prompt_ids, B, L, gen_len, out_ids, caches, workspace, ws_bytes, timing,
+                       as_stream(stream));
+}
+
+int fg_profile_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = on != 0;
+  return FG_OK;
+}
+
+int fg_profile_read(int kind, double* total_ms, int64_t* launches, double* flops, double* bytes) {
+  if (kind < 0 || kind >= PROF_NKINDS) return fail(FG_ERR_INVALID_ARG, "bad profile kind");
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  collect_locked();
+  if (total_ms) *total_ms = g_prof_ms[kind];
+  if (launches) *launches = g_prof_n[kind];
+  if (flops) *flops = g_prof_flops[kind];
+  if (bytes) *bytes = g_prof_bytes[kind];
+  return FG_OK;
+}
+
+int fg_profile_reset(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  collect_locked();
+  for (int i = 0; i < PROF_NKINDS; ++i) {
+    g_prof_ms[i] = 0;
+    g_prof_n[i] = 0;
+    g_prof_flops[i] = 0;
+    g_prof_bytes[i] = 0;
+  }
+  return FG_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,562 @@
+// K3: dequant-fused GEMM on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+//   Y[M][N] = [relu](X[M][K] * W_hat[K][N] + b) [+ R]
+//
+// The weights W ("FlexGen" README mirror, key features: parameters compressed to 4 bits)
+// are 4-bit codes [K][N/2] with {min, scale} fp16 pairs per group of G along N.  W_hat is
+// exactly fg_dequantize's fp16 value, so fp16 x fp16 products accumulated in fp32 are the
+// contraction the layer defines.
+//
+// Structure (one CTA per SM, persistent over output tiles of 128 x 256):
+//   warp 0      TMA producer: X tile [128 x 64] (128-byte swizzle, K-major) and the code
+//               tile [64 x 128 B] + param tile [64 x PB] of the k-block into a stage.
+//   warp 1      MMA issuer: 4 x tcgen05.mma (M128 N256 K16) per k-block into one of two
+//               TMEM accumulators (2 x 256 fp32 columns); tcgen05.commit frees the stage.
+//   warps 4-7   epilogue: tcgen05.ld rows of the finished accumulator, bias / ReLU /
+//               residual, fp16 (or fp32) stores; frees the accumulator for tile i+2.
+//   warps 8-15  dequant (4-bit mode): expand the stage's codes to fp16 directly into
+//               the MN-major 128-byte-swizzled operand layout the MMA reads.
+// Other operand modes reuse the skeleton: B as a ready fp16 [K][N] tensor (MN-major, by
+// TMA) or as an fp16 [N][K] tensor (K-major by TMA, the tied LM head).  Tiles are
+// rasterized in bands of 16 M-tiles so a band of X stays in L2 while weights stream.
+// With few tiles (decode batches) the K loop is split and fp32 partials are reduced by a
+// second kernel that applies the epilogue.
+#include <algorithm>
+#include <cstring>
+#include <cudaTypedefs.h>
+
+#include "fg_common.cuh"
+#include "sm100.cuh"
+
+namespace fg {
+
+__device__ int g_device_error = 0;  // set by bounded waits that gave up (host-readable)
+
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int kBand = 16;
+constexpr int kABytes = BM * BK * 2;   // 16 KB
+constexpr int kBBytes = BN * BK * 2;   // 32 KB
+constexpr int kCodeBytes = BK * BN / 2; // 8 KB
+constexpr int kParamBytesMax = BK * 8 * 4;  // up to 8 half2 per k row (G = 32)
+
+enum BMode { B_Q4 = 0, B_F16_MN = 1, B_F16_K = 2 };
+
+template <int MODE>
+struct Cfg {
+  static constexpr int kStages = MODE == B_Q4 ? 3 : 4;
+  static constexpr int kStageBytes = kABytes + kBBytes + (MODE == B_Q4 ? kCodeBytes + kParamBytesMax : 0);
+  static constexpr int kDequantWarps = MODE == B_Q4 ? 8 : 0;
+  static constexpr int kThreads = 256 + kDequantWarps * 32;
+  static constexpr int kSmem = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+struct GemmArgs {
+  int M, N, K;
+  int m_tiles, n_tiles, k_blocks, splits;
+  int total;        // m_tiles * n_tiles * splits
+  int G, PB;        // group size, params per k row in a stage
+  const __half* bias;
+  const __half* R;
+  int relu;
+  void* Y;          // fp16 or fp32 [M][N]
+  float* partial;   // [splits][M][N] when splits > 1
+};
+
+struct TileCoord {
+  int m0, n0, kb0, kb1, ks;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t) {
+  TileCoord c;
+  c.ks = t % a.splits;
+  const int r = t / a.splits;
+  const int band_tiles = kBand * a.n_tiles;
+  const int bi = r / band_tiles;
+  const int rr = r - bi * band_tiles;
+  const int mt_in_band = min(kBand, a.m_tiles - bi * kBand);
+  const int n = rr / mt_in_band;
+  const int m = bi * kBand + (rr - n * mt_in_band);
+  c.m0 = m * BM;
+  c.n0 = n * BN;
+  c.kb0 = int((int64_t(c.ks) * a.k_blocks) / a.splits);
+  c.kb1 = int((int64_t(c.ks + 1) * a.k_blocks) / a.splits);
+  return c;
+}
+
+template <int MODE, bool OUT_F32>
+__global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                   const __grid_constant__ CUtensorMap tm_p, const GemmArgs args) {
+  using C = Cfg<MODE>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t base_u32 = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024 - (base_u32 & 1023)) & 1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint64_t* full = bars;              // [S] TMA landed
+  uint64_t* bfull = bars + S;         // [S] dequant wrote B (4-bit mode)
+  uint64_t* empty = bars + 2 * S;     // [S] MMA finished reading the stage
+  uint64_t* acc_full = bars + 3 * S;  // [2]
+  uint64_t* acc_empty = bars + 3 * S + 2;  // [2]
+  uint64_t* drain = bars + 3 * S + 4;      // [1] MMA drain on abort
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 3 * S + 6);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&bfull[i], C::kDequantWarps > 0 ? C::kDequantWarps : 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_b);
+    if (MODE == B_Q4) prefetch_tmap(&tm_p);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t tx = kABytes + (MODE == B_Q4 ? (kCodeBytes + BK * args.PB * 4) : kBBytes);
+      bool ok = true;
+      bool pend[S];
+      uint32_t pend_phase[S];
+#pragma unroll
+      for (int i = 0; i < S; ++i) { pend[i] = false; pend_phase[i] = 0; }
+      for (int t = blockIdx.x; t < args.total && ok; t += gridDim.x) {
+        const TileCoord c = tile_coord(args, t);
+        for (int kb = c.kb0; kb < c.kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, &g_device_error, 1)) { ok = false; break; }
+          uint8_t* st = smem + stage * C::kStageBytes;
+          mbar_expect_tx(&full[stage], tx);
+          tma_load_2d(st, &tm_a, kb * BK, c.m0, &full[stage]);
+          if (MODE == B_Q4) {
+            tma_load_2d(st + kABytes + kBBytes, &tm_b, c.n0 / 2, kb * BK, &full[stage]);
+            const int px = (c.n0 / args.G) & ~3;
+            tma_load_2d(st + kABytes + kBBytes + kCodeBytes, &tm_p, px, kb * BK, &full[stage]);
+          } else if (MODE == B_F16_MN) {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d(st + kABytes + j * 8192, &tm_b, c.n0 + 64 * j, kb * BK, &full[stage]);
+          } else {
+            tma_load_2d(st + kABytes, &tm_b, kb * BK, c.n0, &full[stage]);
+          }
+          pend[stage] = true;
+          pend_phase[stage] = phase;
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (*abort_flag) {
+        // let every copy this thread issued land before the CTA exits
+        for (int i = 0; i < S; ++i)
+          if (pend[i]) mbar_wait_drain(&full[i], pend_phase[i]);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(BM, BN, MODE != B_F16_K);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < args.total && ok; t += gridDim.x) {
+        const TileCoord c = tile_coord(args, t);
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag, &g_device_error, 2)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
+        for (int kb = c.kb0; kb < c.kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, &g_device_error, 4)) { ok = false; break; }
+          if (MODE == B_Q4 && !mbar_wait(&bfull[stage], phase, abort_flag, &g_device_error, 8)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = smem_desc_sw128(a_addr + k * 32, 16, 1024);
+            uint64_t bd;
+            if (MODE == B_F16_K) bd = smem_desc_sw128(b_addr + k * 32, 16, 1024);
+            else bd = smem_desc_sw128(b_addr + k * 2048, 8192, 1024);
+            mma_f16_ss(d_tmem, ad, bd, idesc, (kb > c.kb0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+      if (*abort_flag) {
+        // wait for the MMAs already issued before TMEM is released
+        mma_commit(drain);
+        mbar_wait_drain(drain, 0);
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp - 4;  // TMEM lane quarter
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < args.total; t += gridDim.x) {
+      const TileCoord c = tile_coord(args, t);
+      if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, &g_device_error, 16)) break;
+      tc_fence_after();
+      const int m = c.m0 + q * 32 + lane;
+      const bool row_ok = m < args.M;
+      for (int cc = 0; cc < BN; cc += 32) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + cc), r);
+        tmem_ld_wait();
+        const int n = c.n0 + cc;
+        if (!row_ok || n >= args.N) continue;
+        if (args.partial != nullptr) {
+          float4* dst = reinterpret_cast<float4*>(args.partial + (int64_t(c.ks) * args.M + m) * args.N + n);
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                 __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+          continue;
+        }
+        if (OUT_F32) {
+          float* dst = reinterpret_cast<float*>(args.Y) + int64_t(m) * args.N + n;
+          if (n + 32 <= args.N) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              reinterpret_cast<float4*>(dst)[j] =
+                  make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                              __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+          } else {
+            for (int j = 0; j < 32 && n + j < args.N; ++j) dst[j] = __uint_as_float(r[j]);
+          }
+          continue;
+        }
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        if (args.bias != nullptr) {
+          const uint4* bp = reinterpret_cast<const uint4*>(args.bias + n);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 bw = __ldg(bp + j);
+            const __half2* bh = reinterpret_cast<const __half2*>(&bw);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __half22float2(bh[e]);
+              v[8 * j + 2 * e] += f.x;
+              v[8 * j + 2 * e + 1] += f.y;
+            }
+          }
+        }
+        if (args.relu) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.f);
+        }
+        if (args.R != nullptr) {
+          const uint4* rp = reinterpret_cast<const uint4*>(args.R + int64_t(m) * args.N + n);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 rw = __ldg(rp + j);
+            const __half2* rh = reinterpret_cast<const __half2*>(&rw);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __half22float2(rh[e]);
+              v[8 * j + 2 * e] += f.x;
+              v[8 * j + 2 * e + 1] += f.y;
+            }
+          }
+        }
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__half*>(args.Y) + int64_t(m) * args.N + n);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 o;
+          o.x = h2_as_u32(__floats2half2_rn(v[8 * j + 0], v[8 * j + 1]));
+          o.y = h2_as_u32(__floats2half2_rn(v[8 * j + 2], v[8 * j + 3]));
+          o.z = h2_as_u32(__floats2half2_rn(v[8 * j + 4], v[8 * j + 5]));
+          o.w = h2_as_u32(__floats2half2_rn(v[8 * j + 6], v[8 * j + 7]));
+          dst[j] = o;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  } else if (MODE == B_Q4 && warp >= 8) {
+    // ------------------------------------------------------------ dequant warps
+    const int dw = warp - 8;       // 0..7: k rows dw, dw+8, ..., dw+56
+    const int nb = lane >> 3;      // 64-wide MN block of the word
+    const int ch = lane & 7;       // 16-byte chunk inside the block
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < args.total && ok; t += gridDim.x) {
+      const TileCoord c = tile_coord(args, t);
+      const int poff = (c.n0 / args.G) & 3;
+      const int pcol = poff + (lane * 8) / args.G;
+      for (int kb = c.kb0; kb < c.kb1; ++kb) {
+        if (!mbar_wait(&full[stage], phase, abort_flag, &g_device_error, 32)) { ok = false; break; }
+        uint8_t* st = smem + stage * C::kStageBytes;
+        const uint32_t* codes = reinterpret_cast<const uint32_t*>(st + kABytes + kBBytes);
+        const uint32_t* prm = reinterpret_cast<const uint32_t*>(st + kABytes + kBBytes + kCodeBytes);
+        uint8_t* bt = st + kABytes;
+        uint32_t w[8], p[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int row = dw + 8 * i;
+          w[i] = codes[row * (BN / 8) + lane];
+          p[i] = prm[row * args.PB + pcol];
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int row = dw + 8 * i;  // k index inside the block
+          const __half2 pr = u32_as_h2(p[i]);
+          uint32_t o[4];
+          dequant8(w[i], __high2half2(pr), __low2half2(pr), o);
+          const int kg = row >> 3, rr = row & 7;
+          uint4* dst = reinterpret_cast<uint4*>(bt + nb * 8192 + kg * 1024 + rr * 128 + ((ch ^ rr) << 4));
+          *dst = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bfull[stage]);
+        if (++stage == S) { stage = 0; phase ^= 1; }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// Split-K reduction + epilogue: Y = [relu](sum_s P[s] + b) [+ R], 8 columns per thread.
+__global__ void splitk_reduce_kernel(const float* __restrict__ P, int splits, int64_t MN, int N,
+                                     const __half* __restrict__ bias, const __half* __restrict__ R,
+                                     int relu, __half* __restrict__ Y) {
+  const int64_t n8 = MN / 8;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += int64_t(gridDim.x) * blockDim.x) {
+    float v[8];
+    const float4* p0 = reinterpret_cast<const float4*>(P) + i * 2;
+    float4 a = p0[0], b = p0[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    for (int s = 1; s < splits; ++s) {
+      const float4* ps = reinterpret_cast<const float4*>(P + s * MN) + i * 2;
+      a = ps[0];
+      b = ps[1];
+      v[0] += a.x; v[1] += a.y; v[2] += a.z; v[3] += a.w; v[4] += b.x; v[5] += b.y; v[6] += b.z; v[7] += b.w;
+    }
+    const int n = int((i * 8) % N);
+    if (bias) {
+      const uint4 bw = __ldg(reinterpret_cast<const uint4*>(bias + n));
+      const __half2* bh = reinterpret_cast<const __half2*>(&bw);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(bh[e]);
+        v[2 * e] += f.x;
+        v[2 * e + 1] += f.y;
+      }
+    }
+    if (relu) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = fmaxf(v[j], 0.f);
+    }
+    if (R) {
+      const uint4 rw = __ldg(reinterpret_cast<const uint4*>(R) + i);
+      const __half2* rh = reinterpret_cast<const __half2*>(&rw);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(rh[e]);
+        v[2 * e] += f.x;
+        v[2 * e + 1] += f.y;
+      }
+    }
+    uint4 o;
+    o.x = h2_as_u32(__floats2half2_rn(v[0], v[1]));
+    o.y = h2_as_u32(__floats2half2_rn(v[2], v[3]));
+    o.z = h2_as_u32(__floats2half2_rn(v[4], v[5]));
+    o.w = h2_as_u32(__floats2half2_rn(v[6], v[7]));
+    reinterpret_cast<uint4*>(Y)[i] = o;
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+int make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t inner,
+                uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (!fn) return fail(FG_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  (void)elem_bytes;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return FG_OK;
+}
+
+template <int MODE, bool F32>
+int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& p, const GemmArgs& args, cudaStream_t s) {
+  using C = Cfg<MODE>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    FG_CHECK_CUDA(cudaFuncSetAttribute(gemm_tc_kernel<MODE, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem));
+    attr_set = true;
+  }
+  const int grid = std::min(args.total, num_sms());
+  gemm_tc_kernel<MODE, F32><<<grid, C::kThreads, C::kSmem, s>>>(a, b, p, args);
+  FG_CHECK_LAUNCH("tcgen05 gemm kernel");
+  return FG_OK;
+}
+
+int pick_splits(int tiles, int k_blocks) {
+  const int sms = num_sms();
+  if (tiles >= sms / 2) return 1;
+  int sp = sms / tiles;
+  sp = std::min(sp, k_blocks / 2);
+  return std::max(sp, 1);
+}
+
+}  // namespace
+
+int read_device_error(int* out) {
+  return cudaMemcpyFromSymbol(out, g_device_error, sizeof(int)) == cudaSuccess ? FG_OK : FG_ERR_CUDA;
+}
+
+size_t qgemm_ws_bytes(int64_t M, int N, int K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  const int m_tiles = int((M + BM - 1) / BM);
+  const int n_tiles = (N + BN - 1) / BN;
+  const int sp = pick_splits(m_tiles * n_tiles, K / BK);
+  if (sp <= 1) return 0;
+  return size_t(sp) * size_t(M) * size_t(N) * sizeof(float);
+}
+
+// mode: 0 = 4-bit weight W (codes/params), 1 = fp16 [K][N] weight, 2 = fp16 [N][K] weight.
+int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, const void* wparams, int G,
+              const void* bias, const void* R, int relu, void* Y, bool out_f32, void* ws, size_t ws_bytes,
+              cudaStream_t s) {
+  if (!X || !w || !Y) return fail(FG_ERR_INVALID_ARG, "null pointer");
+  if (M < 0 || N <= 0 || K <= 0) return fail(FG_ERR_SHAPE, "bad GEMM shape");
+  if (K % BK) return fail(FG_ERR_SHAPE, "K must be a multiple of 64");
+  if (M > 0x7fffff00LL) return fail(FG_ERR_SHAPE, "M too large");
+  if (mode == B_Q4) {
+    if (!wparams) return fail(FG_ERR_INVALID_ARG, "null params");
+    if (G != 32 && G != 64 && G != 128) return fail(FG_ERR_SHAPE, "group must be 32, 64 or 128");
+    if (N % BN) return fail(FG_ERR_SHAPE, "N must be a multiple of 256");
+    if (N % (4 * G)) return fail(FG_ERR_SHAPE, "N must be a multiple of 4*group");
+  } else if (mode == B_F16_MN) {
+    if (N % BN) return fail(FG_ERR_SHAPE, "N must be a multiple of 256");
+  } else if (N % 8) {
+    return fail(FG_ERR_SHAPE, "N must be a multiple of 8");
+  }
+  if (!out_f32 && N % 8) return fail(FG_ERR_SHAPE, "N must be a multiple of 8");
+  if (!aligned16(X) || !aligned16(w) || !aligned16(Y) || (wparams && !aligned16(wparams)) ||
+      (bias && !aligned16(bias)) || (R && !aligned16(R)))
+    return fail(FG_ERR_ALIGN, "pointers must be 16-byte aligned");
+  if (M == 0) return FG_OK;
+
+  GemmArgs a{};
+  a.M = int(M);
+  a.N = N;
+  a.K = K;
+  a.m_tiles = int((M + BM - 1) / BM);
+  a.n_tiles = (N + BN - 1) / BN;
+  a.k_blocks = K / BK;
+  a.splits = out_f32 ? 1 : pick_splits(a.m_tiles * a.n_tiles, a.k_blocks);
+  a.total = a.m_tiles * a.n_tiles * a.splits;
+  a.G = G;
+  a.PB = G == 32 ? 8 : 4;
+  a.bias = reinterpret_cast<const __half*>(bias);
+  a.R = reinterpret_cast<const __half*>(R);
+  a.relu = relu;
+  a.Y = Y;
+  a.partial = nullptr;
+  if (a.splits > 1) {
+    const size_t need = size_t(a.splits) * size_t(M) * size_t(N) * sizeof(float);
+    if (!ws || ws_bytes < need) return fail(FG_ERR_WORKSPACE, "GEMM split-K needs %zu workspace bytes", need);
+    if (!aligned16(ws)) return fail(FG_ERR_ALIGN, "workspace must be 16-byte aligned");
+    a.partial = reinterpret_cast<float*>(ws);
+  }
+
+  CUtensorMap ta, tb, tp;
+  memset(&tp, 0, sizeof(tp));
+  FG_TRY(make_map_2d(&ta, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, uint64_t(K), uint64_t(M), uint64_t(K) * 2, BK, BM,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
+  if (mode == B_Q4) {
+    FG_TRY(make_map_2d(&tb, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(N / 2), uint64_t(K), uint64_t(N / 2),
+                       BN / 2, BK, CU_TENSOR_MAP_SWIZZLE_NONE));
+    FG_TRY(make_map_2d(&tp, wparams, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, uint64_t(N / G), uint64_t(K),
+                       uint64_t(N / G) * 4, uint32_t(a.PB), BK, CU_TENSOR_MAP_SWIZZLE_NONE));
+  } else if (mode == B_F16_MN) {
+    FG_TRY(make_map_2d(&tb, w, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, uint64_t(N), uint64_t(K), uint64_t(N) * 2, 64, BK,
+                       CU_TENSOR_MAP_SWIZZLE_128B));
+  } else {
+    FG_TRY(make_map_2d(&tb, w, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, uint64_t(K), uint64_t(N), uint64_t(K) * 2, BK, BN,
+                       CU_TENSOR_MAP_SWIZZLE_128B));
+  }
+  if (mode != B_Q4) tp = tb;
+
+  const double flops = 2.0 * double(M) * N * K;
+  const double bytes = (mode == B_Q4 ? double(N) * K * (0.5 + 4.0 / G) : double(N) * K * 2.0) +
+                       double(M) * K * 2.0 + double(M) * N * (out_f32 ? 4.0 : 2.0) + (R ? double(M) * N * 2.0 : 0.0);
+  {
+    ProfScope ps(PROF_GEMM, s, flops, bytes);
+    int st;
+    if (mode == B_Q4) st = launch<B_Q4, false>(ta, tb, tp, a, s);
+    else if (mode == B_F16_MN) st = launch<B_F16_MN, false>(ta, tb, tp, a, s);
+    else st = out_f32 ? launch<B_F16_K, true>(ta, tb, tp, a, s) : launch<B_F16_K, false>(ta, tb, tp, a, s);
+    if (st != FG_OK) return st;
+  }
+  if (a.splits > 1) {
+    const int64_t MN = M * N;
+    const int grid = int(std::min<int64_t>((MN / 8 + 255) / 256, int64_t(num_sms()) * 8));
+    splitk_reduce_kernel<<<grid, 256, 0, s>>>(a.partial, a.splits, MN, N, a.bias, a.R, relu,
+                                              reinterpret_cast<__half*>(Y));
+    FG_CHECK_LAUNCH("split-K reduce kernel");
+  }
+  return FG_OK;
+}
+
+}  // namespace fg

@@ -266,7 +266,6 @@ int grid_for(int64_t units, int64_t per_block) {
 
 int check_qargs(const void* a, const void* b, const void* c, int64_t rows, int64_t cols, int group,
                 int axis) {
-  if (!a || !b || !c) return fail(FG_ERR_INVALID_ARG, "null pointer");
   if (rows < 0 || cols < 0) return fail(FG_ERR_SHAPE, "negative size");
   if (group != 32 && group != 64 && group != 128)
     return fail(FG_ERR_SHAPE, "group must be 32, 64 or 128 (got %d)", group);
@@ -276,6 +275,8 @@ int check_qargs(const void* a, const void* b, const void* c, int64_t rows, int64
   if (axis == 0 && rows % group) return fail(FG_ERR_SHAPE, "rows %% group != 0");
   if (rows > 0 && cols > 0 && rows > (int64_t(1) << 34) / cols)
     return fail(FG_ERR_SHAPE, "tensor larger than 2^34 elements");
+  if (rows == 0 || cols == 0) return FG_OK;  // nothing to touch: pointers may be null
+  if (!a || !b || !c) return fail(FG_ERR_INVALID_ARG, "null pointer");
   if (!aligned16(a) || !aligned16(b) || !aligned16(c)) return fail(FG_ERR_ALIGN, "pointers must be 16-byte aligned");
   return FG_OK;
 }

@@ -20,7 +20,7 @@ Distributions (all exact integer work followed by IEEE-rounded float64 operation
   mean 0, variance 1); value = fp16(z * sigma), one round-to-nearest-even.
 * uniform(lo, hi): u = (bits >> 11) * 2**-53; value = fp16(lo + (hi-lo)*u).
 * t3: z0..z3 are normals at element indices 4i..4i+3; chi = z1^2+z2^2+z3^2;
-  value = fp16(z0 / sqrt(chi/3)) (0 when chi == 0).
+  value = fp16(clip(scale * z0 / sqrt(chi/3), -65504, 65504)) (0 when chi == 0).
 * outlier columns: a 2-D [rows, cols] normal(1) tensor whose column j is multiplied by
   50 when ``bits(seed, stream ^ OUTLIER_TAG, j) >> 40`` is divisible by 100 (about 1 %).
 * token ids: ``(bits >> 32) % vocab``.
@@ -107,7 +107,7 @@ def values(seed: int, stream: int, idx, dist: str = "normal", scale: float = 1.0
         den = np.sqrt(chi / 3.0)
         with np.errstate(divide="ignore", invalid="ignore"):
             v = np.where(chi == 0.0, 0.0, z0 / np.where(den == 0.0, 1.0, den))
-        v = v * np.float64(scale)
+        v = np.clip(v * np.float64(scale), -65504.0, 65504.0)   # keep every value finite in fp16
     elif dist == "outlier":
         if cols <= 0:
             raise ValueError("outlier distribution needs cols > 0")

@@ -1,0 +1,98 @@
+"""GPU parity of decode attention over the 4-bit cache (K4 + split combine) and of the
+causal prefill attention (K5) against the oracle; tolerance max|err| <= 1e-2 * RMS."""
+import numpy as np
+import pytest
+
+import fg_synth
+import oracle
+from gpu_util import assert_close_rms, to_dev, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fg():
+    import torch
+    assert torch.cuda.is_available()
+    import bit_group_quantized_fg_b200 as m
+    m.lib()
+    return m
+
+
+def _build(fg, B, nh, hd, g, S, seed, dist="normal"):
+    """Cache filled by the GPU append from seeded K/V; the oracle cache from the same values."""
+    import torch
+    h = nh * hd
+    k = fg_synth.tensor(seed, 1, (B, S, h), dist, 1.0)
+    v = fg_synth.tensor(seed, 2, (B, S, h), dist, 1.0)
+    q = fg_synth.tensor(seed, 3, (B, 3 * h), "normal", 1.0)   # q in the first h columns (QKV row)
+    cache = fg.DeviceKVCache(B, nh, hd, S + 3, g)
+    fg.fg_kv_append(cache, to_dev(k.reshape(B * S, h)), to_dev(v.reshape(B * S, h)), h, S)
+    ref = oracle.KVCache(B, nh, hd, g, S + 3)
+    oracle.kv_append(ref, k, v, 0)
+    ref.length = S
+    torch.cuda.synchronize()
+    return q, cache, ref
+
+
+@pytest.mark.parametrize("B,nh,hd,g,S", [
+    (4, 12, 64, 64, 36),      # config-1 shape (h 768), a few positions
+    (2, 4, 128, 64, 1),       # a single position: output = V
+    (3, 2, 128, 32, 300),     # several groups per head
+    (2, 3, 128, 128, 77),
+    (1, 2, 64, 32, 5000),     # long context, few heads: split over many chunks
+    (1, 1, 128, 64, 8192),    # the sweep's longest context
+])
+def test_decode_attention_matches_oracle(fg, B, nh, hd, g, S):
+    q, cache, ref = _build(fg, B, nh, hd, g, S, seed=S + nh)
+    import torch
+    out = fg.fg_decode_attention(to_dev(q), 3 * nh * hd, cache)
+    torch.cuda.synchronize()
+    exp = oracle.decode_attention(q[:, :nh * hd], ref, S)
+    assert_close_rms(to_np(out), exp, what="decode attention")
+
+
+def test_decode_attention_t3_and_outliers(fg):
+    import torch
+    for dist in ("t3", "outlier"):
+        q, cache, ref = _build(fg, 2, 4, 128, 64, 129, seed=99, dist=dist)
+        out = fg.fg_decode_attention(to_dev(q), 3 * 512, cache)
+        torch.cuda.synchronize()
+        assert_close_rms(to_np(out), oracle.decode_attention(q[:, :512], ref, 129), what=dist)
+
+
+def test_decode_attention_sampled_full_size(fg):
+    """Config-2 decode shape (B 64, 32 heads x 128, context 543) with sampled (b, head)
+    pairs checked against the oracle; the rest checked for finiteness."""
+    import torch
+    B, nh, hd, g, S = 64, 32, 128, 64, 543
+    h = nh * hd
+    from fg_synth import gpu as sg
+    kv = torch.empty((B * S, 2 * h), dtype=torch.float16, device="cuda")
+    sg.fill(kv, 77, 1, "normal", 1.0)
+    q = torch.empty((B, 3 * h), dtype=torch.float16, device="cuda")
+    sg.fill(q, 77, 2, "normal", 1.0)
+    cache = fg.DeviceKVCache(B, nh, hd, S + 1, g)
+    fg.fg_kv_append(cache, kv, kv[:, h:], 2 * h, S)
+    out = fg.fg_decode_attention(q, 3 * h, cache)
+    torch.cuda.synchronize()
+    assert bool(torch.isfinite(out.float()).all())
+    qn = to_np(q)
+    for b in (0, 31, 63):
+        rows = fg_synth.values(77, 1, np.arange(b * S * 2 * h, (b + 1) * S * 2 * h), "normal", 1.0, 2 * h)
+        rows = rows.reshape(1, S, 2 * h)
+        ref = oracle.KVCache(1, nh, hd, g, S)
+        oracle.kv_append(ref, rows[:, :, :h], rows[:, :, h:], 0)
+        exp = oracle.decode_attention(qn[b:b + 1, :h], ref, S)
+        assert_close_rms(to_np(out[b:b + 1]), exp, what=f"row {b}")
+
+
+@pytest.mark.parametrize("B,L,nh,hd", [(4, 32, 12, 64), (2, 100, 2, 128), (1, 200, 3, 64), (2, 64, 1, 128)])
+def test_prefill_attention_matches_oracle(fg, B, L, nh, hd):
+    import torch
+    h = nh * hd
+    qkv = fg_synth.tensor(L, nh, (B, L, 3 * h), "normal", 1.0)
+    out = fg.fg_prefill_attention(to_dev(qkv.reshape(B * L, 3 * h)), B, L, nh, hd)
+    torch.cuda.synchronize()
+    exp = oracle.prefill_attention(qkv, nh, hd)
+    assert_close_rms(to_np(out).reshape(B, L, h), exp, what="prefill attention")

@@ -1,0 +1,107 @@
+"""GPU parity of the dequant-fused tcgen05 GEMM (K3) and the tied LM head against the
+oracle's float64 product of the same fp16 operands; tolerance max|err| <= 1e-2 * RMS."""
+import numpy as np
+import pytest
+
+import fg_synth
+import oracle
+from gpu_util import assert_close_rms, to_dev, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fg():
+    import torch
+    assert torch.cuda.is_available()
+    import bit_group_quantized_fg_b200 as m
+    m.lib()
+    return m
+
+
+def _case(fg, M, N, K, g, relu, resid, seed):
+    import torch
+    x = fg_synth.tensor(seed, 1, (M, K), "normal", 1.0)
+    w = fg_synth.tensor(seed, 2, (K, N), "normal", 0.02)
+    b = fg_synth.tensor(seed, 3, (N,), "normal", 0.5)
+    r = fg_synth.tensor(seed, 4, (M, N), "normal", 1.0) if resid else None
+    lin = fg.DeviceQLinear.from_fp16(to_dev(w), to_dev(b), g)
+    y = fg.fg_qgemm(to_dev(x), lin, R=None if r is None else to_dev(r), relu=relu)
+    torch.cuda.synchronize()
+    ref_lin = oracle.QLinear.from_fp16(w, b, g)
+    assert np.array_equal(to_np(lin.codes), ref_lin.codes)
+    exp = oracle.qlinear(x, ref_lin, relu=relu, residual16=r)
+    return to_np(y), exp
+
+
+@pytest.mark.parametrize("M,N,K,g,relu,resid", [
+    (4, 256, 64, 64, False, False),        # one k-block, tiny M
+    (4, 2304, 768, 64, False, False),      # config-1 QKV at decode
+    (128, 768, 768, 64, False, True),      # config-1 out-proj (prefill rows), residual
+    (128, 3072, 768, 64, True, False),     # config-1 fc1 + ReLU
+    (128, 768, 3072, 64, False, True),     # config-1 fc2 + residual
+    (300, 512, 320, 32, True, True),       # ragged M over 3 tiles, g 32
+    (64, 1024, 512, 128, False, False),    # g 128
+    (1000, 768, 256, 64, False, False),    # 8 M-tiles, band raster
+])
+def test_qgemm_matches_oracle(fg, M, N, K, g, relu, resid):
+    got, exp = _case(fg, M, N, K, g, relu, resid, seed=M + N + K)
+    assert_close_rms(got, exp, what="qgemm")
+
+
+def test_qgemm_decode_split_k(fg):
+    """M = 64 rows with few output tiles: the K loop is split and reduced."""
+    assert fg.fg_qgemm_workspace_bytes(64, 4096, 4096) > 0
+    got, exp = _case(fg, 64, 4096, 4096, 64, False, True, seed=7)
+    assert_close_rms(got, exp, what="split-K")
+
+
+def test_qgemm_prefill_size_sampled(fg):
+    """Config-2 prefill QKV shape (M 32768, N 12288, K 4096) on sampled outputs."""
+    import torch
+    from fg_synth import gpu as sg
+    M, N, K, g = 32768, 12288, 4096, 64
+    x = torch.empty((M, K), dtype=torch.float16, device="cuda")
+    sg.fill(x, 11, 1, "normal", 1.0)
+    w = torch.empty((K, N), dtype=torch.float16, device="cuda")
+    sg.fill(w, 11, 2, "normal", 0.02)
+    b = torch.empty((N,), dtype=torch.float16, device="cuda")
+    sg.fill(b, 11, 3, "normal", 0.5)
+    lin = fg.DeviceQLinear.from_fp16(w, b, g)
+    del w
+    y = fg.fg_qgemm(x, lin)
+    torch.cuda.synchronize()
+    assert bool(torch.isfinite(y.float()).all())
+    rng = np.random.default_rng(0)
+    rows = np.concatenate([[0, 127, 128, M - 1], rng.integers(0, M, 12)])
+    cols = np.concatenate([[0, 255, 256, N - 1], rng.integers(0, N, 28)])
+    ref_lin = oracle.QLinear(to_np(lin.codes), to_np(lin.params), to_np(b), K, N, g)
+    wcols = ref_lin.columns(cols)                      # [K, ncols] exact fp16 weights
+    xr = fg_synth.values(11, 1, (rows[:, None] * K + np.arange(K)[None, :]).ravel(), "normal", 1.0).reshape(-1, K)
+    exp = (xr.astype(np.float64) @ wcols + to_np(b)[cols].astype(np.float64)).astype(np.float16)
+    got = to_np(y)[rows][:, cols]
+    assert_close_rms(got, exp, what="sampled prefill GEMM")
+
+
+def test_lm_head_argmax(fg):
+    import torch
+    B, h, V = 5, 256, 1000      # V not a multiple of the 256-wide tile
+    x = fg_synth.tensor(3, 1, (B, h), "normal", 1.0)
+    E = fg_synth.tensor(3, 2, (V, h), "normal", 0.5)
+    logits = torch.empty((B, V), dtype=torch.float32, device="cuda")
+    tok = fg.fg_lm_head_argmax(to_dev(x), to_dev(E), logits=logits)
+    torch.cuda.synchronize()
+    exp = oracle.linear_fp16(x, E)
+    assert_close_rms(to_np(logits), exp, tol=1e-3, what="logits")
+    top2 = np.sort(exp, axis=1)[:, -2:]
+    for i in range(B):
+        if top2[i, 1] - top2[i, 0] > 1e-3 * np.sqrt(np.mean(exp ** 2)):
+            assert int(to_np(tok)[i]) == int(np.argmax(exp[i]))
+    # ties go to the lowest id
+    E2 = E.copy()
+    E2[700] = E2[123] = np.float16(0)
+    E2[123, :] = x[0] * np.float16(0.25)
+    E2[700] = E2[123]
+    tok2 = fg.fg_lm_head_argmax(to_dev(x[:1]), to_dev(E2))
+    torch.cuda.synchronize()
+    assert int(to_np(tok2)[0]) == 123

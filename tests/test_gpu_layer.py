@@ -1,0 +1,162 @@
+"""GPU parity of LayerNorm, embedding, the decoder layer (prefill and decode) and greedy
+generation against the oracle.  Float outputs: max|err| <= 1e-2 * RMS(oracle).  Tokens:
+free-running generation must agree at >= 99 % of positions; a disagreement is accepted
+only where the oracle's own top-2 logit margin at that position is within the float
+tolerance (a near tie, where either token is a correct argmax), and the comparison stops
+for that sequence there."""
+import numpy as np
+import pytest
+
+import fg_synth
+import oracle
+from fg_synth import layer_stream as ls
+from gpu_util import TOL_RMS, assert_close_rms, to_dev, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fg():
+    import torch
+    assert torch.cuda.is_available()
+    import bit_group_quantized_fg_b200 as m
+    m.lib()
+    return m
+
+
+def make_layer(seed, l, h, F, g=64, wscale=0.02, ln_random=False):
+    """Oracle and device copies of one decoder layer from seeded fp16 tensors."""
+    def t(kind, shape, dist="normal", scale=wscale):
+        return fg_synth.tensor(seed, ls(l, kind), shape, dist, scale)
+    if ln_random:
+        ln = [t(0, (h,), scale=0.1) + np.float16(1.0), t(1, (h,), scale=0.1),
+              t(2, (h,), scale=0.1) + np.float16(1.0), t(3, (h,), scale=0.1)]
+    else:
+        ln = [np.ones(h, np.float16), np.zeros(h, np.float16), np.ones(h, np.float16), np.zeros(h, np.float16)]
+    ws = [(fg_synth.S_WQKV, fg_synth.S_BQKV, h, 3 * h), (fg_synth.S_WO, fg_synth.S_BO, h, h),
+          (fg_synth.S_W1, fg_synth.S_B1, h, F), (fg_synth.S_W2, fg_synth.S_B2, F, h)]
+    o_lins, d_lins = [], []
+    for wk, bk, K, N in ws:
+        w = t(wk, (K, N))
+        b = t(bk, (N,), scale=0.02)
+        o_lins.append(oracle.QLinear.from_fp16(w, b, g))
+        d_lins.append((w, b, K, N))
+    ol = oracle.QLayer(*ln, *o_lins)
+    return ol, ln, d_lins
+
+
+def to_device_layer(fg, ln, d_lins, g=64):
+    lins = [fg.DeviceQLinear.from_fp16(to_dev(w), to_dev(b), g) for (w, b, K, N) in d_lins]
+    return fg.DeviceLayer(*[to_dev(x) for x in ln], *lins)
+
+
+def test_layernorm(fg):
+    import torch
+    x = fg_synth.tensor(1, 1, (33, 4096), "normal", 3.0)
+    g = fg_synth.tensor(1, 2, (4096,), "normal", 0.5)
+    b = fg_synth.tensor(1, 3, (4096,), "normal", 0.5)
+    y = fg.fg_layernorm(to_dev(x), to_dev(g), to_dev(b))
+    torch.cuda.synchronize()
+    assert_close_rms(to_np(y), oracle.layernorm(x, g, b), tol=2e-3, what="layernorm")
+    for h in (768, 7168, 12288):
+        x = fg_synth.tensor(2, h, (5, h), "t3", 1.0)
+        y = fg.fg_layernorm(to_dev(x), to_dev(np.ones(h, np.float16)), to_dev(np.zeros(h, np.float16)))
+        torch.cuda.synchronize()
+        assert_close_rms(to_np(y), oracle.layernorm(x, np.ones(h, np.float16), np.zeros(h, np.float16)),
+                         tol=2e-3, what=f"layernorm h={h}")
+
+
+def test_embed_exact(fg):
+    import torch
+    V, h, P = 50, 64, 40
+    E = fg_synth.tensor(4, 1, (V, h), "normal", 1.0)
+    Pm = fg_synth.tensor(4, 2, (P, h), "normal", 1.0)
+    ids = fg_synth.token_ids(4, 3, (3, 7), V)
+    m = oracle.Model(0, h, 1, h, 4 * h, V, P, 64, E, Pm, np.ones(h, np.float16), np.zeros(h, np.float16), [])
+    out = fg.fg_embed(to_dev(ids), 5, to_dev(E), to_dev(Pm))
+    torch.cuda.synchronize()
+    exp = oracle.embed(m, ids, 5).reshape(21, h)
+    assert np.array_equal(to_np(out).view(np.uint16), exp.view(np.uint16))
+
+
+@pytest.mark.parametrize("ln_random", [False, True])
+def test_config1_layer_prefill_then_decode(fg, ln_random):
+    """Config 1: OPT-125M-shaped layer (h 768, 12 x 64, F 3072), batch 4, prompt 32 hidden
+    states ~ N(0,1), then 4 decode steps with a 4-bit cache (group 64)."""
+    import torch
+    h, nh, hd, F, B, L, steps = 768, 12, 64, 3072, 4, 32, 4
+    ol, ln, d_lins = make_layer(1234, 0, h, F, ln_random=ln_random)
+    dl = to_device_layer(fg, ln, d_lins)
+    x = fg_synth.tensor(1234, fg_synth.S_HIDDEN, (B, L, h), "normal", 1.0)
+    xd = to_dev(x.reshape(B * L, h))
+    dcache = fg.DeviceKVCache(B, nh, hd, L + steps, 64)
+    fg.fg_prefill_layer(dl, dcache, xd, B, L)
+    torch.cuda.synchronize()
+    ocache = oracle.KVCache(B, nh, hd, 64, L + steps)
+    xo = oracle.prefill_layer(ol, ocache, x)
+    assert_close_rms(to_np(xd).reshape(B, L, h), xo, what="prefill layer")
+    assert dcache.length == L == ocache.length
+    for s in range(steps):
+        xin = fg_synth.tensor(1234, fg_synth.S_DECODE_X, (B, h), "normal", 1.0, offset=s * B * h)
+        y = fg.fg_decode_layer(dl, dcache, to_dev(xin))
+        torch.cuda.synchronize()
+        yo = oracle.decode_layer(ol, ocache, xin)
+        assert_close_rms(to_np(y), yo, what=f"decode step {s}")
+    assert dcache.length == L + steps
+
+
+def small_model(fg, seed=5, n_layers=2, h=256, nh=4, F=1024, V=1000, max_pos=64, g=64):
+    hd = h // nh
+    layers_o, layers_d = [], []
+    for l in range(n_layers):
+        ol, ln, d_lins = make_layer(seed, l, h, F, g, wscale=0.05, ln_random=True)
+        layers_o.append(ol)
+        layers_d.append(to_device_layer(fg, ln, d_lins, g))
+    E = fg_synth.tensor(seed, fg_synth.S_EMBED, (V, h), "normal", 0.5)
+    P = fg_synth.tensor(seed, fg_synth.S_POS, (max_pos, h), "normal", 0.1)
+    lnf_g = np.ones(h, np.float16)
+    lnf_b = np.zeros(h, np.float16)
+    mo = oracle.Model(n_layers, h, nh, hd, F, V, max_pos, g, E, P, lnf_g, lnf_b, layers_o)
+    md = fg.DeviceModel(n_layers, h, nh, hd, F, V, max_pos, g, to_dev(E), to_dev(P), to_dev(lnf_g),
+                        to_dev(lnf_b), layers_d)
+    return mo, md
+
+
+def compare_tokens(got, exp_tokens, exp_logits):
+    """Positions that agree, with near ties (top-2 margin within tolerance) accepted."""
+    B, T = exp_tokens.shape
+    agree = total = 0
+    for b in range(B):
+        for t in range(T):
+            total += 1
+            if got[b, t] == exp_tokens[b, t]:
+                agree += 1
+                continue
+            lg = exp_logits[t, b]
+            top2 = np.sort(lg)[-2:]
+            margin = top2[1] - top2[0]
+            tol = TOL_RMS * np.sqrt(np.mean(lg * lg))
+            assert margin <= tol, f"seq {b} pos {t}: token {got[b, t]} vs {exp_tokens[b, t]}, margin {margin}"
+            agree += T - t   # a near tie: both continuations are valid; stop comparing this sequence
+            break
+    return agree / total
+
+
+def test_generate_small_model(fg):
+    import torch
+    mo, md = small_model(fg)
+    B, L, T = 4, 16, 8
+    ids = fg_synth.token_ids(5, fg_synth.S_IDS, (B, L), mo.vocab)
+    caches = [fg.DeviceKVCache(B, mo.n_heads, mo.head_dim, L + T, 64) for _ in range(mo.n_layers)]
+    out, timing = fg.fg_generate(md, to_dev(ids), T, caches)
+    torch.cuda.synchronize()
+    exp, logits = oracle.generate(mo, ids, T, return_logits=True)
+    frac = compare_tokens(to_np(out), exp, logits)
+    assert frac >= 0.99
+    assert timing.tokens == B * T and timing.tok_per_s > 0
+    assert all(c.length == L + T - 1 for c in caches)
+    # rows are independent: a sub-batch generates the same tokens
+    caches2 = [fg.DeviceKVCache(2, mo.n_heads, mo.head_dim, L + T, 64) for _ in range(mo.n_layers)]
+    out2, _ = fg.fg_generate(md, to_dev(ids[[3, 1]]), T, caches2)
+    torch.cuda.synchronize()
+    assert compare_tokens(to_np(out2), exp[[3, 1]], logits[:, [3, 1]]) >= 0.99
