@@ -1,0 +1,469 @@
+"""Throughput benchmark: greedy generation over 4-bit weights and a 4-bit KV cache.
+
+Workload (one "step"): an OPT-6.7B-shaped decoder (32 layers, hidden 4096, 32 heads x 128,
+FFN 16384, vocab 50272, learned positions), random fp16 init ~ N(0, 0.02) compressed to
+4 bits in groups of 64 along each weight's output channel, batch 64, prompt 512 token ids
+uniform over the vocabulary, 32 generated tokens (1 from the prompt pass + 31 decode steps)
+- the metric of the FlexGen README mirror's benchmark table: generated tokens / (prompt
+time + generation time).  Synthetic, seeded data (no checkpoints or datasets).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs N independent replicas (one process per GPU, launched by torchrun): the batch
+dimension shards with no exchange step, so each rank generates its own batch of 64
+(weak scaling) and the value is all ranks' tokens divided by the slowest rank's time.
+`--impl reference` times the CPU oracle on a bounded sample of the same workload.
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "generated tokens/s at 1 B200 (prefill+decode) vs roofline; quantizer GB/s"
+CFG = dict(model="OPT-6.7B-shaped 32-layer decoder", n_layers=32, hidden=4096, n_heads=32, head_dim=128,
+           ffn=16384, vocab=50272, max_pos=2048, group=64, batch=64, prompt_len=512, gen_len=32)
+SEED = 1234
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], tf=d["bf16_tflops"], tf_sust=d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                    src="measured")
+    return dict(hbm=6650.0, tf=1590.0, tf_sust=1400.0, src="fallback")
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.f = None
+
+    def __enter__(self):
+        try:
+            self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.index)], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.f is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.f.flush()
+        rows = [l.split(",") for l in open(self.f.name).read().strip().splitlines() if l.count(",") >= 8]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- model
+def build_model(fg, torch, dev):
+    from fg_synth import gpu as sg
+    from fg_synth import layer_stream as ls
+    import fg_synth
+    c = CFG
+    h, F, g = c["hidden"], c["ffn"], c["group"]
+    ones = torch.ones(h, dtype=torch.float16, device=dev)
+    zeros = torch.zeros(h, dtype=torch.float16, device=dev)
+    layers = []
+    for l in range(c["n_layers"]):
+        lins = []
+        for kind, K, N in ((fg_synth.S_WQKV, h, 3 * h), (fg_synth.S_WO, h, h), (fg_synth.S_W1, h, F),
+                           (fg_synth.S_W2, F, h)):
+            w = torch.empty((K, N), dtype=torch.float16, device=dev)
+            sg.fill(w, SEED, ls(l, kind), "normal", 0.02)
+            lins.append(fg.DeviceQLinear.from_fp16(w, torch.zeros(N, dtype=torch.float16, device=dev), g))
+            del w
+        layers.append(fg.DeviceLayer(ones, zeros, ones, zeros, *lins))
+    E = torch.empty((c["vocab"], h), dtype=torch.float16, device=dev)
+    sg.fill(E, SEED, fg_synth.S_EMBED, "normal", 0.02)
+    P = torch.empty((c["max_pos"], h), dtype=torch.float16, device=dev)
+    sg.fill(P, SEED, fg_synth.S_POS, "normal", 0.02)
+    model = fg.DeviceModel(c["n_layers"], h, c["n_heads"], c["head_dim"], F, c["vocab"], c["max_pos"], g, E, P,
+                           ones, zeros, layers)
+    caches = [fg.DeviceKVCache(c["batch"], c["n_heads"], c["head_dim"], c["prompt_len"] + c["gen_len"], g, dev)
+              for _ in range(c["n_layers"])]
+    return model, caches
+
+
+# ---------------------------------------------------------------------------- oracle baseline
+def synth_host(stream, shape, dist="normal", scale=1.0):
+    """fg_synth values as a host numpy array; generated by the generator's GPU twin when a
+    GPU is present (same bits, much faster than the numpy generator for 10^8 elements)."""
+    import fg_synth
+    try:
+        import torch
+        if torch.cuda.is_available():
+            from fg_synth import gpu as sg
+            t = torch.empty(shape, dtype=torch.float16, device="cuda")
+            sg.fill(t, SEED, stream, dist, scale)
+            return t.cpu().numpy()
+    except Exception:
+        pass
+    return fg_synth.tensor(SEED, stream, shape, dist, scale)
+
+
+def oracle_sample():
+    """Time the CPU oracle on a bounded sample: one sequence through one decoder layer's
+    prompt pass (512 tokens), one decode step at context 528 (the mid-point of the 31
+    decode steps) and one LM-head token, at the OPT-6.7B shapes; returns the seconds of
+    each part (weights are generated and quantized before the clock starts)."""
+    import numpy as np
+    import fg_synth
+    import oracle
+    from fg_synth import layer_stream as ls
+    c = CFG
+    h, F, g, L = c["hidden"], c["ffn"], c["group"], c["prompt_len"]
+    nh, hd = c["n_heads"], c["head_dim"]
+    lins = []
+    for kind, K, N in ((fg_synth.S_WQKV, h, 3 * h), (fg_synth.S_WO, h, h), (fg_synth.S_W1, h, F),
+                       (fg_synth.S_W2, F, h)):
+        w = synth_host(ls(0, kind), (K, N), "normal", 0.02)
+        lin = oracle.QLinear.from_fp16(w, np.zeros(N, np.float16), g)
+        lin.weight()
+        lins.append(lin)
+    ones, zeros = np.ones(h, np.float16), np.zeros(h, np.float16)
+    layer = oracle.QLayer(ones, zeros, ones, zeros, *lins)
+    E = synth_host(fg_synth.S_EMBED, (c["vocab"], h), "normal", 0.02)
+    P = synth_host(fg_synth.S_POS, (c["max_pos"], h), "normal", 0.02)
+    model = oracle.Model(1, h, nh, hd, F, c["vocab"], c["max_pos"], g, E, P, ones, zeros, [layer])
+    ids = fg_synth.token_ids(SEED, fg_synth.S_IDS, (1, L), c["vocab"])
+
+    def run():
+        cache = oracle.KVCache(1, nh, hd, g, L + c["gen_len"])
+        t0 = time.perf_counter()
+        x = oracle.prefill_layer(layer, cache, oracle.embed(model, ids, 0))
+        t1 = time.perf_counter()
+        cache.length = 528 - 1 if L + c["gen_len"] > 528 else cache.length
+        xd = oracle.decode_layer(layer, cache, x[:, -1, :])
+        t2 = time.perf_counter()
+        oracle.lm_head_argmax(model, xd)
+        t3 = time.perf_counter()
+        return t1 - t0, t2 - t1, t3 - t2
+    return run
+
+
+def oracle_rate(t_pf, t_dec, t_lm):
+    """Extrapolated tokens/s of the whole workload from one sample (sequences independent:
+    B sequences x n_layers x (prompt + T-1 decode steps) + T LM-head tokens per sequence)."""
+    c = CFG
+    per_seq = c["n_layers"] * (t_pf + (c["gen_len"] - 1) * t_dec) + c["gen_len"] * t_lm
+    return c["batch"] * c["gen_len"] / (c["batch"] * per_seq)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline_line(args, steps, warmup):
+    run = oracle_sample()
+    for _ in range(warmup):
+        run()
+    ts = [run() for _ in range(steps)]
+    t_pf = statistics.median(t[0] for t in ts)
+    t_dec = statistics.median(t[1] for t in ts)
+    t_lm = statistics.median(t[2] for t in ts)
+    rate = oracle_rate(t_pf, t_dec, t_lm)
+    sample = (f"oracle on 1 sequence x 1 layer: prompt pass 512 tokens ({t_pf:.2f} s), one decode step at "
+              f"context 528 ({t_dec:.2f} s), one LM-head token ({t_lm:.2f} s); extrapolated to 64 sequences x "
+              f"32 layers x (prompt + 31 decode steps) + 32 LM-head tokens")
+    return {"value": rate, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle", "sample": sample,
+            "sample_seconds": sum(ts[-1])}
+
+
+# ---------------------------------------------------------------------------- kernel-only cases
+def kernel_case(args):
+    """One kernel class on its own (for ncu captures and micro-measurements):
+    qgemm            prompt-pass QKV slice: M 16384, N 12288, K 4096, group 64 (X 134 MB)
+    decode_attention config-2 decode step: B 64, 32 heads x 128, context 543 (160 MB of cache)
+    quantize         1 GiB fp16 tensor [131072 x 4096], group 64
+    Runs `--warmup` untimed and `--steps` timed launches and prints their mean time."""
+    import torch
+    import bit_group_quantized_fg_b200 as fg
+    from fg_synth import gpu as sg
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if args.case == "qgemm":
+        M, N, K = 16384, 12288, 4096
+        x = torch.empty((M, K), dtype=torch.float16, device=dev)
+        sg.fill(x, SEED, 1, "normal", 1.0)
+        w = torch.empty((K, N), dtype=torch.float16, device=dev)
+        sg.fill(w, SEED, 2, "normal", 0.02)
+        lin = fg.DeviceQLinear.from_fp16(w, torch.zeros(N, dtype=torch.float16, device=dev), 64)
+        del w
+        y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        run = lambda: fg.fg_qgemm(x, lin, Y=y)
+        work = {"flops": 2.0 * M * N * K}
+    elif args.case == "decode_attention":
+        B, nh, hd, S = 64, 32, 128, 543
+        h = nh * hd
+        kv = torch.empty((B * S, 2 * h), dtype=torch.float16, device=dev)
+        sg.fill(kv, SEED, 3, "normal", 1.0)
+        q = torch.empty((B, 3 * h), dtype=torch.float16, device=dev)
+        sg.fill(q, SEED, 4, "normal", 1.0)
+        cache = fg.DeviceKVCache(B, nh, hd, S + 1, 64, dev)
+        fg.fg_kv_append(cache, kv, kv[:, h:], 2 * h, S)
+        del kv
+        out = torch.empty((B, h), dtype=torch.float16, device=dev)
+        run = lambda: fg.fg_decode_attention(q, 3 * h, cache, out=out)
+        work = {"bytes": B * nh * S * 2.0 * (hd / 2 + 4.0 * hd / 64) + 4.0 * B * h}
+    else:
+        x = torch.empty((131072, 4096), dtype=torch.float16, device=dev)
+        sg.fill(x, SEED, 7, "normal", 0.02)
+        codes = torch.empty((131072, 2048), dtype=torch.uint8, device=dev)
+        params = torch.empty((131072, 64, 2), dtype=torch.float16, device=dev)
+        run = lambda: fg.fg_quantize_pack(x, 64, 1, codes, params)
+        work = {"bytes": x.numel() * (2 + 0.5 + 4 / 64)}
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / max(args.steps, 1)
+    res = {"case": args.case, "ms_per_launch": ms}
+    if "flops" in work:
+        res["TFLOP/s"] = work["flops"] / (ms * 1e-3) / 1e12
+    if "bytes" in work:
+        res["GB/s"] = work["bytes"] / (ms * 1e-3) / 1e9
+    print(json.dumps(res))
+
+
+# ---------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", choices=["generate", "qgemm", "decode_attention", "quantize"], default="generate",
+                    help="kernel-only cases sized for ncu captures (inputs larger than L2, a few GB at most)")
+    args = ap.parse_args()
+    if args.case != "generate":
+        return kernel_case(args)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    c = CFG
+    config = {"workload": "OPT-6.7B-shaped decoder, 4-bit weights + 4-bit KV (group 64), batch 64 per GPU, "
+                          "prompt 512, generate 32", "layers": c["n_layers"], "hidden": c["hidden"],
+              "heads": f"{c['n_heads']}x{c['head_dim']}", "ffn": c["ffn"], "vocab": c["vocab"],
+              "global_batch": c["batch"] * max(world, args.gpus if world == 1 else world),
+              "prompt_len": c["prompt_len"], "gen_len": c["gen_len"], "group": c["group"],
+              "parallelism": f"replicas x{max(world, 1)} (batch-sharded, no exchange)",
+              "l2": "inputs larger than L2 (3.6 GB of 4-bit weights + 5 GB KV cache per step)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        steps, warmup = args.steps, args.warmup
+        cb = cpu_baseline_line(args, steps, warmup)
+        line = {"metric": METRIC, "value": cb["value"], "unit": "tokens/s", "n_gpus": world, "steps": steps,
+                "warmup": warmup, "ms_per_step": 1000.0 * c["batch"] * c["gen_len"] / cb["value"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": config, "impl": "reference",
+                "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import torch
+    import bit_group_quantized_fg_b200 as fg
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    model, caches = build_model(fg, torch, dev)
+    B, L, T = c["batch"], c["prompt_len"], c["gen_len"]
+    from fg_synth import gpu as sg
+    import fg_synth
+    ids = torch.empty((B, L), dtype=torch.int32, device=dev)
+    sg.fill_ids(ids, SEED + rank, fg_synth.S_IDS, c["vocab"])
+    out = torch.empty((B, T), dtype=torch.int32, device=dev)
+    ws = torch.empty((fg.fg_workspace_bytes(model, B, L, T),), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
+    # ---- timed region: device-resident inputs
+    fg.fg_profile_reset()
+    fg.fg_profile_enable(True)
+    launches0 = fg.fg_launch_count()
+    timings = []
+    barrier()
+    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local) as clk:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            _, tm = fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
+            timings.append((tm.prefill_ms, tm.decode_ms))
+        e1.record(stream)
+        barrier()
+    launches = fg.fg_launch_count() - launches0
+    fg.fg_profile_enable(False)
+    ms_total = e0.elapsed_time(e1)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    tokens_step = B * T * world
+    value = tokens_step / (ms_step / 1000.0)
+    prof = {fg.PROF_NAMES[k]: fg.fg_profile_read(k) for k in range(7)}
+    clocks = clk.summary()
+
+    # ---- e2e: host buffers through the public API, copies inside the timed region
+    ids_host = ids.cpu().pin_memory()
+    out_host = torch.empty((B, T), dtype=torch.int32).pin_memory()
+    ids_dev = torch.empty_like(ids)
+    barrier()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(args.steps):
+        ids_dev.copy_(ids_host, non_blocking=True)
+        fg.fg_generate(model, ids_dev, T, caches, out_ids=out, workspace=ws)
+        out_host.copy_(out, non_blocking=True)
+    e3.record(stream)
+    barrier()
+    ms_e2e = e2.elapsed_time(e3)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    e2e_value = tokens_step * args.steps / (ms_e2e / 1000.0)
+
+    # ---- quantizer GB/s on a 1 GiB fp16 tensor (group 64), bytes = 2 + 0.5 + 4/64 per element
+    xq = torch.empty((131072, 4096), dtype=torch.float16, device=dev)
+    sg.fill(xq, SEED, 7, "normal", 0.02)
+    codes = torch.empty((131072, 2048), dtype=torch.uint8, device=dev)
+    params = torch.empty((131072, 64, 2), dtype=torch.float16, device=dev)
+    for _ in range(3):
+        fg.fg_quantize_pack(xq, 64, 1, codes, params)
+    e4, e5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 10
+    e4.record(stream)
+    for _ in range(reps):
+        fg.fg_quantize_pack(xq, 64, 1, codes, params)
+    e5.record(stream)
+    torch.cuda.synchronize()
+    q_ms = e4.elapsed_time(e5) / reps
+    q_gbs = xq.numel() * (2 + 0.5 + 4 / 64) / (q_ms * 1e-3) / 1e9
+    del xq, codes, params
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    pk = peaks()
+    g = prof["gemm_prefill"]
+    g_ms = g["ms"] / max(g["launches"], 1)
+    g_flops = g["flops"] / max(g["launches"], 1)
+    achieved_tf = g_flops / (g_ms * 1e-3) / 1e12 if g_ms > 0 else 0.0
+    traffic = None
+    tfile = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tfile):
+        traffic = json.load(open(tfile)).get("gemm_prefill_bytes_per_launch")
+    da = prof["decode_attention"]
+    kernels = {}
+    for name, p in prof.items():
+        if p["launches"]:
+            d = {"launches_per_step": p["launches"] / args.steps, "ms_per_step": p["ms"] / args.steps}
+            if p["flops"] and p["ms"]:
+                d["TFLOP/s"] = p["flops"] / (p["ms"] * 1e-3) / 1e12
+            if p["bytes"] and p["ms"]:
+                d["GB/s"] = p["bytes"] / (p["ms"] * 1e-3) / 1e9
+            kernels[name] = d
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic", "config": config,
+        "prefill_ms": statistics.median(t[0] for t in timings), "decode_ms": statistics.median(t[1] for t in timings),
+        "roofline": {"kernel": "dequant-fused tcgen05 GEMM, prompt pass (M = 32768)", "bound": "tensor",
+                     "achieved": achieved_tf, "peak": pk["tf_sust"], "unit": "TFLOP/s",
+                     "frac": achieved_tf / pk["tf_sust"], "traffic": traffic,
+                     "peak_source": f"bf16_tflops_sustained of {pk['src']} peaks (fp16 and bf16 dense rates are equal)"},
+        "quantizer": {"GB/s": q_gbs, "frac": q_gbs / pk["hbm"], "peak_GB/s": pk["hbm"],
+                      "tensor": "1 GiB fp16 (131072 x 4096), group 64"},
+        "decode_attention": {"GB/s": da["bytes"] / (da["ms"] * 1e-3) / 1e9 if da["ms"] else None,
+                             "frac": (da["bytes"] / (da["ms"] * 1e-3) / 1e9) / pk["hbm"] if da["ms"] else None},
+        "kernels": kernels,
+        "clocks": clocks,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": B * L * 4,
+                "d2h_bytes_per_step": B * T * 4},
+        "gpu_launches": launches,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        try:
+            cb = cpu_baseline_line(args, 1, 0)
+            line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        except Exception as ex:  # the baseline is informative only
+            line["cpu_baseline"] = {"value": None, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+                                    "sample": f"failed: {ex}"}
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

@@ -17,7 +17,10 @@ LIB_PATH = os.path.join(HERE, "libfg.so")
 FG_OK = 0
 STATUS = {0: "FG_OK", -1: "FG_ERR_INVALID_ARG", -2: "FG_ERR_SHAPE", -3: "FG_ERR_ALIGN",
           -4: "FG_ERR_CAPACITY", -5: "FG_ERR_CUDA", -6: "FG_ERR_UNSUPPORTED", -7: "FG_ERR_WORKSPACE"}
-PROF_GEMM, PROF_DECODE_ATTN, PROF_PREFILL_ATTN, PROF_QUANT, PROF_OTHER = range(5)
+(PROF_GEMM, PROF_DECODE_ATTN, PROF_PREFILL_ATTN, PROF_QUANT, PROF_OTHER, PROF_GEMM_DECODE,
+ PROF_LM_HEAD) = range(7)
+PROF_NAMES = ["gemm_prefill", "decode_attention", "prefill_attention", "quantize_append", "other",
+              "gemm_decode", "lm_head"]
 
 
 class FGError(RuntimeError):
@@ -86,6 +89,7 @@ _SIGS = {
     "fg_profile_read": (c_int, [c_int, POINTER(c_double), POINTER(c_int64), POINTER(c_double),
                                 POINTER(c_double)]),
     "fg_profile_reset": (c_int, []),
+    "fg_launch_count": (c_int64, []),
 }
 
 _lib = None
@@ -334,6 +338,10 @@ def fg_profile_enable(on: bool = True):
 
 def fg_profile_reset():
     _check(lib().fg_profile_reset())
+
+
+def fg_launch_count() -> int:
+    return lib().fg_launch_count()
 
 
 def fg_profile_read(kind: int):

@@ -4,6 +4,7 @@
 // Generation follows the "FlexGen" README mirror's benchmark notes: a prompt pass over
 // input length L yields the first token, then gen_len-1 decode steps; throughput =
 // generated tokens / (prompt time + generation time), both measured with CUDA events.
+#include <atomic>
 #include <cstdarg>
 #include <cstring>
 #include <mutex>
@@ -62,6 +63,10 @@ int num_sms() {
   }
   return cached[dev];
 }
+
+// ---------------------------------------------------------------- launch counter
+static std::atomic<int64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 // ---------------------------------------------------------------- profiling
 namespace {
@@ -487,6 +492,8 @@ int fg_profile_read(int kind, double* total_ms, int64_t* launches, double* flops
   if (bytes) *bytes = g_prof_bytes[kind];
   return FG_OK;
 }
+
+int64_t fg_launch_count(void) { return g_launches.load(); }
 
 int fg_profile_reset(void) {
   std::lock_guard<std::mutex> lk(g_prof_mu);

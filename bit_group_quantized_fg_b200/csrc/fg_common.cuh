@@ -22,8 +22,11 @@ int cuda_fail(cudaError_t e, const char* what);
     if (_e != cudaSuccess) return ::fg::cuda_fail(_e, #expr); \
   } while (0)
 
+void count_launch();
+
 #define FG_CHECK_LAUNCH(what)                               \
   do {                                                      \
+    ::fg::count_launch();                                   \
     cudaError_t _e = cudaGetLastError();                    \
     if (_e != cudaSuccess) return ::fg::cuda_fail(_e, what); \
   } while (0)
@@ -41,7 +44,7 @@ int num_sms();
 
 // Kernel classes for fg_profile_* (same numbering as the header).
 enum ProfKind { PROF_GEMM = 0, PROF_DECODE_ATTN = 1, PROF_PREFILL_ATTN = 2, PROF_QUANT = 3,
-                PROF_OTHER = 4, PROF_NKINDS = 5 };
+                PROF_OTHER = 4, PROF_GEMM_DECODE = 5, PROF_LM_HEAD = 6, PROF_NKINDS = 7 };
 // RAII pair of events around a launch when profiling is on.
 struct ProfScope {
   int slot;

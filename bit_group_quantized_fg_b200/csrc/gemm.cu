@@ -542,7 +542,7 @@ int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, c
   const double bytes = (mode == B_Q4 ? double(N) * K * (0.5 + 4.0 / G) : double(N) * K * 2.0) +
                        double(M) * K * 2.0 + double(M) * N * (out_f32 ? 4.0 : 2.0) + (R ? double(M) * N * 2.0 : 0.0);
   {
-    ProfScope ps(PROF_GEMM, s, flops, bytes);
+    ProfScope ps(out_f32 ? PROF_LM_HEAD : (M > 256 ? PROF_GEMM : PROF_GEMM_DECODE), s, flops, bytes);
     int st;
     if (mode == B_Q4) st = launch<B_Q4, false>(ta, tb, tp, a, s);
     else if (mode == B_F16_MN) st = launch<B_F16_MN, false>(ta, tb, tp, a, s);

@@ -200,12 +200,18 @@ int fg_generate(const fg_model* model, const int32_t* prompt_ids, int B, int L, 
                 fg_timing* timing, void* stream);
 
 /* Per-kernel device timing of the library's own launches (CUDA events on the launching
- * stream).  kind: 0 = dequant GEMM, 1 = decode attention, 2 = prefill attention,
- * 3 = quantize/append, 4 = other.  Enabling adds one event pair per launch. */
+ * stream).  kind: 0 = dequant GEMM of a prompt pass (M > 256), 1 = decode attention,
+ * 2 = prefill attention, 3 = quantize/append, 4 = other (LayerNorm, embedding, argmax),
+ * 5 = dequant GEMM of a decode step (M <= 256), 6 = LM head GEMM.  flops and bytes are the
+ * algorithmic work of the timed launches.  Enabling adds one event pair per launch;
+ * fg_profile_read synchronizes the recorded events. */
 int fg_profile_enable(int on);
 int fg_profile_read(int kind, double* total_ms, int64_t* launches, double* flops,
                     double* bytes);
 int fg_profile_reset(void);
+
+/* Number of kernels this library has launched in the process so far. */
+int64_t fg_launch_count(void);
 
 #ifdef __cplusplus
 }
