@@ -70,6 +70,7 @@ _SIGS = {
     "fg_decode_attention_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int]),
     "fg_decode_attention": (c_int, [c_void_p, c_int64, POINTER(KVCache), c_void_p, c_void_p, c_size_t,
                                     c_void_p]),
+    "fg_decode_attention_noalloc": (c_int, [c_void_p, c_int64, POINTER(KVCache), c_void_p, c_void_p]),
     "fg_prefill_attention": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p]),
     "fg_layernorm": (c_int, [c_void_p, c_int64, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
     "fg_embed": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p]),
@@ -241,6 +242,17 @@ def fg_decode_attention(q, q_stride: int, cache: DeviceKVCache, out=None, worksp
         workspace = _empty((wsb,), torch.uint8, q.device)
     _check(lib().fg_decode_attention(_ptr(q), q_stride, ctypes.byref(cache.c), _ptr(out), _ptr(workspace),
                                      0 if workspace is None else workspace.numel(), _stream(stream)))
+    return out
+
+
+def fg_decode_attention_noalloc(q, q_stride: int, cache: DeviceKVCache, out=None, stream=None):
+    """fg_decode_attention with its scratch in the library's fixed device array (no workspace).
+    Only `out` may be allocated here, and only when the caller passes none."""
+    import torch
+    B, nh, hd = cache.c.B, cache.c.n_heads, cache.c.head_dim
+    if out is None:
+        out = _empty((B, nh * hd), torch.float16, q.device)
+    _check(lib().fg_decode_attention_noalloc(_ptr(q), q_stride, ctypes.byref(cache.c), _ptr(out), _stream(stream)))
     return out
 
 

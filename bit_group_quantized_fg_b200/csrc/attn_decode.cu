@@ -12,6 +12,7 @@
 // identity with weights p_t s_t.  Softmax is fp32 with exp2 (q pre-scaled by
 // log2(e)/sqrt(hd)); chunks are merged with the usual (max, sum, acc) rescaling.
 #include <algorithm>
+#include <mutex>
 
 #include "fg_common.cuh"
 
@@ -318,3 +319,58 @@ int decode_attention_impl(const void* q, int64_t q_stride, const fg_kv_cache* c,
 }
 
 }  // namespace fg
+
+// ==================================================================== no-allocation variant
+// fg_decode_attention_noalloc: the same kernels, with the split-context partials in a fixed
+// array compiled into the library instead of a caller-provided workspace.  It serves callers
+// that may not allocate device memory themselves (see include/fg.h).  The array is held by
+// every GPU that loads the library until the process exits.
+namespace fg {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB of fp32 partials
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Device address of the array for the current device, looked up once per device (with
+// that device current) on the first call; host code must not use the symbol itself.
+int noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(FG_ERR_UNSUPPORTED, "device ordinal %d above 63", dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return FG_OK;
+}
+
+}  // namespace
+}  // namespace fg
+
+extern "C" int fg_decode_attention_noalloc(const void* q, int64_t q_stride, const fg_kv_cache* cache, void* out,
+                                           void* stream) {
+  using namespace fg;
+  if (!cache) return fail(FG_ERR_INVALID_ARG, "null cache");
+  const size_t need = decode_attention_ws_bytes(cache->B, cache->n_heads, cache->head_dim, cache->len);
+  if (need > kNoAllocScratchBytes)
+    return fail(FG_ERR_WORKSPACE,
+                "this shape needs %zu bytes of split-context scratch; the fixed no-allocation array holds %zu "
+                "(use fg_decode_attention with a workspace)",
+                need, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  FG_TRY(noalloc_scratch(&scratch));
+  // Every partial the combine step reads is written by this call first: nothing to clear.
+  return decode_attention_impl(q, q_stride, cache, out, scratch, kNoAllocScratchBytes, as_stream(stream));
+}

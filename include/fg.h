@@ -150,6 +150,23 @@ size_t fg_decode_attention_workspace_bytes(int B, int n_heads, int head_dim, int
 int fg_decode_attention(const void* q, int64_t q_stride, const fg_kv_cache* cache, void* out,
                         void* workspace, size_t ws_bytes, void* stream);
 
+/* Decode attention that needs no device memory from the caller and allocates none itself.
+ * The pages have no counterpart to this call; it exists for callers that cannot call
+ * cudaMalloc: code embedded in a host program that owns every byte of device memory through
+ * its own pool (a stray allocation would break its accounting), or a latency-critical decode
+ * loop where an allocation and the synchronization it implies are not allowed.
+ * Same arguments and results as fg_decode_attention without the workspace: the partial
+ * (max, sum, acc) results of a split context go to a fixed 4 MiB array built into the library,
+ * which every GPU that loads the library holds until the process exits.
+ *  - A shape whose partials need more than 4 MiB (fg_decode_attention_workspace_bytes tells)
+ *    is rejected with FG_ERR_WORKSPACE before any launch.
+ *  - The first call on a device looks up the array's address with that device current; make
+ *    that first call before any stream capture.
+ *  - All calls share the array.  Each call writes every partial it reads, so nothing carries
+ *    over between calls, but calls that overlap on the GPU (other streams or threads) race. */
+int fg_decode_attention_noalloc(const void* q, int64_t q_stride, const fg_kv_cache* cache,
+                                void* out, void* stream);
+
 /* Causal prefill attention on unquantized fp16 projections: qkv fp16 [B*L][3h]
  * (q | k | v), out fp16 [B*L][h].  "FlexGen" README mirror: prompt processing time is
  * part of the throughput metric. */
