@@ -291,6 +291,98 @@ size_t generate_ws(const fg_model* m, int B, int L, int T) {
 }
 }  // namespace
 
+// ---------------------------------------------------------------- CUDA graphs for generate
+// A generation is ~12k short launches (31 decode steps x 32 layers x ~10 kernels); issuing
+// them one by one makes the decode steps host-bound.  The first call with a configuration
+// runs eagerly (and loads every kernel); the second records the prompt pass and the decode
+// steps as two graphs on a private capture stream; later calls with the same configuration
+// replay them.  The key covers every pointer and size the launches bake in.
+namespace {
+struct GraphKey {
+  std::vector<uint8_t> bytes;
+  bool operator==(const GraphKey& o) const { return bytes == o.bytes; }
+};
+template <class T>
+void put(std::vector<uint8_t>& v, const T& x) {
+  const uint8_t* p = reinterpret_cast<const uint8_t*>(&x);
+  v.insert(v.end(), p, p + sizeof(T));
+}
+GraphKey make_key(const fg_model* m, const int32_t* ids, int B, int L, int T, int32_t* out,
+                  const fg_kv_cache* caches, void* ws, size_t wsb, cudaStream_t s) {
+  GraphKey k;
+  int dev = -1;
+  cudaGetDevice(&dev);
+  put(k.bytes, dev);
+  put(k.bytes, *m);
+  for (int l = 0; l < m->n_layers; ++l) put(k.bytes, m->layers[l]);
+  for (int l = 0; l < m->n_layers; ++l) {
+    fg_kv_cache c = caches[l];
+    c.len = 0;
+    put(k.bytes, c);
+  }
+  put(k.bytes, ids);
+  put(k.bytes, B);
+  put(k.bytes, L);
+  put(k.bytes, T);
+  put(k.bytes, out);
+  put(k.bytes, ws);
+  put(k.bytes, wsb);
+  put(k.bytes, s);
+  return k;
+}
+struct GraphCache {
+  GraphKey key;
+  bool seen = false, valid = false;
+  cudaGraphExec_t prefill = nullptr, decode = nullptr;
+  int64_t n_prefill = 0, n_decode = 0;
+  cudaStream_t cap = nullptr;
+};
+std::mutex g_graph_mu;
+GraphCache g_graph;
+
+bool profiling_on() {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  return g_prof_on;
+}
+
+void reset_graphs() {
+  if (g_graph.prefill) cudaGraphExecDestroy(g_graph.prefill);
+  if (g_graph.decode) cudaGraphExecDestroy(g_graph.decode);
+  g_graph.prefill = g_graph.decode = nullptr;
+  g_graph.valid = g_graph.seen = false;
+}
+
+template <class F>
+int capture_one(F&& seq, cudaGraphExec_t* exec, int64_t* n_launches) {
+  cudaStream_t cs = g_graph.cap;
+  const int64_t before = g_launches.load();
+  FG_CHECK_CUDA(cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal));
+  const int st = seq(cs);
+  cudaGraph_t graph = nullptr;
+  const cudaError_t ce = cudaStreamEndCapture(cs, &graph);
+  *n_launches = g_launches.load() - before;
+  g_launches.fetch_sub(*n_launches);  // recorded, not executed
+  if (st != FG_OK) {
+    if (graph) cudaGraphDestroy(graph);
+    return st;
+  }
+  if (ce != cudaSuccess) return cuda_fail(ce, "stream capture");
+  const cudaError_t ie = cudaGraphInstantiate(exec, graph, 0);
+  cudaGraphDestroy(graph);
+  if (ie != cudaSuccess) return cuda_fail(ie, "graph instantiate");
+  return FG_OK;
+}
+
+template <class P, class D>
+int capture_graphs(P&& prefill_seq, D&& decode_seq) {
+  if (!g_graph.cap) FG_CHECK_CUDA(cudaStreamCreateWithFlags(&g_graph.cap, cudaStreamNonBlocking));
+  FG_TRY(capture_one(prefill_seq, &g_graph.prefill, &g_graph.n_prefill));
+  FG_TRY(capture_one(decode_seq, &g_graph.decode, &g_graph.n_decode));
+  g_graph.valid = true;
+  return FG_OK;
+}
+}  // namespace
+
 int generate_impl(const fg_model* m, const int32_t* ids, int B, int L, int T, int32_t* out, fg_kv_cache* caches,
                   void* ws, size_t wsb, fg_timing* timing, cudaStream_t s) {
   if (!m || !ids || !out || !caches) return fail(FG_ERR_INVALID_ARG, "null pointer");
@@ -316,38 +408,71 @@ int generate_impl(const fg_model* m, const int32_t* ids, int B, int L, int T, in
   void* lws = c.take(layer_b);
   void* lgw = c.take(lm_ws(B, m->vocab));
 
+  // The two launch sequences of a generation (prompt pass; decode steps).  They run directly
+  // on `s`, or on the capture stream while a CUDA graph is recorded.
+  auto prefill_seq = [&](cudaStream_t st_) -> int {
+    for (int l = 0; l < m->n_layers; ++l) caches[l].len = 0;
+    FG_TRY(embed_impl(ids, B, L, L, 0, m->embed, m->pos_embed, h, x, st_));
+    for (int l = 0; l < m->n_layers; ++l) FG_TRY(prefill_layer_impl(&m->layers[l], &caches[l], x, B, L, lws, layer_b, st_));
+    // hidden state of each sequence's last prompt position
+    FG_CHECK_CUDA(cudaMemcpy2DAsync(xd, size_t(h) * 2, reinterpret_cast<uint8_t*>(x) + size_t(L - 1) * h * 2,
+                                    size_t(L) * h * 2, size_t(h) * 2, B, cudaMemcpyDeviceToDevice, st_));
+    FG_TRY(layernorm_impl(xd, B, h, m->lnf_g, m->lnf_b, xn, st_));
+    return lm_head_impl(xn, B, h, m->embed, m->vocab, nullptr, out, T, lgw, lm_ws(B, m->vocab), st_);
+  };
+  auto decode_seq = [&](cudaStream_t st_) -> int {
+    for (int j = 1; j < T; ++j) {
+      // token j-1 sits at position L + j - 1
+      FG_TRY(embed_impl(out + (j - 1), B, 1, T, L + j - 1, m->embed, m->pos_embed, h, xd, st_));
+      for (int l = 0; l < m->n_layers; ++l) FG_TRY(decode_layer_impl(&m->layers[l], &caches[l], xd, xd, B, lws, layer_b, st_));
+      FG_TRY(layernorm_impl(xd, B, h, m->lnf_g, m->lnf_b, xn, st_));
+      FG_TRY(lm_head_impl(xn, B, h, m->embed, m->vocab, nullptr, out + j, T, lgw, lm_ws(B, m->vocab), st_));
+    }
+    return FG_OK;
+  };
+
+  std::lock_guard<std::mutex> glk(g_graph_mu);
+  GraphKey key = make_key(m, ids, B, L, T, out, caches, ws, wsb, s);
+  const bool use_graphs = !profiling_on();
+  bool replay = false;
+  if (use_graphs && g_graph.valid && g_graph.key == key) {
+    replay = true;
+  } else if (use_graphs && g_graph.seen && g_graph.key == key) {
+    // second call with this configuration: record both sequences as graphs, then replay
+    FG_TRY(capture_graphs(prefill_seq, decode_seq));
+    replay = true;
+  } else {
+    reset_graphs();
+    g_graph.key = key;
+    g_graph.seen = use_graphs;
+  }
+
   cudaEvent_t e0, e1, e2;
   FG_CHECK_CUDA(cudaEventCreate(&e0));
   FG_CHECK_CUDA(cudaEventCreate(&e1));
   FG_CHECK_CUDA(cudaEventCreate(&e2));
   int st = FG_OK;
   do {
-    for (int l = 0; l < m->n_layers; ++l) caches[l].len = 0;
-    if ((st = cudaEventRecord(e0, s)) != cudaSuccess) { st = cuda_fail(cudaError_t(st), "event"); break; }
-    if ((st = embed_impl(ids, B, L, L, 0, m->embed, m->pos_embed, h, x, s)) != FG_OK) break;
-    for (int l = 0; l < m->n_layers && st == FG_OK; ++l)
-      st = prefill_layer_impl(&m->layers[l], &caches[l], x, B, L, lws, layer_b, s);
-    if (st != FG_OK) break;
-    // hidden state of each sequence's last prompt position
-    if (cudaMemcpy2DAsync(xd, size_t(h) * 2, reinterpret_cast<uint8_t*>(x) + size_t(L - 1) * h * 2,
-                          size_t(L) * h * 2, size_t(h) * 2, B, cudaMemcpyDeviceToDevice, s) != cudaSuccess) {
-      st = cuda_fail(cudaGetLastError(), "gather last positions");
+    cudaError_t ce = cudaEventRecord(e0, s);
+    if (ce != cudaSuccess) { st = cuda_fail(ce, "event"); break; }
+    if (replay) {
+      ce = cudaGraphLaunch(g_graph.prefill, s);
+      if (ce != cudaSuccess) { st = cuda_fail(ce, "graph launch (prompt pass)"); break; }
+      g_launches.fetch_add(g_graph.n_prefill);
+    } else if ((st = prefill_seq(s)) != FG_OK) {
       break;
     }
-    if ((st = layernorm_impl(xd, B, h, m->lnf_g, m->lnf_b, xn, s)) != FG_OK) break;
-    if ((st = lm_head_impl(xn, B, h, m->embed, m->vocab, nullptr, out, T, lgw, lm_ws(B, m->vocab), s)) != FG_OK) break;
     cudaEventRecord(e1, s);
-    for (int j = 1; j < T && st == FG_OK; ++j) {
-      // token j-1 sits at position L + j - 1
-      st = embed_impl(out + (j - 1), B, 1, T, L + j - 1, m->embed, m->pos_embed, h, xd, s);
-      for (int l = 0; l < m->n_layers && st == FG_OK; ++l)
-        st = decode_layer_impl(&m->layers[l], &caches[l], xd, xd, B, lws, layer_b, s);
-      if (st == FG_OK) st = layernorm_impl(xd, B, h, m->lnf_g, m->lnf_b, xn, s);
-      if (st == FG_OK) st = lm_head_impl(xn, B, h, m->embed, m->vocab, nullptr, out + j, T, lgw, lm_ws(B, m->vocab), s);
+    if (replay) {
+      ce = cudaGraphLaunch(g_graph.decode, s);
+      if (ce != cudaSuccess) { st = cuda_fail(ce, "graph launch (decode)"); break; }
+      g_launches.fetch_add(g_graph.n_decode);
+      for (int l = 0; l < m->n_layers; ++l) caches[l].len = L + T - 1;
+    } else if ((st = decode_seq(s)) != FG_OK) {
+      break;
     }
-    if (st != FG_OK) break;
     cudaEventRecord(e2, s);
-    cudaError_t ce = cudaEventSynchronize(e2);
+    ce = cudaEventSynchronize(e2);
     if (ce != cudaSuccess) { st = cuda_fail(ce, "generate"); break; }
     int derr = 0;
     if (read_device_error(&derr) == FG_OK && derr != 0) {

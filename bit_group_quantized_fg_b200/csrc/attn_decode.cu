@@ -5,7 +5,7 @@
 //   score_t = (q . K_t) / sqrt(hd),  K_t = mn_t + code_t * s_t (per group of G dims)
 //   out = sum_t softmax(score)_t V_t
 // The cache is read exactly once: one CTA per (chunk of positions, head, sequence)
-// streams the chunk's K codes (pass 1: scores into shared memory) and V codes (pass 2).
+// streams the chunk's K and V codes together in a single pass with an online softmax.
 // Codes are never expanded to fp16: with f = 0.5 + code/256 (built by one byte
 // permute into the mantissa of 0.5f), sum_i q_i code_i = 256 (sum_i q_i f_i - 0.5 sum_i q_i),
 // and a group contributes s * sum(q code) + mn * sum(q).  The V side uses the same
@@ -32,8 +32,7 @@ __device__ __forceinline__ void code_floats(uint32_t w, float f[8]) {
   const uint32_t even = w & 0x0F0F0F0Fu;
   const uint32_t odd = (w >> 4) & 0x0F0F0F0Fu;
   const uint32_t half = 0x3F000000u;
-  // selector nibbles: result byte r takes byte sel_r of {b (4..7), a (0..3)} = {half, src}
-  // result = [half.b0, half.b1, src.bk, half.b3] -> sel = 0x7 k 5 4 (byte3..byte0)
+  // result bytes (3..0) = [half.b3, src.bk, half.b1, half.b0] -> selector 0x7k54
   f[0] = __uint_as_float(__byte_perm(even, half, 0x7054));
   f[1] = __uint_as_float(__byte_perm(odd, half, 0x7054));
   f[2] = __uint_as_float(__byte_perm(even, half, 0x7154));
@@ -44,173 +43,177 @@ __device__ __forceinline__ void code_floats(uint32_t w, float f[8]) {
   f[7] = __uint_as_float(__byte_perm(odd, half, 0x7354));
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
+__device__ __forceinline__ uint4 ldg_v4(const uint4* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
 }
 
-// HD = head dim (64 or 128), G = group size (divides HD).
+// HD = head dim (64 or 128), G = group size (divides HD, >= 32).
+// Lane layout: LPT = HD/32 lanes per token, each owning 32 dims (one 16-byte load of K
+// codes and one of V codes per token, inside one group); TPW = 32/LPT tokens per warp
+// step.  Every lane keeps an online-softmax state (max m, sum l, weighted sums) for the
+// tokens of its slot; slots, warps and chunks are merged at the end with the usual rescaling.
 template <int HD, int G>
 __global__ void __launch_bounds__(kThreads) decode_attn_kernel(
-    const __half* __restrict__ q, int64_t q_stride, const uint32_t* __restrict__ kc,
-    const __half2* __restrict__ kp, const uint32_t* __restrict__ vc, const __half2* __restrict__ vp,
+    const __half* __restrict__ q, int64_t q_stride, const uint4* __restrict__ kc,
+    const __half2* __restrict__ kp, const uint4* __restrict__ vc, const __half2* __restrict__ vp,
     int nh, int cap, int S, int chunk_len, __half* __restrict__ out, float* __restrict__ part_ml,
     float* __restrict__ part_acc) {
-  constexpr int LPT = HD / 8;   // lanes per token: each lane owns 8 dims (one code word)
-  constexpr int TPW = 32 / LPT; // tokens per warp step
+  constexpr int LPT = HD / 32;
+  constexpr int TPW = 32 / LPT;
   constexpr int STEP = kWarps * TPW;
-  constexpr int WPT = HD / 8;   // code words per token
+  constexpr int VPT = HD / 32;  // 16-byte code vectors per token
   constexpr int PPT = HD / G;   // params per token
-  extern __shared__ float smem[];  // [chunk_len] scores, then reduction scratch
-  float* sc = smem;
-  __shared__ float red[kWarps][HD];
-  __shared__ float red2[2][kWarps];
+  constexpr int U = 2;          // token steps in flight per lane
+  __shared__ float red_v[kWarps][HD];
+  __shared__ float red_ml[kWarps][2];
 
   const int b = blockIdx.z, head = blockIdx.y, chunk = blockIdx.x;
   const int t0 = chunk * chunk_len;
   const int t1 = min(S, t0 + chunk_len);
-  const int n = t1 - t0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane % LPT, slot = lane / LPT;
-  const int d0 = sub * 8;
+  const int d0 = sub * 32;
 
-  // query slice, pre-scaled so that scores are in log2 units
-  float qf[8];
+  // query slice (32 dims), pre-scaled so scores are in log2 units
+  float qf[32];
   {
-    const uint4 raw = *reinterpret_cast<const uint4*>(q + int64_t(b) * q_stride + head * HD + d0);
-    const __half2* h = reinterpret_cast<const __half2*>(&raw);
+    const uint4* qp = reinterpret_cast<const uint4*>(q + int64_t(b) * q_stride + head * HD + d0);
     const float scale = kLog2e * rsqrtf(float(HD));
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float2 f = __half22float2(h[j]);
-      qf[2 * j] = f.x * scale;
-      qf[2 * j + 1] = f.y * scale;
+    for (int v = 0; v < 4; ++v) {
+      const uint4 raw = qp[v];
+      const __half2* h = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __half22float2(h[j]);
+        qf[8 * v + 2 * j] = f.x * scale;
+        qf[8 * v + 2 * j + 1] = f.y * scale;
+      }
     }
   }
   float qs = 0.f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) qs += qf[i];
+  for (int i = 0; i < 32; ++i) qs += qf[i];
 
   const int64_t slot0 = (int64_t(b) * nh + head) * cap;
-  const uint32_t* kw = kc + slot0 * WPT + sub;
-  const uint32_t* vw = vc + slot0 * WPT + sub;
+  const uint4* kw = kc + slot0 * VPT + sub;
+  const uint4* vw = vc + slot0 * VPT + sub;
   const __half2* kpp = kp + slot0 * PPT + d0 / G;
   const __half2* vpp = vp + slot0 * PPT + d0 / G;
 
-  // ---------------- pass 1: scores
-  for (int tb = t0 + warp * TPW; tb < t1; tb += STEP * kUnroll) {
-    uint32_t w[kUnroll];
-    __half2 p[kUnroll];
+  float m = -INFINITY, l = 0.f, accb = 0.f, accm = 0.f;
+  float acc[32];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+  for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+
+  for (int tb = t0 + warp * TPW; tb < t1; tb += STEP * U) {
+    uint4 kq[U], vq[U];
+    __half2 kpar[U], vpar[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
       const int t = tb + u * STEP + slot;
       const bool ok = t < t1;
-      w[u] = ok ? __ldg(kw + int64_t(t) * WPT) : 0u;
-      p[u] = ok ? __ldg(kpp + int64_t(t) * PPT) : __half2();
+      kq[u] = ok ? ldg_v4(kw + int64_t(t) * VPT) : make_uint4(0, 0, 0, 0);
+      vq[u] = ok ? ldg_v4(vw + int64_t(t) * VPT) : make_uint4(0, 0, 0, 0);
+      kpar[u] = ok ? __ldg(kpp + int64_t(t) * PPT) : __half2();
+      vpar[u] = ok ? __ldg(vpp + int64_t(t) * PPT) : __half2();
     }
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int t = tb + u * STEP + slot;
-      float f[8];
-      code_floats(w[u], f);
+    for (int u = 0; u < U; ++u) {
+      const bool ok = tb + u * STEP + slot < t1;
+      // score partial over this lane's 32 dims: s*sum(q code) + mn*sum(q)
       float dot = 0.f;
+      {
+        const uint32_t wv[4] = {kq[u].x, kq[u].y, kq[u].z, kq[u].w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) dot = fmaf(qf[i], f[i], dot);
-      const float2 ms = __half22float2(p[u]);  // {mn, s}
-      const float cq = (dot - 0.5f * qs) * 256.f;
-      float part = fmaf(ms.y, cq, ms.x * qs);
+        for (int v = 0; v < 4; ++v) {
+          float f[8];
+          code_floats(wv[v], f);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) dot = fmaf(qf[8 * v + i], f[i], dot);
+        }
+      }
+      const float2 km = __half22float2(kpar[u]);  // {mn, s}
+      float part = fmaf(km.y, (dot - 0.5f * qs) * 256.f, km.x * qs);
 #pragma unroll
       for (int o = 1; o < LPT; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-      if (sub == 0 && t < t1) sc[t - t0] = part;
-    }
-  }
-  __syncthreads();
-
-  // ---------------- softmax over the chunk
-  float m = -INFINITY;
-  for (int i = threadIdx.x; i < n; i += kThreads) m = fmaxf(m, sc[i]);
-  m = warp_max(m);
-  if (lane == 0) red2[0][warp] = m;
-  __syncthreads();
-  m = red2[0][0];
+      if (!ok) continue;
+      if (part > m) {  // new running max for this slot: rescale its sums
+        const float sc = exp2f(m - part);  // m = -inf -> 0
+        l *= sc;
+        accb *= sc;
+        accm *= sc;
 #pragma unroll
-  for (int i = 1; i < kWarps; ++i) m = fmaxf(m, red2[0][i]);
-  float l = 0.f;
-  for (int i = threadIdx.x; i < n; i += kThreads) {
-    const float e = exp2f(sc[i] - m);
-    sc[i] = e;
-    l += e;
-  }
-  l = warp_sum(l);
-  if (lane == 0) red2[1][warp] = l;
-  __syncthreads();
-  l = 0.f;
-#pragma unroll
-  for (int i = 0; i < kWarps; ++i) l += red2[1][i];
-
-  // ---------------- pass 2: weighted sum of V
-  float acc[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  float accb = 0.f, accm = 0.f;
-  for (int tb = t0 + warp * TPW; tb < t1; tb += STEP * kUnroll) {
-    uint32_t w[kUnroll];
-    __half2 p[kUnroll];
-    float pt[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int t = tb + u * STEP + slot;
-      const bool ok = t < t1;
-      w[u] = ok ? __ldg(vw + int64_t(t) * WPT) : 0u;
-      p[u] = ok ? __ldg(vpp + int64_t(t) * PPT) : __half2();
-      pt[u] = ok ? sc[t - t0] : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      float f[8];
-      code_floats(w[u], f);
-      const float2 ms = __half22float2(p[u]);
-      const float bt = pt[u] * ms.y;
-      accm = fmaf(pt[u], ms.x, accm);
+        for (int i = 0; i < 32; ++i) acc[i] *= sc;
+        m = part;
+      }
+      const float p = exp2f(part - m);
+      l += p;
+      const float2 vm = __half22float2(vpar[u]);
+      const float bt = p * vm.y;
+      accm = fmaf(p, vm.x, accm);
       accb += bt;
+      const uint32_t wv[4] = {vq[u].x, vq[u].y, vq[u].z, vq[u].w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = fmaf(bt, f[i], acc[i]);
+      for (int v = 0; v < 4; ++v) {
+        float f[8];
+        code_floats(wv[v], f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[8 * v + i] = fmaf(bt, f[i], acc[8 * v + i]);
+      }
     }
   }
-  float vals[8];
+
+  // sum_t p_t (mn_t + s_t c_td) = accm + 256 (acc_d - 0.5 accb), then merge the slots of the warp
+  float M = m;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    float v = fmaf(256.f, acc[i] - 0.5f * accb, accm);
-    // sum over the token slots of this warp (lanes with equal `sub`)
+  for (int o = LPT; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float sc = (m == -INFINITY) ? 0.f : exp2f(m - M);
+  float lw = l * sc;
+#pragma unroll
+  for (int o = LPT; o < 32; o <<= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+  const float base = accm * sc;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    float v = fmaf(256.f * sc, acc[i] - 0.5f * accb, base);
 #pragma unroll
     for (int o = LPT; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    vals[i] = v;
+    if (slot == 0) red_v[warp][d0 + i] = v;
   }
-  if (slot == 0) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) red[warp][d0 + i] = vals[i];
+  if (lane == 0) {
+    red_ml[warp][0] = M;
+    red_ml[warp][1] = lw;
   }
   __syncthreads();
+  // merge the warps
+  float Mc = red_ml[0][0];
+#pragma unroll
+  for (int w = 1; w < kWarps; ++w) Mc = fmaxf(Mc, red_ml[w][0]);
+  float wsc[kWarps];
+  float L = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    wsc[w] = (red_ml[w][0] == -INFINITY) ? 0.f : exp2f(red_ml[w][0] - Mc);
+    L = fmaf(red_ml[w][1], wsc[w], L);
+  }
   const int64_t bh = int64_t(b) * nh + head;
   for (int d = threadIdx.x; d < HD; d += kThreads) {
     float v = 0.f;
 #pragma unroll
-    for (int i = 0; i < kWarps; ++i) v += red[i][d];
+    for (int w = 0; w < kWarps; ++w) v = fmaf(red_v[w][d], wsc[w], v);
     if (part_ml == nullptr) {
-      out[int64_t(b) * nh * HD + head * HD + d] = __float2half_rn(v / l);
+      out[int64_t(b) * nh * HD + head * HD + d] = __float2half_rn(v / L);
     } else {
       part_acc[(bh * gridDim.x + chunk) * HD + d] = v;
     }
   }
   if (part_ml != nullptr && threadIdx.x == 0) {
-    part_ml[(bh * gridDim.x + chunk) * 2 + 0] = m;
-    part_ml[(bh * gridDim.x + chunk) * 2 + 1] = l;
+    part_ml[(bh * gridDim.x + chunk) * 2 + 0] = Mc;
+    part_ml[(bh * gridDim.x + chunk) * 2 + 1] = L;
   }
 }
 
@@ -250,8 +253,8 @@ int pick_chunks(int B, int nh, int S) {
   int nc = (target + bh - 1) / bh;
   const int max_by_len = (S + 127) / 128;  // at least 128 positions per chunk
   nc = std::min(nc, std::max(1, max_by_len));
-  const int min_by_smem = (S + 4095) / 4096;  // at most 4096 positions per chunk
-  return std::max(nc, std::max(1, min_by_smem));
+  const int min_by_len = (S + 4095) / 4096;  // at most 4096 positions per chunk
+  return std::max(nc, std::max(1, min_by_len));
 }
 
 }  // namespace
@@ -290,10 +293,10 @@ int decode_attention_impl(const void* q, int64_t q_stride, const fg_kv_cache* c,
   const double bytes = double(B) * nh * S * 2.0 * (hd / 2 + 4.0 * hd / G) + 4.0 * B * nh * hd;
   ProfScope ps(PROF_DECODE_ATTN, s, 4.0 * B * nh * double(S) * hd, bytes);
   dim3 grid(nc, nh, B);
-  const size_t smem = size_t(chunk_len) * sizeof(float);
+  const size_t smem = 0;
   auto* qh = reinterpret_cast<const __half*>(q);
-  auto* kc = reinterpret_cast<const uint32_t*>(c->k_codes);
-  auto* vc = reinterpret_cast<const uint32_t*>(c->v_codes);
+  auto* kc = reinterpret_cast<const uint4*>(c->k_codes);
+  auto* vc = reinterpret_cast<const uint4*>(c->v_codes);
   auto* kp = reinterpret_cast<const __half2*>(c->k_params);
   auto* vp = reinterpret_cast<const __half2*>(c->v_params);
   auto* o = reinterpret_cast<__half*>(out);

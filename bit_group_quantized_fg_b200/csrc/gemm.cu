@@ -47,13 +47,24 @@ constexpr int kParamBytesMax = BK * 8 * 4;  // up to 8 half2 per k row (G = 32)
 
 enum BMode { B_Q4 = 0, B_F16_MN = 1, B_F16_K = 2 };
 
+// Shared memory: a ring of TMA stages, then (4-bit mode) a ring of expanded fp16 B tiles.
+// 4-bit mode: TMA stage = X tile + code tile + param tile (26 KB), 6 deep, so that the loads
+// run far enough ahead of the tensor cores to cover their latency; the dequant warps fill a
+// separate 2-deep ring of 32 KB fp16 B tiles.  fp16 modes: TMA stage = X tile + B tile, 4 deep.
 template <int MODE>
 struct Cfg {
-  static constexpr int kStages = MODE == B_Q4 ? 3 : 4;
-  static constexpr int kStageBytes = kABytes + kBBytes + (MODE == B_Q4 ? kCodeBytes + kParamBytesMax : 0);
-  static constexpr int kDequantWarps = MODE == B_Q4 ? 8 : 0;
+  static constexpr bool kQ4 = MODE == B_Q4;
+  static constexpr int kStages = kQ4 ? 6 : 4;
+  static constexpr int kCodeOff = kABytes;
+  static constexpr int kParamOff = kABytes + kCodeBytes;
+  static constexpr int kStageBytes = kQ4 ? kABytes + kCodeBytes + kParamBytesMax : kABytes + kBBytes;
+  static constexpr int kBStages = kQ4 ? 2 : 0;
+  static constexpr int kBRingOff = kStages * kStageBytes;
+  static constexpr int kDequantWarps = kQ4 ? 8 : 0;
   static constexpr int kThreads = 256 + kDequantWarps * 32;
-  static constexpr int kSmem = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int kSmem = kBRingOff + kBStages * kBBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static_assert(kBRingOff % 1024 == 0 && kStageBytes % 1024 == 0, "1024-byte aligned operand tiles");
+  static_assert(kSmem <= 232448, "shared memory budget");
 };
 
 struct GemmArgs {
@@ -98,15 +109,18 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base_u32 = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024 - (base_u32 & 1023)) & 1023);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
-  uint64_t* full = bars;              // [S] TMA landed
-  uint64_t* bfull = bars + S;         // [S] dequant wrote B (4-bit mode)
-  uint64_t* empty = bars + 2 * S;     // [S] MMA finished reading the stage
-  uint64_t* acc_full = bars + 3 * S;  // [2]
-  uint64_t* acc_empty = bars + 3 * S + 2;  // [2]
-  uint64_t* drain = bars + 3 * S + 4;      // [1] MMA drain on abort
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 3 * S + 6);
+  constexpr int SB = 2;  // B-ring depth (4-bit mode)
+  uint8_t* bring = smem + C::kBRingOff;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBRingOff + C::kBStages * kBBytes);
+  uint64_t* full = bars;                   // [S]  TMA stage landed
+  uint64_t* empty = bars + S;              // [S]  MMA finished reading the TMA stage
+  uint64_t* bfull = bars + 2 * S;          // [SB] dequant wrote a B tile
+  uint64_t* bempty = bars + 2 * S + SB;    // [SB] MMA finished reading a B tile
+  uint64_t* acc_full = bars + 2 * S + 2 * SB;       // [2]
+  uint64_t* acc_empty = bars + 2 * S + 2 * SB + 2;  // [2]
+  uint64_t* drain = bars + 2 * S + 2 * SB + 4;      // [1] MMA drain on abort
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * SB + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * S + 2 * SB + 6);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -114,8 +128,11 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&bfull[i], C::kDequantWarps > 0 ? C::kDequantWarps : 1);
       mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < SB; ++i) {
+      mbar_init(&bfull[i], C::kDequantWarps > 0 ? C::kDequantWarps : 1);
+      mbar_init(&bempty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&acc_full[i], 1);
@@ -155,9 +172,9 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
           mbar_expect_tx(&full[stage], tx);
           tma_load_2d(st, &tm_a, kb * BK, c.m0, &full[stage]);
           if (MODE == B_Q4) {
-            tma_load_2d(st + kABytes + kBBytes, &tm_b, c.n0 / 2, kb * BK, &full[stage]);
+            tma_load_2d(st + C::kCodeOff, &tm_b, c.n0 / 2, kb * BK, &full[stage]);
             const int px = (c.n0 / args.G) & ~3;
-            tma_load_2d(st + kABytes + kBBytes + kCodeBytes, &tm_p, px, kb * BK, &full[stage]);
+            tma_load_2d(st + C::kParamOff, &tm_p, px, kb * BK, &full[stage]);
           } else if (MODE == B_F16_MN) {
 #pragma unroll
             for (int j = 0; j < BN / 64; ++j)
@@ -180,8 +197,8 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16_f32(BM, BN, MODE != B_F16_K);
-      int stage = 0;
-      uint32_t phase = 0;
+      int stage = 0, bs = 0;
+      uint32_t phase = 0, bphase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
@@ -192,10 +209,10 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
         const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
         for (int kb = c.kb0; kb < c.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, &g_device_error, 4)) { ok = false; break; }
-          if (MODE == B_Q4 && !mbar_wait(&bfull[stage], phase, abort_flag, &g_device_error, 8)) { ok = false; break; }
+          if (MODE == B_Q4 && !mbar_wait(&bfull[bs], bphase, abort_flag, &g_device_error, 8)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + stage * C::kStageBytes);
-          const uint32_t b_addr = a_addr + kABytes;
+          const uint32_t b_addr = MODE == B_Q4 ? smem_u32(bring + bs * kBBytes) : a_addr + kABytes;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t ad = smem_desc_sw128(a_addr + k * 32, 16, 1024);
@@ -206,6 +223,10 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
           }
           mma_commit(&empty[stage]);
           if (++stage == S) { stage = 0; phase ^= 1; }
+          if (MODE == B_Q4) {
+            mma_commit(&bempty[bs]);
+            if (++bs == SB) { bs = 0; bphase ^= 1; }
+          }
         }
         if (!ok) break;
         mma_commit(&acc_full[acc]);
@@ -232,6 +253,18 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
         uint32_t r[32];
         tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + cc), r);
         tmem_ld_wait();
+        if (MODE == B_Q4) {
+          // the dequant warps stored each 8 columns in the order [0,4,1,5,2,6,3,7]:
+          // natural column j of a group sits at position (j < 4 ? 2j : 2(j-4)+1)
+          uint32_t t[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int jj = j & 7;
+            t[j] = r[(j & ~7) + (jj < 4 ? 2 * jj : 2 * (jj - 4) + 1)];
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) r[j] = t[j];
+        }
         const int n = c.n0 + cc;
         if (!row_ok || n >= args.N) continue;
         if (args.partial != nullptr) {
@@ -311,8 +344,8 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
     const int dw = warp - 8;       // 0..7: k rows dw, dw+8, ..., dw+56
     const int nb = lane >> 3;      // 64-wide MN block of the word
     const int ch = lane & 7;       // 16-byte chunk inside the block
-    int stage = 0;
-    uint32_t phase = 0;
+    int stage = 0, bs = 0;
+    uint32_t phase = 0, bphase = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < args.total && ok; t += gridDim.x) {
       const TileCoord c = tile_coord(args, t);
@@ -320,10 +353,9 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
       const int pcol = poff + (lane * 8) / args.G;
       for (int kb = c.kb0; kb < c.kb1; ++kb) {
         if (!mbar_wait(&full[stage], phase, abort_flag, &g_device_error, 32)) { ok = false; break; }
-        uint8_t* st = smem + stage * C::kStageBytes;
-        const uint32_t* codes = reinterpret_cast<const uint32_t*>(st + kABytes + kBBytes);
-        const uint32_t* prm = reinterpret_cast<const uint32_t*>(st + kABytes + kBBytes + kCodeBytes);
-        uint8_t* bt = st + kABytes;
+        const uint8_t* st = smem + stage * C::kStageBytes;
+        const uint32_t* codes = reinterpret_cast<const uint32_t*>(st + C::kCodeOff);
+        const uint32_t* prm = reinterpret_cast<const uint32_t*>(st + C::kParamOff);
         uint32_t w[8], p[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -331,20 +363,27 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
           w[i] = codes[row * (BN / 8) + lane];
           p[i] = prm[row * args.PB + pcol];
         }
+        uint32_t o[8][4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const __half2 pr = u32_as_h2(p[i]);
+          dequant8_interleaved(w[i], __high2half2(pr), __low2half2(pr), o[i]);
+        }
+        // the B tile this k-block fills must have been consumed by the MMA two blocks ago
+        if (!mbar_wait(&bempty[bs], bphase ^ 1, abort_flag, &g_device_error, 64)) { ok = false; break; }
+        uint8_t* bt = bring + bs * kBBytes;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int row = dw + 8 * i;  // k index inside the block
-          const __half2 pr = u32_as_h2(p[i]);
-          uint32_t o[4];
-          dequant8(w[i], __high2half2(pr), __low2half2(pr), o);
           const int kg = row >> 3, rr = row & 7;
           uint4* dst = reinterpret_cast<uint4*>(bt + nb * 8192 + kg * 1024 + rr * 128 + ((ch ^ rr) << 4));
-          *dst = make_uint4(o[0], o[1], o[2], o[3]);
+          *dst = make_uint4(o[i][0], o[i][1], o[i][2], o[i][3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bfull[stage]);
+        if (lane == 0) mbar_arrive(&bfull[bs]);
         if (++stage == S) { stage = 0; phase ^= 1; }
+        if (++bs == SB) { bs = 0; bphase ^= 1; }
       }
     }
   }

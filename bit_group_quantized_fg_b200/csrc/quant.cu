@@ -32,30 +32,24 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
 }
 
 struct GroupQ {
-  uint32_t word;  // 8 packed codes
-  __half2 params; // {mn, s}
+  uint2 words;     // 16 packed codes (element i in bits 4i..4i+3 of words.x, then words.y)
+  __half2 params;  // {mn, s}
 };
 
-// Quantize the 8 values of `v` as part of a group spread over TPG adjacent lanes.
-// Every lane of the warp must call this (shuffles use the full mask).
+// Quantize 16 consecutive values (two 16-byte vectors) that are part of a group spread over
+// TPG = G/16 adjacent lanes.  Every lane of the warp must call this (full-mask shuffles).
+// min/max run on packed fp16 (comparisons are exact); the scale and the reciprocal are
+// computed once per 16 values.
 template <int TPG>
-__device__ __forceinline__ GroupQ quantize_chunk(uint4 v) {
-  float x[8];
-  {
-    const __half2* h = reinterpret_cast<const __half2*>(&v);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float2 f = __half22float2(h[j]);
-      x[2 * j] = f.x;
-      x[2 * j + 1] = f.y;
-    }
-  }
-  float mn = x[0], mx = x[0];
-#pragma unroll
-  for (int i = 1; i < 8; ++i) {
-    mn = fminf(mn, x[i]);
-    mx = fmaxf(mx, x[i]);
-  }
+__device__ __forceinline__ GroupQ quantize_chunk16(uint4 a, uint4 b) {
+  const __half2* ha = reinterpret_cast<const __half2*>(&a);
+  const __half2* hb = reinterpret_cast<const __half2*>(&b);
+  __half2 lo = __hmin2(__hmin2(ha[0], ha[1]), __hmin2(ha[2], ha[3]));
+  __half2 hi = __hmax2(__hmax2(ha[0], ha[1]), __hmax2(ha[2], ha[3]));
+  lo = __hmin2(lo, __hmin2(__hmin2(hb[0], hb[1]), __hmin2(hb[2], hb[3])));
+  hi = __hmax2(hi, __hmax2(__hmax2(hb[0], hb[1]), __hmax2(hb[2], hb[3])));
+  float mn = fminf(__low2float(lo), __high2float(lo));
+  float mx = fmaxf(__low2float(hi), __high2float(hi));
 #pragma unroll
   for (int o = 1; o < TPG; o <<= 1) {
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
@@ -63,46 +57,62 @@ __device__ __forceinline__ GroupQ quantize_chunk(uint4 v) {
   }
   mn = __fadd_rn(mn, 0.0f);  // -0 -> +0
   mx = __fadd_rn(mx, 0.0f);
-  const float d = __fsub_rn(mx, mn);
-  const __half s16 = __float2half_rn(__fdiv_rn(d, 15.0f));
+  const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
   const float sf = __half2float(s16);
   const bool zero = (sf == 0.0f);
   const float den = zero ? 1.0f : sf;
-  uint32_t word = 0;
+  // The code is rint of r = RN(d / s).  r1 = RN(d * RN(1/s)) differs from r by less than
+  // 1.5 * 2^-23 * |r| < 2^-18 (r < 16), so rint(r1) == rint(r) unless r1 lies within 2^-18 of
+  // a half-integer; inside the wider 2^-17 window the exact IEEE quotient is used instead.
+  // rint is taken by adding 1.5 * 2^23 (for 0 <= r1 < 2^22 the sum's ulp is 1, so the add
+  // rounds half to even and the low mantissa bits hold the integer).
+  const float rcp = __frcp_rn(den);
+  const float kMagic = 12582912.0f;  // 1.5 * 2^23
+  uint32_t w[2] = {0u, 0u};
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    int q = __float2int_rn(__fdiv_rn(__fsub_rn(x[i], mn), den));
-    q = q < 0 ? 0 : (q > 15 ? 15 : q);
+  for (int i = 0; i < 16; ++i) {
+    const __half2 pr = (i < 8) ? ha[i / 2] : hb[(i - 8) / 2];
+    const float x = (i & 1) ? __high2float(pr) : __low2float(pr);
+    const float d = __fsub_rn(x, mn);
+    const float r1 = __fmul_rn(d, rcp);
+    const float t = __fadd_rn(r1, kMagic);
+    int q = __float_as_int(t) - __float_as_int(kMagic);
+    if (fabsf(__fsub_rn(r1, __fsub_rn(t, kMagic))) > 0.5f - 7.62939453125e-06f)  // 2^-17
+      q = __float2int_rn(__fdiv_rn(d, den));
+    q = q > 15 ? 15 : q;  // r >= 0, so q >= 0
     if (zero) q = 0;
-    word |= uint32_t(q) << (4 * i);
+    w[i / 8] |= uint32_t(q) << (4 * (i % 8));
   }
   GroupQ r;
-  r.word = word;
+  r.words = make_uint2(w[0], w[1]);
   r.params = __halves2half2(__float2half_rn(mn), s16);
   return r;
 }
 
 // ------------------------------------------------------------------ K1, axis = 1
+// One thread per 16 consecutive elements (a "chunk"); G/16 lanes per group.
 template <int G>
 __global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const uint4* __restrict__ x,
                                                                  int64_t n_chunks,
-                                                                 uint32_t* __restrict__ codes,
+                                                                 uint2* __restrict__ codes,
                                                                  __half2* __restrict__ params) {
-  constexpr int TPG = G / 8;
+  constexpr int TPG = G / 16;
   const int64_t tile = int64_t(kThreads) * kUnroll;
   for (int64_t base = int64_t(blockIdx.x) * tile; base < n_chunks; base += int64_t(gridDim.x) * tile) {
-    uint4 v[kUnroll];
+    uint4 va[kUnroll], vb[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int64_t c = base + u * kThreads + threadIdx.x;
-      v[u] = c < n_chunks ? ld_nc_v4(x + c) : make_uint4(0, 0, 0, 0);
+      const bool ok = c < n_chunks;
+      va[u] = ok ? ld_nc_v4(x + 2 * c) : make_uint4(0, 0, 0, 0);
+      vb[u] = ok ? ld_nc_v4(x + 2 * c + 1) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int64_t c = base + u * kThreads + threadIdx.x;
-      GroupQ q = quantize_chunk<TPG>(v[u]);
+      GroupQ q = quantize_chunk16<TPG>(va[u], vb[u]);
       if (c < n_chunks) {
-        codes[c] = q.word;
+        codes[c] = q.words;
         if ((threadIdx.x % TPG) == 0) params[c / TPG] = q.params;
       }
     }
@@ -110,47 +120,51 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const uint4* __
 }
 
 // ------------------------------------------------------------------ KV append
-// Rows r = b*T + t of k (blockIdx.y == 0) or v (== 1); h valid values per row.
-// Group g of head `hd`-slice lands at cache position len + t.
+// Rows r = b*T + t of k (blockIdx.y == 0) or v (== 1); h valid values per row, quantized in
+// chunks of 16 along the hidden dimension.  The group of head `head` lands at cache
+// position pos0 + t.
 template <int G>
 __global__ void __launch_bounds__(kThreads) kv_append_kernel(
     const __half* __restrict__ k, const __half* __restrict__ v, int64_t row_stride, int T, int h,
-    int hd, int cap, int pos0, int64_t n_chunks, uint32_t* __restrict__ kc, uint32_t* __restrict__ vc,
+    int hd, int cap, int pos0, int64_t n_chunks, uint2* __restrict__ kc, uint2* __restrict__ vc,
     __half2* __restrict__ kp, __half2* __restrict__ vp) {
-  constexpr int TPG = G / 8;
+  constexpr int TPG = G / 16;
   const __half* src = blockIdx.y == 0 ? k : v;
-  uint32_t* dc = blockIdx.y == 0 ? kc : vc;
+  uint2* dc = blockIdx.y == 0 ? kc : vc;
   __half2* dp = blockIdx.y == 0 ? kp : vp;
-  const int chunks_per_row = h / 8;
+  const int chunks_per_row = h / 16;
   const int nh = h / hd;
   const int64_t tile = int64_t(kThreads) * kUnroll;
   for (int64_t base = int64_t(blockIdx.x) * tile; base < n_chunks; base += int64_t(gridDim.x) * tile) {
-    uint4 val[kUnroll];
+    uint4 va[kUnroll], vb[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int64_t c = base + u * kThreads + threadIdx.x;
       if (c < n_chunks) {
         const int64_t row = c / chunks_per_row;
         const int cc = int(c - row * chunks_per_row);
-        val[u] = ld_nc_v4(src + row * row_stride + cc * 8);
+        const uint4* p = reinterpret_cast<const uint4*>(src + row * row_stride + cc * 16);
+        va[u] = ld_nc_v4(p);
+        vb[u] = ld_nc_v4(p + 1);
       } else {
-        val[u] = make_uint4(0, 0, 0, 0);
+        va[u] = make_uint4(0, 0, 0, 0);
+        vb[u] = va[u];
       }
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int64_t c = base + u * kThreads + threadIdx.x;
-      GroupQ q = quantize_chunk<TPG>(val[u]);
+      GroupQ q = quantize_chunk16<TPG>(va[u], vb[u]);
       if (c < n_chunks) {
         const int64_t row = c / chunks_per_row;
         const int cc = int(c - row * chunks_per_row);
         const int64_t b = row / T;
         const int t = int(row - b * T);
-        const int d = cc * 8;
+        const int d = cc * 16;
         const int head = d / hd;
         const int dh = d - head * hd;
         const int64_t slot = (b * nh + head) * int64_t(cap) + (pos0 + t);
-        dc[slot * (hd / 8) + dh / 8] = q.word;
+        dc[slot * (hd / 16) + dh / 16] = q.words;
         if ((threadIdx.x % TPG) == 0) dp[slot * (hd / G) + dh / G] = q.params;
       }
     }
@@ -291,10 +305,10 @@ int quantize_pack_impl(const void* x, int64_t rows, int64_t cols, int group, int
   if (n == 0) return FG_OK;
   ProfScope ps(PROF_QUANT, s, 0.0, double(n) * (2.0 + 0.5 + 4.0 / group));
   if (axis == 1) {
-    const int64_t chunks = n / 8;
+    const int64_t chunks = n / 16;
     const int grid = grid_for(chunks, int64_t(kThreads) * kUnroll);
     auto* xin = reinterpret_cast<const uint4*>(x);
-    auto* cw = reinterpret_cast<uint32_t*>(codes);
+    auto* cw = reinterpret_cast<uint2*>(codes);
     auto* pw = reinterpret_cast<__half2*>(params);
     if (group == 32) quantize_rows_kernel<32><<<grid, kThreads, 0, s>>>(xin, chunks, cw, pw);
     else if (group == 64) quantize_rows_kernel<64><<<grid, kThreads, 0, s>>>(xin, chunks, cw, pw);
@@ -350,13 +364,13 @@ int kv_append_impl(fg_kv_cache* c, const void* k, const void* v, int64_t row_str
       !aligned16(c->k_params) || !aligned16(c->v_params))
     return fail(FG_ERR_ALIGN, "pointers must be 16-byte aligned");
   if (n_tokens == 0) return FG_OK;
-  const int64_t chunks = int64_t(c->B) * n_tokens * (h / 8);
-  ProfScope ps(PROF_QUANT, s, 0.0, double(chunks) * 8 * 2 * (2.0 + 0.5 + 4.0 / G));
+  const int64_t chunks = int64_t(c->B) * n_tokens * (h / 16);
+  ProfScope ps(PROF_QUANT, s, 0.0, double(chunks) * 16 * 2 * (2.0 + 0.5 + 4.0 / G));
   dim3 grid(unsigned(grid_for(chunks, int64_t(kThreads) * kUnroll)), 2);
   auto* K = reinterpret_cast<const __half*>(k);
   auto* V = reinterpret_cast<const __half*>(v);
-  auto* kc = reinterpret_cast<uint32_t*>(c->k_codes);
-  auto* vc = reinterpret_cast<uint32_t*>(c->v_codes);
+  auto* kc = reinterpret_cast<uint2*>(c->k_codes);
+  auto* vc = reinterpret_cast<uint2*>(c->v_codes);
   auto* kp = reinterpret_cast<__half2*>(c->k_params);
   auto* vp = reinterpret_cast<__half2*>(c->v_params);
   if (G == 32)

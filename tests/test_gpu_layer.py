@@ -160,3 +160,25 @@ def test_generate_small_model(fg):
     out2, _ = fg.fg_generate(md, to_dev(ids[[3, 1]]), T, caches2)
     torch.cuda.synchronize()
     assert compare_tokens(to_np(out2), exp[[3, 1]], logits[:, [3, 1]]) >= 0.99
+
+
+def test_generate_graph_replay_matches_eager(fg):
+    """The first call runs eagerly, the second records CUDA graphs, the third replays them:
+    all three produce the same tokens and leave the caches at length L + T - 1."""
+    import torch
+    mo, md = small_model(fg, seed=8, n_layers=1)
+    B, L, T = 3, 12, 6
+    ids = to_dev(fg_synth.token_ids(8, fg_synth.S_IDS, (B, L), mo.vocab))
+    caches = [fg.DeviceKVCache(B, mo.n_heads, mo.head_dim, L + T, 64) for _ in range(mo.n_layers)]
+    out = torch.empty((B, T), dtype=torch.int32, device="cuda")
+    ws = torch.empty((fg.fg_workspace_bytes(md, B, L, T),), dtype=torch.uint8, device="cuda")
+    results = []
+    for _ in range(3):
+        out.fill_(-1)
+        n0 = fg.fg_launch_count()
+        fg.fg_generate(md, ids, T, caches, out_ids=out, workspace=ws)
+        torch.cuda.synchronize()
+        results.append((to_np(out).copy(), fg.fg_launch_count() - n0))
+        assert all(c.length == L + T - 1 for c in caches)
+    assert np.array_equal(results[0][0], results[1][0]) and np.array_equal(results[0][0], results[2][0])
+    assert results[0][1] == results[1][1] == results[2][1] > 0   # same kernels, counted once each
