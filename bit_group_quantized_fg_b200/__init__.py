@@ -67,6 +67,8 @@ _SIGS = {
     "fg_qgemm_workspace_bytes": (c_size_t, [c_int64, c_int, c_int]),
     "fg_qgemm": (c_int, [c_void_p, c_int64, POINTER(QLinear), c_void_p, c_int, c_void_p, c_void_p, c_size_t,
                          c_void_p]),
+    "fg_gemm_f16": (c_int, [c_void_p, c_int64, c_void_p, c_int, c_int, c_void_p, c_void_p, c_int, c_void_p,
+                            c_void_p, c_size_t, c_void_p]),
     "fg_decode_attention_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int]),
     "fg_decode_attention": (c_int, [c_void_p, c_int64, POINTER(KVCache), c_void_p, c_void_p, c_size_t,
                                     c_void_p]),
@@ -229,6 +231,21 @@ def fg_qgemm(X, W: DeviceQLinear, R=None, relu: bool = False, Y=None, workspace=
         workspace = _empty((wsb,), torch.uint8, X.device)
     _check(lib().fg_qgemm(_ptr(X), M, ctypes.byref(W.c), _ptr(R), int(relu), _ptr(Y), _ptr(workspace),
                           0 if workspace is None else workspace.numel(), _stream(stream)))
+    return Y
+
+
+def fg_gemm_f16(X, W, bias=None, R=None, relu: bool = False, Y=None, workspace=None, stream=None):
+    """Y = [relu](X @ W + b) [+ R] with an uncompressed fp16 weight W [K, N] on the tensor cores."""
+    import torch
+    M = X.shape[0]
+    K, N = W.shape
+    if Y is None:
+        Y = _empty((M, N), torch.float16, X.device)
+    wsb = fg_qgemm_workspace_bytes(M, N, K)
+    if workspace is None and wsb:
+        workspace = _empty((wsb,), torch.uint8, X.device)
+    _check(lib().fg_gemm_f16(_ptr(X), M, _ptr(W), K, N, _ptr(bias), _ptr(R), int(relu), _ptr(Y), _ptr(workspace),
+                             0 if workspace is None else workspace.numel(), _stream(stream)))
     return Y
 
 

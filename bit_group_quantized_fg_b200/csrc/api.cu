@@ -161,8 +161,19 @@ int check_layer(const fg_layer* L, int h, int* ffn) {
   return FG_OK;
 }
 
+// Y = [relu](X W_hat + b) [+ R] for a 4-bit weight.  With many rows (a prompt pass) each
+// weight tile is reused by M/128 row tiles, so the weight is first expanded once into an
+// fp16 copy in the workspace (an HBM-bound pass, ~1 % of the GEMM) and the tensor-core GEMM
+// then runs without dequant warps; with few rows (decode) the fused kernel reads the 4-bit
+// weight directly, once.  Both compute with the same fp16 values W_hat.
 int qlinear_run(const void* X, int64_t M, const fg_qlinear& w, const void* R, int relu, void* Y, void* ws,
                 size_t wsb, cudaStream_t s) {
+  const size_t wbytes = (size_t(w.K) * size_t(w.N) * 2 + 255) & ~size_t(255);
+  if (M >= kExpandRows && ws != nullptr && wsb >= wbytes && aligned16(ws)) {
+    FG_TRY(dequantize_impl(w.codes, w.params, w.K, w.N, w.group, 1, ws, s));
+    return gemm_impl(1, X, M, w.N, w.K, ws, nullptr, 0, w.bias, R, relu, Y, false,
+                     reinterpret_cast<uint8_t*>(ws) + wbytes, wsb - wbytes, s);
+  }
   return gemm_impl(0, X, M, w.N, w.K, w.codes, w.params, w.group, w.bias, R, relu, Y, false, ws, wsb, s);
 }
 
@@ -539,6 +550,11 @@ int fg_qgemm(const void* X, int64_t M, const fg_qlinear* W, const void* R, int r
              size_t ws_bytes, void* stream) {
   if (!W) return fail(FG_ERR_INVALID_ARG, "null weight");
   return qlinear_run(X, M, *W, R, relu, Y, workspace, ws_bytes, as_stream(stream));
+}
+
+int fg_gemm_f16(const void* X, int64_t M, const void* W, int K, int N, const void* bias, const void* R, int relu,
+                void* Y, void* workspace, size_t ws_bytes, void* stream) {
+  return gemm_impl(1, X, M, N, K, W, nullptr, 0, bias, R, relu, Y, false, workspace, ws_bytes, as_stream(stream));
 }
 
 size_t fg_decode_attention_workspace_bytes(int B, int n_heads, int head_dim, int ctx) {

@@ -42,6 +42,10 @@ inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s
 
 int num_sms();
 
+// Row count from which a 4-bit GEMM expands its weight to fp16 once and runs the plain
+// fp16 tensor-core GEMM (measured break-even ~700 rows on B200).
+constexpr int64_t kExpandRows = 1024;
+
 // Kernel classes for fg_profile_* (same numbering as the header).
 enum ProfKind { PROF_GEMM = 0, PROF_DECODE_ATTN = 1, PROF_PREFILL_ATTN = 2, PROF_QUANT = 3,
                 PROF_OTHER = 4, PROF_GEMM_DECODE = 5, PROF_LM_HEAD = 6, PROF_NKINDS = 7 };

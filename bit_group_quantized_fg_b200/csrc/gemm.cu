@@ -503,13 +503,23 @@ int read_device_error(int* out) {
   return cudaMemcpyFromSymbol(out, g_device_error, sizeof(int)) == cudaSuccess ? FG_OK : FG_ERR_CUDA;
 }
 
-size_t qgemm_ws_bytes(int64_t M, int N, int K) {
+// Split-K partials of one GEMM (0 when the tiles alone fill the GPU).
+size_t splitk_ws_bytes(int64_t M, int N, int K) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
   const int m_tiles = int((M + BM - 1) / BM);
   const int n_tiles = (N + BN - 1) / BN;
   const int sp = pick_splits(m_tiles * n_tiles, K / BK);
   if (sp <= 1) return 0;
   return size_t(sp) * size_t(M) * size_t(N) * sizeof(float);
+}
+
+// Workspace of a 4-bit GEMM: with M >= kExpandRows the fp16 copy of the weight, then the
+// partials (both 256-byte aligned).
+size_t qgemm_ws_bytes(int64_t M, int N, int K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  size_t w = 0;
+  if (M >= kExpandRows) w = (size_t(K) * size_t(N) * 2 + 255) & ~size_t(255);
+  return w + splitk_ws_bytes(M, N, K);
 }
 
 // mode: 0 = 4-bit weight W (codes/params), 1 = fp16 [K][N] weight, 2 = fp16 [N][K] weight.

@@ -141,6 +141,13 @@ size_t fg_qgemm_workspace_bytes(int64_t M, int N, int K);
 int fg_qgemm(const void* X, int64_t M, const fg_qlinear* W, const void* R, int relu, void* Y,
              void* workspace, size_t ws_bytes, void* stream);
 
+/* The same tensor-core GEMM over an uncompressed fp16 weight W [K][N] (N contiguous): the
+ * "FlexGen" README mirror's benchmark table contrasts FlexGen with and without compression;
+ * this is the uncompressed side.  Y[M][N] = [relu](X W + b) [+ R], fp32 accumulation.
+ * K % 64 == 0, N % 256 == 0; workspace as fg_qgemm_workspace_bytes(M, N, K). */
+int fg_gemm_f16(const void* X, int64_t M, const void* W, int K, int N, const void* bias,
+                const void* R, int relu, void* Y, void* workspace, size_t ws_bytes, void* stream);
+
 /* Decode attention over a 4-bit cache: for each sequence b and head j,
  * out = softmax(q K^T / sqrt(hd)) V over positions 0..cache->len-1, with K and V the
  * dequantized cache values (mn + code*s) and an fp32 softmax.  q: fp16, row b at

@@ -83,6 +83,20 @@ def test_qgemm_prefill_size_sampled(fg):
     assert_close_rms(got, exp, what="sampled prefill GEMM")
 
 
+@pytest.mark.parametrize("M,N,K", [(4, 256, 64), (300, 768, 320), (64, 4096, 2048)])
+def test_gemm_f16_matches_oracle(fg, M, N, K):
+    """The uncompressed fp16-weight GEMM against the float64 product of the same fp16 values."""
+    import torch
+    x = fg_synth.tensor(M, 1, (M, K), "normal", 1.0)
+    w = fg_synth.tensor(M, 2, (K, N), "normal", 0.02)
+    b = fg_synth.tensor(M, 3, (N,), "normal", 0.5)
+    r = fg_synth.tensor(M, 4, (M, N), "normal", 1.0)
+    y = fg.fg_gemm_f16(to_dev(x), to_dev(w), bias=to_dev(b), R=to_dev(r), relu=True)
+    torch.cuda.synchronize()
+    exp = np.maximum(x.astype(np.float64) @ w.astype(np.float64) + b.astype(np.float64), 0) + r.astype(np.float64)
+    assert_close_rms(to_np(y), exp.astype(np.float16), what="fp16 GEMM")
+
+
 def test_lm_head_argmax(fg):
     import torch
     B, h, V = 5, 256, 1000      # V not a multiple of the 256-wide tile
