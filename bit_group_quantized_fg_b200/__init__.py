@@ -67,6 +67,7 @@ _SIGS = {
     "fg_qgemm_workspace_bytes": (c_size_t, [c_int64, c_int, c_int]),
     "fg_qgemm": (c_int, [c_void_p, c_int64, POINTER(QLinear), c_void_p, c_int, c_void_p, c_void_p, c_size_t,
                          c_void_p]),
+    "fg_gemm_f16_workspace_bytes": (c_size_t, [c_int64, c_int, c_int]),
     "fg_gemm_f16": (c_int, [c_void_p, c_int64, c_void_p, c_int, c_int, c_void_p, c_void_p, c_int, c_void_p,
                             c_void_p, c_size_t, c_void_p]),
     "fg_decode_attention_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int]),
@@ -89,6 +90,7 @@ _SIGS = {
     "fg_generate": (c_int, [POINTER(Model), c_void_p, c_int, c_int, c_int, c_void_p, POINTER(KVCache),
                             c_void_p, c_size_t, POINTER(Timing), c_void_p]),
     "fg_profile_enable": (c_int, [c_int]),
+    "fg_profile_select": (c_int, [ctypes.c_uint]),
     "fg_profile_read": (c_int, [c_int, POINTER(c_double), POINTER(c_int64), POINTER(c_double),
                                 POINTER(c_double)]),
     "fg_profile_reset": (c_int, []),
@@ -241,7 +243,7 @@ def fg_gemm_f16(X, W, bias=None, R=None, relu: bool = False, Y=None, workspace=N
     K, N = W.shape
     if Y is None:
         Y = _empty((M, N), torch.float16, X.device)
-    wsb = fg_qgemm_workspace_bytes(M, N, K)
+    wsb = lib().fg_gemm_f16_workspace_bytes(M, N, K)
     if workspace is None and wsb:
         workspace = _empty((wsb,), torch.uint8, X.device)
     _check(lib().fg_gemm_f16(_ptr(X), M, _ptr(W), K, N, _ptr(bias), _ptr(R), int(relu), _ptr(Y), _ptr(workspace),
@@ -363,6 +365,12 @@ def fg_generate(model: DeviceModel, prompt_ids, gen_len: int, caches, out_ids=No
 
 def fg_profile_enable(on: bool = True):
     _check(lib().fg_profile_enable(int(on)))
+
+
+def fg_profile_select(kinds=None):
+    """Time only these kinds (indices into PROF_NAMES) while profiling is on; None = all."""
+    mask = (1 << len(PROF_NAMES)) - 1 if kinds is None else sum(1 << int(k) for k in kinds)
+    _check(lib().fg_profile_select(mask))
 
 
 def fg_profile_reset():

@@ -25,6 +25,7 @@ int layernorm_impl(const void*, int64_t, int, const void*, const void*, void*, c
 int embed_impl(const int32_t*, int64_t, int, int, int, const void*, const void*, int, void*, cudaStream_t);
 int argmax_impl(const float*, int, int, int32_t*, int64_t, cudaStream_t);
 size_t qgemm_ws_bytes(int64_t, int, int);
+size_t splitk_ws_bytes(int64_t, int, int);
 int gemm_impl(int, const void*, int64_t, int, int, const void*, const void*, int, const void*, const void*, int,
               void*, bool, void*, size_t, cudaStream_t);
 int read_device_error(int*);
@@ -75,8 +76,20 @@ struct ProfRec {
   cudaEvent_t a, b;
   double flops, bytes;
 };
+// Events are recorded as graph nodes while the stream is being captured, so that a profiled
+// generation still replays its CUDA graphs.
+void record_event(cudaEvent_t e, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+  else
+    cudaEventRecord(e, s);
+}
 std::mutex g_prof_mu;
+constexpr uint32_t kAllKinds = (1u << PROF_NKINDS) - 1;
 bool g_prof_on = false;
+uint32_t g_prof_sel = kAllKinds;  // kinds timed while profiling is on
+uint32_t g_prof_mask = 0;         // g_prof_on ? g_prof_sel : 0
 std::vector<ProfRec> g_prof_pending;
 double g_prof_ms[PROF_NKINDS] = {0};
 int64_t g_prof_n[PROF_NKINDS] = {0};
@@ -95,15 +108,18 @@ cudaEvent_t take_event() {
   return e;
 }
 
+void add_record(const ProfRec& r) {
+  float ms = 0.f;
+  if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) {
+    g_prof_ms[r.kind] += ms;
+    g_prof_n[r.kind] += 1;
+    g_prof_flops[r.kind] += r.flops;
+    g_prof_bytes[r.kind] += r.bytes;
+  }
+}
 void collect_locked() {
   for (auto& r : g_prof_pending) {
-    float ms = 0.f;
-    if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) {
-      g_prof_ms[r.kind] += ms;
-      g_prof_n[r.kind] += 1;
-      g_prof_flops[r.kind] += r.flops;
-      g_prof_bytes[r.kind] += r.bytes;
-    }
+    add_record(r);
     g_event_pool.push_back(r.a);
     g_event_pool.push_back(r.b);
   }
@@ -113,9 +129,9 @@ void collect_locked() {
 
 ProfScope::ProfScope(int kind, cudaStream_t st, double flops, double bytes) : slot(-1), s(st) {
   std::lock_guard<std::mutex> lk(g_prof_mu);
-  if (!g_prof_on) return;
+  if (!((g_prof_mask >> kind) & 1u)) return;
   ProfRec r{kind, take_event(), take_event(), flops, bytes};
-  cudaEventRecord(r.a, s);
+  record_event(r.a, s);
   g_prof_pending.push_back(r);
   slot = int(g_prof_pending.size()) - 1;
 }
@@ -123,7 +139,7 @@ ProfScope::ProfScope(int kind, cudaStream_t st, double flops, double bytes) : sl
 ProfScope::~ProfScope() {
   if (slot < 0) return;
   std::lock_guard<std::mutex> lk(g_prof_mu);
-  if (slot < int(g_prof_pending.size())) cudaEventRecord(g_prof_pending[slot].b, s);
+  if (slot < int(g_prof_pending.size())) record_event(g_prof_pending[slot].b, s);
 }
 
 // ---------------------------------------------------------------- workspace carving
@@ -164,10 +180,13 @@ int check_layer(const fg_layer* L, int h, int* ffn) {
 // Y = [relu](X W_hat + b) [+ R] for a 4-bit weight.  With many rows (a prompt pass) each
 // weight tile is reused by M/128 row tiles, so the weight is first expanded once into an
 // fp16 copy in the workspace (an HBM-bound pass, ~1 % of the GEMM) and the tensor-core GEMM
-// then runs without dequant warps; with few rows (decode) the fused kernel reads the 4-bit
-// weight directly, once.  Both compute with the same fp16 values W_hat.
+// then runs without dequant warps.  Decode batches (M <= 256) run the kernel that expands
+// the weight into tensor memory; the rows in between, the fused kernel that expands it into
+// shared memory.  All compute with the same fp16 values W_hat.
 int qlinear_run(const void* X, int64_t M, const fg_qlinear& w, const void* R, int relu, void* Y, void* ws,
                 size_t wsb, cudaStream_t s) {
+  if (qgemm_dec_supported(M, w.N, w.K, w.group))
+    return qgemm_dec_impl(X, M, w.N, w.K, w.codes, w.params, w.group, w.bias, R, relu, Y, s);
   const size_t wbytes = (size_t(w.K) * size_t(w.N) * 2 + 255) & ~size_t(255);
   if (M >= kExpandRows && ws != nullptr && wsb >= wbytes && aligned16(ws)) {
     FG_TRY(dequantize_impl(w.codes, w.params, w.K, w.N, w.group, 1, ws, s));
@@ -319,7 +338,7 @@ void put(std::vector<uint8_t>& v, const T& x) {
   v.insert(v.end(), p, p + sizeof(T));
 }
 GraphKey make_key(const fg_model* m, const int32_t* ids, int B, int L, int T, int32_t* out,
-                  const fg_kv_cache* caches, void* ws, size_t wsb, cudaStream_t s) {
+                  const fg_kv_cache* caches, void* ws, size_t wsb, cudaStream_t s, uint32_t prof) {
   GraphKey k;
   int dev = -1;
   cudaGetDevice(&dev);
@@ -339,6 +358,7 @@ GraphKey make_key(const fg_model* m, const int32_t* ids, int B, int L, int T, in
   put(k.bytes, ws);
   put(k.bytes, wsb);
   put(k.bytes, s);
+  put(k.bytes, prof);
   return k;
 }
 struct GraphCache {
@@ -347,13 +367,15 @@ struct GraphCache {
   cudaGraphExec_t prefill = nullptr, decode = nullptr;
   int64_t n_prefill = 0, n_decode = 0;
   cudaStream_t cap = nullptr;
+  // timing events the graphs record (captured while profiling was on)
+  std::vector<ProfRec> prof_prefill, prof_decode;
 };
 std::mutex g_graph_mu;
 GraphCache g_graph;
 
-bool profiling_on() {
+uint32_t profiling_mask() {
   std::lock_guard<std::mutex> lk(g_prof_mu);
-  return g_prof_on;
+  return g_prof_mask;
 }
 
 void reset_graphs() {
@@ -361,18 +383,45 @@ void reset_graphs() {
   if (g_graph.decode) cudaGraphExecDestroy(g_graph.decode);
   g_graph.prefill = g_graph.decode = nullptr;
   g_graph.valid = g_graph.seen = false;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto* v : {&g_graph.prof_prefill, &g_graph.prof_decode}) {
+    for (auto& r : *v) {
+      g_event_pool.push_back(r.a);
+      g_event_pool.push_back(r.b);
+    }
+    v->clear();
+  }
+}
+
+// Adds the durations of the launches that a replayed graph timed.
+void collect_graph(const std::vector<ProfRec>& recs) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& r : recs) add_record(r);
 }
 
 template <class F>
-int capture_one(F&& seq, cudaGraphExec_t* exec, int64_t* n_launches) {
+int capture_one(F&& seq, cudaGraphExec_t* exec, int64_t* n_launches, std::vector<ProfRec>* recs) {
   cudaStream_t cs = g_graph.cap;
   const int64_t before = g_launches.load();
+  size_t rec0 = 0;
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    rec0 = g_prof_pending.size();
+  }
   FG_CHECK_CUDA(cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal));
   const int st = seq(cs);
   cudaGraph_t graph = nullptr;
   const cudaError_t ce = cudaStreamEndCapture(cs, &graph);
   *n_launches = g_launches.load() - before;
   g_launches.fetch_sub(*n_launches);  // recorded, not executed
+  {
+    // the timing events of the captured launches now belong to the graph
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (rec0 < g_prof_pending.size()) {
+      recs->assign(g_prof_pending.begin() + rec0, g_prof_pending.end());
+      g_prof_pending.resize(rec0);
+    }
+  }
   if (st != FG_OK) {
     if (graph) cudaGraphDestroy(graph);
     return st;
@@ -387,8 +436,8 @@ int capture_one(F&& seq, cudaGraphExec_t* exec, int64_t* n_launches) {
 template <class P, class D>
 int capture_graphs(P&& prefill_seq, D&& decode_seq) {
   if (!g_graph.cap) FG_CHECK_CUDA(cudaStreamCreateWithFlags(&g_graph.cap, cudaStreamNonBlocking));
-  FG_TRY(capture_one(prefill_seq, &g_graph.prefill, &g_graph.n_prefill));
-  FG_TRY(capture_one(decode_seq, &g_graph.decode, &g_graph.n_decode));
+  FG_TRY(capture_one(prefill_seq, &g_graph.prefill, &g_graph.n_prefill, &g_graph.prof_prefill));
+  FG_TRY(capture_one(decode_seq, &g_graph.decode, &g_graph.n_decode, &g_graph.prof_decode));
   g_graph.valid = true;
   return FG_OK;
 }
@@ -443,19 +492,18 @@ int generate_impl(const fg_model* m, const int32_t* ids, int B, int L, int T, in
   };
 
   std::lock_guard<std::mutex> glk(g_graph_mu);
-  GraphKey key = make_key(m, ids, B, L, T, out, caches, ws, wsb, s);
-  const bool use_graphs = !profiling_on();
+  GraphKey key = make_key(m, ids, B, L, T, out, caches, ws, wsb, s, profiling_mask());
   bool replay = false;
-  if (use_graphs && g_graph.valid && g_graph.key == key) {
+  if (g_graph.valid && g_graph.key == key) {
     replay = true;
-  } else if (use_graphs && g_graph.seen && g_graph.key == key) {
+  } else if (g_graph.seen && g_graph.key == key) {
     // second call with this configuration: record both sequences as graphs, then replay
     FG_TRY(capture_graphs(prefill_seq, decode_seq));
     replay = true;
   } else {
     reset_graphs();
     g_graph.key = key;
-    g_graph.seen = use_graphs;
+    g_graph.seen = true;
   }
 
   cudaEvent_t e0, e1, e2;
@@ -485,6 +533,10 @@ int generate_impl(const fg_model* m, const int32_t* ids, int B, int L, int T, in
     cudaEventRecord(e2, s);
     ce = cudaEventSynchronize(e2);
     if (ce != cudaSuccess) { st = cuda_fail(ce, "generate"); break; }
+    if (replay) {
+      collect_graph(g_graph.prof_prefill);
+      collect_graph(g_graph.prof_decode);
+    }
     int derr = 0;
     if (read_device_error(&derr) == FG_OK && derr != 0) {
       st = fail(FG_ERR_CUDA, "a device-side wait timed out (code %d)", derr);
@@ -551,6 +603,8 @@ int fg_qgemm(const void* X, int64_t M, const fg_qlinear* W, const void* R, int r
   if (!W) return fail(FG_ERR_INVALID_ARG, "null weight");
   return qlinear_run(X, M, *W, R, relu, Y, workspace, ws_bytes, as_stream(stream));
 }
+
+size_t fg_gemm_f16_workspace_bytes(int64_t M, int N, int K) { return splitk_ws_bytes(M, N, K); }
 
 int fg_gemm_f16(const void* X, int64_t M, const void* W, int K, int N, const void* bias, const void* R, int relu,
                 void* Y, void* workspace, size_t ws_bytes, void* stream) {
@@ -620,6 +674,14 @@ int fg_generate(const fg_model* model, const int32_t* prompt_ids, int B, int L, 
 int fg_profile_enable(int on) {
   std::lock_guard<std::mutex> lk(g_prof_mu);
   g_prof_on = on != 0;
+  g_prof_mask = g_prof_on ? g_prof_sel : 0u;
+  return FG_OK;
+}
+
+int fg_profile_select(unsigned kinds) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_sel = kinds & kAllKinds;
+  g_prof_mask = g_prof_on ? g_prof_sel : 0u;
   return FG_OK;
 }
 

@@ -6,11 +6,10 @@
 //   out = sum_t softmax(score)_t V_t
 // The cache is read exactly once: one CTA per (chunk of positions, head, sequence)
 // streams the chunk's K and V codes together in a single pass with an online softmax.
-// Codes are never expanded to fp16: with f = 0.5 + code/256 (built by one byte
-// permute into the mantissa of 0.5f), sum_i q_i code_i = 256 (sum_i q_i f_i - 0.5 sum_i q_i),
-// and a group contributes s * sum(q code) + mn * sum(q).  The V side uses the same
-// identity with weights p_t s_t.  Softmax is fp32 with exp2 (q pre-scaled by
-// log2(e)/sqrt(hd)); chunks are merged with the usual (max, sum, acc) rescaling.
+// Both contractions run on the tensor cores (mma.sync) over codes that are only unpacked
+// into exact fp16 (offset + code) values, with the per-group {min, scale} applied to the
+// fp32 results.  Softmax is fp32 with exp2 (scores scaled by log2(e)/sqrt(hd)); warps and
+// chunks are merged with the usual (max, sum, acc) rescaling.
 #include <algorithm>
 #include <mutex>
 
@@ -21,27 +20,7 @@ namespace {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
-constexpr int kUnroll = 4;
 constexpr float kLog2e = 1.4426950408889634f;
-
-// f_i = 0.5 + c_i/256 for the 8 codes of w (element i in bits 4i..4i+3).
-// even = w & 0x0F0F0F0F holds codes 0,2,4,6 in bytes 0..3; odd = (w>>4) & 0x0F0F0F0F
-// codes 1,3,5,7.  __byte_perm(src, 0x3F000000, sel) puts byte k of src into byte 2 of
-// 0x3F000000 (0.5f), i.e. into mantissa bits 16..19.
-__device__ __forceinline__ void code_floats(uint32_t w, float f[8]) {
-  const uint32_t even = w & 0x0F0F0F0Fu;
-  const uint32_t odd = (w >> 4) & 0x0F0F0F0Fu;
-  const uint32_t half = 0x3F000000u;
-  // result bytes (3..0) = [half.b3, src.bk, half.b1, half.b0] -> selector 0x7k54
-  f[0] = __uint_as_float(__byte_perm(even, half, 0x7054));
-  f[1] = __uint_as_float(__byte_perm(odd, half, 0x7054));
-  f[2] = __uint_as_float(__byte_perm(even, half, 0x7154));
-  f[3] = __uint_as_float(__byte_perm(odd, half, 0x7154));
-  f[4] = __uint_as_float(__byte_perm(even, half, 0x7254));
-  f[5] = __uint_as_float(__byte_perm(odd, half, 0x7254));
-  f[6] = __uint_as_float(__byte_perm(even, half, 0x7354));
-  f[7] = __uint_as_float(__byte_perm(odd, half, 0x7354));
-}
 
 __device__ __forceinline__ uint4 ldg_v4(const uint4* p) {
   uint4 r;
@@ -51,23 +30,59 @@ __device__ __forceinline__ uint4 ldg_v4(const uint4* p) {
   return r;
 }
 
-// HD = head dim (64 or 128), G = group size (divides HD, >= 32).
-// Lane layout: LPT = HD/32 lanes per token, each owning 32 dims (one 16-byte load of K
-// codes and one of V codes per token, inside one group); TPW = 32/LPT tokens per warp
-// step.  Every lane keeps an online-softmax state (max m, sum l, weighted sums) for the
-// tokens of its slot; slots, warps and chunks are merged at the end with the usual rescaling.
+// ------------------------------------------------------------------ K4, tensor-core form
+// The same attention with both contractions on mma.sync (m16n8k16, fp16 in, fp32 out), so
+// that the codes are only unpacked, never multiplied on the FMA pipe.  A warp takes blocks
+// of 16 positions.
+//   scores:  D[t][n] = sum over the dims d of group n of q_d (o_d + c_td)   (A = codes,
+//            B = q masked per group), with o_d = 1024 for low-nibble and 64 for high-nibble
+//            dims: a code becomes an exact fp16 (o + c) by putting the nibble into the
+//            mantissa of 1024.0 (bits 0-3) or of 64.0 (bits 4-7); K dims are taken in any
+//            order that A and B agree on.  score_t = sum_n s_tn (D[t][n] - O_n) + mn_tn Q_n,
+//            O_n = sum q_d o_d, Q_n = sum q_d over the group.
+//   values:  E[d][n] = sum_t w_tn (o_d + c_td) with w_tn = fp16(p_t s_tn) (A = codes with
+//            pairs of positions per register, B = w), and
+//            out_d = (sum_t p_t mn_tn + E[d][n] - o_d sum_t w_tn) / sum_t p_t, n = group(d).
+// Thread (g = lane/4, q4 = lane%4) holds positions g and g + 8 of a block for the scores and
+// dims DPT*g .. DPT*g + DPT-1 for the values (DPT = HD/8).
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The four fp16 pairs of one code word (dims 8w .. 8w+7): P0 = (o+c) of dims (0, 2),
+// P1 = (4, 6), both low nibbles (o = 1024); P2 = (1, 3), P3 = (5, 7), high nibbles (o = 64).
+__device__ __forceinline__ void code_pairs(uint32_t w, uint32_t (&P)[4]) {
+  const uint32_t x = w & 0x0F0F0F0Fu, y = w & 0xF0F0F0F0u;
+  P[0] = __byte_perm(x, 0x64646464u, 0x4140);
+  P[1] = __byte_perm(x, 0x64646464u, 0x4342);
+  P[2] = __byte_perm(y, 0x54545454u, 0x4140);
+  P[3] = __byte_perm(y, 0x54545454u, 0x4342);
+}
+
 template <int HD, int G>
-__global__ void __launch_bounds__(kThreads) decode_attn_kernel(
-    const __half* __restrict__ q, int64_t q_stride, const uint4* __restrict__ kc,
-    const __half2* __restrict__ kp, const uint4* __restrict__ vc, const __half2* __restrict__ vp,
+struct AttnMma {
+  static constexpr int NG = HD / G;    // groups per head: 1, 2 or 4
+  static constexpr int KW = HD / 32;   // code words a thread reads of a K row
+  static constexpr int KS = HD / 16;   // k-steps of the score MMA
+  static constexpr int MT = HD / 16;   // 16-dim tiles of the value MMA
+  static constexpr int DPT = HD / 8;   // dims per value row-thread
+  static constexpr int VW = HD / 64;   // code words a thread reads of a V row
+  static constexpr int TB = 16;        // positions per block
+};
+
+template <int HD, int G>
+__global__ void __launch_bounds__(kThreads) decode_attn_mma_kernel(
+    const __half* __restrict__ q, int64_t q_stride, const uint8_t* __restrict__ kc,
+    const __half2* __restrict__ kp, const uint8_t* __restrict__ vc, const __half2* __restrict__ vp,
     int nh, int cap, int S, int chunk_len, __half* __restrict__ out, float* __restrict__ part_ml,
     float* __restrict__ part_acc) {
-  constexpr int LPT = HD / 32;
-  constexpr int TPW = 32 / LPT;
-  constexpr int STEP = kWarps * TPW;
-  constexpr int VPT = HD / 32;  // 16-byte code vectors per token
-  constexpr int PPT = HD / G;   // params per token
-  constexpr int U = 2;          // token steps in flight per lane
+  using C = AttnMma<HD, G>;
+  constexpr int NG = C::NG, KW = C::KW, KS = C::KS, MT = C::MT, DPT = C::DPT, VW = C::VW, TB = C::TB;
   __shared__ float red_v[kWarps][HD];
   __shared__ float red_ml[kWarps][2];
 
@@ -75,121 +90,248 @@ __global__ void __launch_bounds__(kThreads) decode_attn_kernel(
   const int t0 = chunk * chunk_len;
   const int t1 = min(S, t0 + chunk_len);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int sub = lane % LPT, slot = lane / LPT;
-  const int d0 = sub * 32;
+  const int g = lane >> 2, q4 = lane & 3;
+  const __half* qh = q + int64_t(b) * q_stride + head * HD;
 
-  // query slice (32 dims), pre-scaled so scores are in log2 units
-  float qf[32];
-  {
-    const uint4* qp = reinterpret_cast<const uint4*>(q + int64_t(b) * q_stride + head * HD + d0);
-    const float scale = kLog2e * rsqrtf(float(HD));
+  // ---- query: B fragments of the score MMA, and per-group O_n, Q_n
+  uint32_t qb[KS][2];
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const uint4 raw = qp[v];
-      const __half2* h = reinterpret_cast<const __half2*>(&raw);
+  for (int st = 0; st < KS; ++st) {
+    const int w = KW * q4 + st / 2, e = st & 1;
+    const bool mine = (8 * w) / G == g;  // column g of B is group g
+    const int d0 = 8 * w + e;
+    const __half z = __float2half(0.f);
+    const __half h0 = mine ? qh[d0] : z, h1 = mine ? qh[d0 + 2] : z;
+    const __half h2 = mine ? qh[d0 + 4] : z, h3 = mine ? qh[d0 + 6] : z;
+    qb[st][0] = h2_as_u32(__halves2half2(h0, h1));
+    qb[st][1] = h2_as_u32(__halves2half2(h2, h3));
+  }
+  float On[NG], Qn[NG];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = __half22float2(h[j]);
-        qf[8 * v + 2 * j] = f.x * scale;
-        qf[8 * v + 2 * j + 1] = f.y * scale;
+  for (int n = 0; n < NG; ++n) On[n] = Qn[n] = 0.f;
+#pragma unroll
+  for (int i = 0; i < HD / 32; ++i) {
+    const int d = lane + 32 * i;
+    const float qd = __half2float(qh[d]);
+#pragma unroll
+    for (int n = 0; n < NG; ++n) {
+      if (d / G == n) {
+        Qn[n] += qd;
+        On[n] += qd * ((d & 1) ? 64.f : 1024.f);
       }
     }
   }
-  float qs = 0.f;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) qs += qf[i];
+  for (int n = 0; n < NG; ++n) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      Qn[n] += __shfl_xor_sync(0xffffffffu, Qn[n], o);
+      On[n] += __shfl_xor_sync(0xffffffffu, On[n], o);
+    }
+  }
+  const float sc = kLog2e * rsqrtf(float(HD));
 
   const int64_t slot0 = (int64_t(b) * nh + head) * cap;
-  const uint4* kw = kc + slot0 * VPT + sub;
-  const uint4* vw = vc + slot0 * VPT + sub;
-  const __half2* kpp = kp + slot0 * PPT + d0 / G;
-  const __half2* vpp = vp + slot0 * PPT + d0 / G;
+  const uint8_t* kbase = kc + slot0 * (HD / 2);
+  const uint8_t* vbase = vc + slot0 * (HD / 2);
+  const __half2* kpb = kp + slot0 * NG;
+  const __half2* vpb = vp + slot0 * NG;
 
-  float m = -INFINITY, l = 0.f, accb = 0.f, accm = 0.f;
-  float acc[32];
+  float m = -INFINITY, lsum = 0.f, amn = 0.f, ssum = 0.f;
+  float acc[MT][4];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+  for (int i = 0; i < MT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
 
-  for (int tb = t0 + warp * TPW; tb < t1; tb += STEP * U) {
-    uint4 kq[U], vq[U];
-    __half2 kpar[U], vpar[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int t = tb + u * STEP + slot;
-      const bool ok = t < t1;
-      kq[u] = ok ? ldg_v4(kw + int64_t(t) * VPT) : make_uint4(0, 0, 0, 0);
-      vq[u] = ok ? ldg_v4(vw + int64_t(t) * VPT) : make_uint4(0, 0, 0, 0);
-      kpar[u] = ok ? __ldg(kpp + int64_t(t) * PPT) : __half2();
-      vpar[u] = ok ? __ldg(vpp + int64_t(t) * PPT) : __half2();
+  // raw loads of one block: K rows g, g+8 (KW words from word KW*q4), V rows 2q4, 2q4+1,
+  // 2q4+8, 2q4+9 (VW words at dim DPT*g), K params of (row, groups 2q4, 2q4+1), V params of
+  // (row, group q4); positions past t1 read as zeros
+  struct Blk {
+    uint32_t kA[KW], kB[KW], vw[4][VW], kpA[2], kpB[2], vpA, vpB;
+  };
+  auto load = [&](Blk& o, int blk) {
+    const int tA = blk + g, tB = blk + g + 8;
+    const bool okA = tA < t1, okB = tB < t1;
+    if (KW == 4) {
+      const uint4 za = okA ? ldg_v4(reinterpret_cast<const uint4*>(kbase + int64_t(tA) * (HD / 2)) + q4)
+                           : make_uint4(0, 0, 0, 0);
+      const uint4 zb = okB ? ldg_v4(reinterpret_cast<const uint4*>(kbase + int64_t(tB) * (HD / 2)) + q4)
+                           : make_uint4(0, 0, 0, 0);
+      o.kA[0] = za.x; o.kA[1 % KW] = za.y; o.kA[2 % KW] = za.z; o.kA[3 % KW] = za.w;
+      o.kB[0] = zb.x; o.kB[1 % KW] = zb.y; o.kB[2 % KW] = zb.z; o.kB[3 % KW] = zb.w;
+    } else {
+      const uint2 za = okA ? __ldg(reinterpret_cast<const uint2*>(kbase + int64_t(tA) * (HD / 2)) + q4)
+                           : make_uint2(0, 0);
+      const uint2 zb = okB ? __ldg(reinterpret_cast<const uint2*>(kbase + int64_t(tB) * (HD / 2)) + q4)
+                           : make_uint2(0, 0);
+      o.kA[0] = za.x; o.kA[1 % KW] = za.y;
+      o.kB[0] = zb.x; o.kB[1 % KW] = zb.y;
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const bool ok = tb + u * STEP + slot < t1;
-      // score partial over this lane's 32 dims: s*sum(q code) + mn*sum(q)
-      float dot = 0.f;
-      {
-        const uint32_t wv[4] = {kq[u].x, kq[u].y, kq[u].z, kq[u].w};
+    for (int r = 0; r < 4; ++r) {
+      const int t = blk + 2 * q4 + (r & 1) + (r >> 1) * 8;
+      const bool ok = t < t1;
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(vbase + int64_t(t) * (HD / 2)) + VW * g;
+      if (VW == 2) {
+        const uint2 z = ok ? __ldg(reinterpret_cast<const uint2*>(src)) : make_uint2(0, 0);
+        o.vw[r][0] = z.x;
+        o.vw[r][VW - 1] = z.y;
+      } else {
+        o.vw[r][0] = ok ? __ldg(src) : 0u;
+      }
+    }
+    const uint32_t* kpu = reinterpret_cast<const uint32_t*>(kpb);
+    const uint32_t* vpu = reinterpret_cast<const uint32_t*>(vpb);
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          float f[8];
-          code_floats(wv[v], f);
+    for (int j = 0; j < 2; ++j) {
+      const int n = 2 * q4 + j;
+      o.kpA[j] = (n < NG && okA) ? __ldg(kpu + int64_t(tA) * NG + n) : 0u;
+      o.kpB[j] = (n < NG && okB) ? __ldg(kpu + int64_t(tB) * NG + n) : 0u;
+    }
+    o.vpA = (q4 < NG && okA) ? __ldg(vpu + int64_t(tA) * NG + q4) : 0u;
+    o.vpB = (q4 < NG && okB) ? __ldg(vpu + int64_t(tB) * NG + q4) : 0u;
+  };
+
+  Blk cur;
+  load(cur, t0 + warp * TB);
+  for (int blk = t0 + warp * TB; blk < t1; blk += kWarps * TB) {
+    Blk nxt;
+    load(nxt, blk + kWarps * TB);  // next block's loads in flight while this one computes
+    const int tA = blk + g, tB = blk + g + 8;
+    const bool okA = tA < t1, okB = tB < t1;
+    const uint32_t(&kA)[KW] = cur.kA;
+    const uint32_t(&kB)[KW] = cur.kB;
+    const uint32_t(&vw)[4][VW] = cur.vw;
+    float ksA[2], kmA[2], ksB[2], kmB[2];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) dot = fmaf(qf[8 * v + i], f[i], dot);
+    for (int j = 0; j < 2; ++j) {
+      const float2 fa = __half22float2(u32_as_h2(cur.kpA[j])), fb = __half22float2(u32_as_h2(cur.kpB[j]));
+      kmA[j] = fa.x;
+      ksA[j] = fa.y;
+      kmB[j] = fb.x;
+      ksB[j] = fb.y;
+    }
+    const float2 fva = __half22float2(u32_as_h2(cur.vpA)), fvb = __half22float2(u32_as_h2(cur.vpB));
+    const float vmA = fva.x, vsA = fva.y, vmB = fvb.x, vsB = fvb.y;
+
+    // ---- scores
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int wi = 0; wi < KW; ++wi) {
+      uint32_t PA[4], PB[4];
+      code_pairs(kA[wi], PA);
+      code_pairs(kB[wi], PB);
+      mma16816(d, PA[0], PB[0], PA[1], PB[1], qb[2 * wi][0], qb[2 * wi][1]);
+      mma16816(d, PA[2], PB[2], PA[3], PB[3], qb[2 * wi + 1][0], qb[2 * wi + 1][1]);
+    }
+    float pa = 0.f, pb = 0.f;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int n = 2 * q4 + j;
+      float o = 0.f, qs = 0.f;
+#pragma unroll
+      for (int k = 0; k < NG; ++k) {
+        if (n == k) {
+          o = On[k];
+          qs = Qn[k];
         }
       }
-      const float2 km = __half22float2(kpar[u]);  // {mn, s}
-      float part = fmaf(km.y, (dot - 0.5f * qs) * 256.f, km.x * qs);
-#pragma unroll
-      for (int o = 1; o < LPT; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-      if (!ok) continue;
-      if (part > m) {  // new running max for this slot: rescale its sums
-        const float sc = exp2f(m - part);  // m = -inf -> 0
-        l *= sc;
-        accb *= sc;
-        accm *= sc;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc[i] *= sc;
-        m = part;
+      if (n < NG) {
+        pa += fmaf(ksA[j], d[j] - o, kmA[j] * qs);
+        pb += fmaf(ksB[j], d[2 + j] - o, kmB[j] * qs);
       }
-      const float p = exp2f(part - m);
-      l += p;
-      const float2 vm = __half22float2(vpar[u]);
-      const float bt = p * vm.y;
-      accm = fmaf(p, vm.x, accm);
-      accb += bt;
-      const uint32_t wv[4] = {vq[u].x, vq[u].y, vq[u].z, vq[u].w};
+    }
+    if (NG > 2) {
+      pa += __shfl_xor_sync(0xffffffffu, pa, 1);
+      pb += __shfl_xor_sync(0xffffffffu, pb, 1);
+    }
+    // every lane of a row now holds the scores (lanes with q4 >= 2 hold 0 when NG <= 2)
+    pa = __shfl_sync(0xffffffffu, pa, lane & ~3);
+    pb = __shfl_sync(0xffffffffu, pb, lane & ~3);
+    const float sA = okA ? pa * sc : -INFINITY, sB = okB ? pb * sc : -INFINITY;
+    float bm = fmaxf(sA, sB);
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        float f[8];
-        code_floats(wv[v], f);
+    for (int o = 4; o < 32; o <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+    if (bm > m) {
+      const float r = exp2f(m - bm);  // m = -inf -> 0
+      lsum *= r;
+      amn *= r;
+      ssum *= r;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[8 * v + i] = fmaf(bt, f[i], acc[8 * v + i]);
+      for (int i = 0; i < MT; ++i) {
+        acc[i][0] *= r; acc[i][1] *= r; acc[i][2] *= r; acc[i][3] *= r;
+      }
+      m = bm;
+    }
+    const float pA = exp2f(sA - m), pB = exp2f(sB - m);  // 0 for positions past the end
+    if (q4 == 0) lsum += pA + pB;
+    // value weights of (row, group q4): w = fp16(p * s)
+    const __half wA = __float2half_rn(pA * vsA), wB = __float2half_rn(pB * vsB);
+    amn = fmaf(pA, vmA, fmaf(pB, vmB, amn));
+    ssum += __half2float(wA) + __half2float(wB);
+    // B fragment of the value MMA for group g: positions 2q4, 2q4+1 (rows of lanes 8q4 + g,
+    // 8q4 + 4 + g as "A"), and 2q4 + 8, 2q4 + 9 (the same lanes' "B" rows)
+    const uint32_t wAu = __half_as_ushort(wA), wBu = __half_as_ushort(wB);
+    const int src0 = 8 * q4 + (g & 3), src1 = src0 + 4;
+    const uint32_t w0 = __shfl_sync(0xffffffffu, wAu, src0), w1 = __shfl_sync(0xffffffffu, wAu, src1);
+    const uint32_t w2 = __shfl_sync(0xffffffffu, wBu, src0), w3 = __shfl_sync(0xffffffffu, wBu, src1);
+    const bool gv = g < NG;
+    const uint32_t b0 = gv ? (w0 | (w1 << 16)) : 0u, b1 = gv ? (w2 | (w3 << 16)) : 0u;
+
+    // ---- values: tile mt covers byte mt of the thread's V words (dims DPT*g + 2mt, +1)
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const int wd = mt / 4, by = mt % 4;
+      const uint32_t sel = uint32_t(by | (by << 4) | ((4 + by) << 8) | ((4 + by) << 12));
+      const uint32_t r01 = __byte_perm(vw[0][wd], vw[1][wd], sel);
+      const uint32_t r23 = __byte_perm(vw[2][wd], vw[3][wd], sel);
+      const uint32_t a0 = (r01 & 0x000F000Fu) | 0x64006400u, a1 = (r01 & 0x00F000F0u) | 0x54005400u;
+      const uint32_t a2 = (r23 & 0x000F000Fu) | 0x64006400u, a3 = (r23 & 0x00F000F0u) | 0x54005400u;
+      mma16816(acc[mt], a0, a1, a2, a3, b0, b1);
+    }
+    cur = nxt;
+  }
+
+  // ---- finish the warp: sums over rows, then out_d for the dims this lane holds
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    amn += __shfl_xor_sync(0xffffffffu, amn, o);
+    ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
+  }
+  float amn_n[NG], ss_n[NG];
+#pragma unroll
+  for (int n = 0; n < NG; ++n) {
+    amn_n[n] = __shfl_sync(0xffffffffu, amn, n);
+    ss_n[n] = __shfl_sync(0xffffffffu, ssum, n);
+  }
+  // acc[mt][0/1]: dim DPT*g + 2mt (low nibble, o = 1024), groups 2q4 / 2q4+1;
+  // acc[mt][2/3]: dim DPT*g + 2mt + 1 (high nibble, o = 64)
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+    for (int hv = 0; hv < 2; ++hv) {
+      const int dd = DPT * g + 2 * mt + hv;
+      const int n = dd / G;
+      if ((n >> 1) == q4) {
+        const float e = (n & 1) ? acc[mt][2 * hv + 1] : acc[mt][2 * hv];
+        float an = amn_n[0], sn = ss_n[0];
+#pragma unroll
+        for (int k = 1; k < NG; ++k) {
+          if (n == k) {
+            an = amn_n[k];
+            sn = ss_n[k];
+          }
+        }
+        red_v[warp][dd] = an + e - (hv ? 64.f : 1024.f) * sn;
       }
     }
   }
-
-  // sum_t p_t (mn_t + s_t c_td) = accm + 256 (acc_d - 0.5 accb), then merge the slots of the warp
-  float M = m;
-#pragma unroll
-  for (int o = LPT; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  const float sc = (m == -INFINITY) ? 0.f : exp2f(m - M);
-  float lw = l * sc;
-#pragma unroll
-  for (int o = LPT; o < 32; o <<= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
-  const float base = accm * sc;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    float v = fmaf(256.f * sc, acc[i] - 0.5f * accb, base);
-#pragma unroll
-    for (int o = LPT; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (slot == 0) red_v[warp][d0 + i] = v;
-  }
   if (lane == 0) {
-    red_ml[warp][0] = M;
-    red_ml[warp][1] = lw;
+    red_ml[warp][0] = m;
+    red_ml[warp][1] = lsum;
   }
   __syncthreads();
-  // merge the warps
   float Mc = red_ml[0][0];
 #pragma unroll
   for (int w = 1; w < kWarps; ++w) Mc = fmaxf(Mc, red_ml[w][0]);
@@ -201,14 +343,15 @@ __global__ void __launch_bounds__(kThreads) decode_attn_kernel(
     L = fmaf(red_ml[w][1], wsc[w], L);
   }
   const int64_t bh = int64_t(b) * nh + head;
-  for (int d = threadIdx.x; d < HD; d += kThreads) {
+  for (int dd = threadIdx.x; dd < HD; dd += kThreads) {
     float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) v = fmaf(red_v[w][d], wsc[w], v);
+    for (int w = 0; w < kWarps; ++w)
+      if (wsc[w] != 0.f) v = fmaf(red_v[w][dd], wsc[w], v);
     if (part_ml == nullptr) {
-      out[int64_t(b) * nh * HD + head * HD + d] = __float2half_rn(v / L);
+      out[int64_t(b) * nh * HD + head * HD + dd] = __float2half_rn(v / L);
     } else {
-      part_acc[(bh * gridDim.x + chunk) * HD + d] = v;
+      part_acc[(bh * gridDim.x + chunk) * HD + dd] = v;
     }
   }
   if (part_ml != nullptr && threadIdx.x == 0) {
@@ -295,14 +438,14 @@ int decode_attention_impl(const void* q, int64_t q_stride, const fg_kv_cache* c,
   dim3 grid(nc, nh, B);
   const size_t smem = 0;
   auto* qh = reinterpret_cast<const __half*>(q);
-  auto* kc = reinterpret_cast<const uint4*>(c->k_codes);
-  auto* vc = reinterpret_cast<const uint4*>(c->v_codes);
   auto* kp = reinterpret_cast<const __half2*>(c->k_params);
   auto* vp = reinterpret_cast<const __half2*>(c->v_params);
   auto* o = reinterpret_cast<__half*>(out);
-#define FG_ATTN_LAUNCH(HD_, G_)                                                                   \
-  decode_attn_kernel<HD_, G_><<<grid, kThreads, smem, s>>>(qh, q_stride, kc, kp, vc, vp, nh,    \
-                                                            c->capacity, S, chunk_len, o, ml, acc)
+  auto* kc8 = reinterpret_cast<const uint8_t*>(c->k_codes);
+  auto* vc8 = reinterpret_cast<const uint8_t*>(c->v_codes);
+#define FG_ATTN_LAUNCH(HD_, G_)                                                                      \
+  decode_attn_mma_kernel<HD_, G_><<<grid, kThreads, smem, s>>>(qh, q_stride, kc8, kp, vc8, vp, nh, \
+                                                                c->capacity, S, chunk_len, o, ml, acc)
   if (hd == 128 && G == 128) FG_ATTN_LAUNCH(128, 128);
   else if (hd == 128 && G == 64) FG_ATTN_LAUNCH(128, 64);
   else if (hd == 128 && G == 32) FG_ATTN_LAUNCH(128, 32);

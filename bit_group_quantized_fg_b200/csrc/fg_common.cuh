@@ -46,6 +46,17 @@ int num_sms();
 // fp16 tensor-core GEMM (measured break-even ~700 rows on B200).
 constexpr int64_t kExpandRows = 1024;
 
+// 4-bit GEMM for decode batches (M <= 256) with the expanded weight in tensor memory.
+bool qgemm_dec_supported(int64_t M, int N, int K, int G);
+int qgemm_dec_impl(const void* X, int64_t M, int N, int K, const void* codes, const void* params, int G,
+                   const void* bias, const void* R, int relu, void* Y, cudaStream_t s);
+
+// Device address of the flag that bounded device-side waits set when they give up.
+int* device_error_ptr();
+
+int splitk_reduce_launch(const float* P, int splits, int64_t M, int N, const void* bias, const void* R, int relu,
+                         void* Y, cudaStream_t s);
+
 // Kernel classes for fg_profile_* (same numbering as the header).
 enum ProfKind { PROF_GEMM = 0, PROF_DECODE_ATTN = 1, PROF_PREFILL_ATTN = 2, PROF_QUANT = 3,
                 PROF_OTHER = 4, PROF_GEMM_DECODE = 5, PROF_LM_HEAD = 6, PROF_NKINDS = 7 };

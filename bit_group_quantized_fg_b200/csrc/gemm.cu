@@ -459,6 +459,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+}  // namespace
+
 int make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t inner,
                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                 CUtensorMapSwizzle swz) {
@@ -474,6 +476,8 @@ int make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int el
   if (r != CUDA_SUCCESS) return fail(FG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
   return FG_OK;
 }
+
+namespace {
 
 template <int MODE, bool F32>
 int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& p, const GemmArgs& args, cudaStream_t s) {
@@ -499,8 +503,31 @@ int pick_splits(int tiles, int k_blocks) {
 
 }  // namespace
 
+int splitk_reduce_launch(const float* P, int splits, int64_t M, int N, const void* bias, const void* R, int relu,
+                         void* Y, cudaStream_t s) {
+  const int64_t MN = M * N;
+  const int grid = int(std::min<int64_t>((MN / 8 + 255) / 256, int64_t(num_sms()) * 8));
+  splitk_reduce_kernel<<<grid, 256, 0, s>>>(P, splits, MN, N, reinterpret_cast<const __half*>(bias),
+                                            reinterpret_cast<const __half*>(R), relu, reinterpret_cast<__half*>(Y));
+  FG_CHECK_LAUNCH("split-K reduce kernel");
+  return FG_OK;
+}
+
 int read_device_error(int* out) {
   return cudaMemcpyFromSymbol(out, g_device_error, sizeof(int)) == cudaSuccess ? FG_OK : FG_ERR_CUDA;
+}
+
+// Device address of the flag, for kernels compiled in other translation units.
+int* device_error_ptr() {
+  static int* ptr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    ptr[dev] = static_cast<int*>(p);
+  }
+  return ptr[dev];
 }
 
 // Split-K partials of one GEMM (0 when the tiles alone fill the GPU).
@@ -598,13 +625,7 @@ int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, c
     else st = out_f32 ? launch<B_F16_K, true>(ta, tb, tp, a, s) : launch<B_F16_K, false>(ta, tb, tp, a, s);
     if (st != FG_OK) return st;
   }
-  if (a.splits > 1) {
-    const int64_t MN = M * N;
-    const int grid = int(std::min<int64_t>((MN / 8 + 255) / 256, int64_t(num_sms()) * 8));
-    splitk_reduce_kernel<<<grid, 256, 0, s>>>(a.partial, a.splits, MN, N, a.bias, a.R, relu,
-                                              reinterpret_cast<__half*>(Y));
-    FG_CHECK_LAUNCH("split-K reduce kernel");
-  }
+  if (a.splits > 1) FG_TRY(splitk_reduce_launch(a.partial, a.splits, M, N, a.bias, a.R, relu, Y, s));
   return FG_OK;
 }
 

@@ -144,7 +144,8 @@ int fg_qgemm(const void* X, int64_t M, const fg_qlinear* W, const void* R, int r
 /* The same tensor-core GEMM over an uncompressed fp16 weight W [K][N] (N contiguous): the
  * "FlexGen" README mirror's benchmark table contrasts FlexGen with and without compression;
  * this is the uncompressed side.  Y[M][N] = [relu](X W + b) [+ R], fp32 accumulation.
- * K % 64 == 0, N % 256 == 0; workspace as fg_qgemm_workspace_bytes(M, N, K). */
+ * K % 64 == 0, N % 256 == 0; workspace >= fg_gemm_f16_workspace_bytes(M, N, K). */
+size_t fg_gemm_f16_workspace_bytes(int64_t M, int N, int K);
 int fg_gemm_f16(const void* X, int64_t M, const void* W, int K, int N, const void* bias,
                 const void* R, int relu, void* Y, void* workspace, size_t ws_bytes, void* stream);
 
@@ -217,6 +218,9 @@ int fg_prefill_layer(const fg_layer* layer, fg_kv_cache* cache, void* x, int B, 
  * (B x L ids, device int32) yields token 1, then gen_len-1 decode steps; out_ids device
  * int32 [B][gen_len].  caches: HOST array of n_layers caches (len reset to 0 here),
  * capacity >= L + gen_len.  Timing uses CUDA events on `stream`; this call synchronizes.
+ * The first call with a given set of pointers, sizes, stream and profiling state runs
+ * eagerly, the second records the prompt pass and the decode steps as two CUDA graphs and
+ * every later one replays them.
  * workspace >= fg_workspace_bytes(model, B, L, gen_len). */
 size_t fg_workspace_bytes(const fg_model* model, int B, int L, int gen_len);
 int fg_generate(const fg_model* model, const int32_t* prompt_ids, int B, int L, int gen_len,
@@ -227,9 +231,13 @@ int fg_generate(const fg_model* model, const int32_t* prompt_ids, int B, int L, 
  * stream).  kind: 0 = dequant GEMM of a prompt pass (M > 256), 1 = decode attention,
  * 2 = prefill attention, 3 = quantize/append, 4 = other (LayerNorm, embedding, argmax),
  * 5 = dequant GEMM of a decode step (M <= 256), 6 = LM head GEMM.  flops and bytes are the
- * algorithmic work of the timed launches.  Enabling adds one event pair per launch;
- * fg_profile_read synchronizes the recorded events. */
+ * algorithmic work of the timed launches.  Enabling adds one event pair per launch (as
+ * event-record nodes inside fg_generate's graphs); fg_profile_read synchronizes the
+ * recorded events. */
 int fg_profile_enable(int on);
+/* Which kinds are timed while profiling is on: bit k selects kind k (default: all).  Timing
+ * a few kinds keeps the recorded graphs close to the unprofiled ones. */
+int fg_profile_select(unsigned kinds);
 int fg_profile_read(int kind, double* total_ms, int64_t* launches, double* flops,
                     double* bytes);
 int fg_profile_reset(void);

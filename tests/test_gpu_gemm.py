@@ -50,10 +50,24 @@ def test_qgemm_matches_oracle(fg, M, N, K, g, relu, resid):
 
 
 def test_qgemm_decode_split_k(fg):
-    """M = 64 rows with few output tiles: the K loop is split and reduced."""
-    assert fg.fg_qgemm_workspace_bytes(64, 4096, 4096) > 0
+    """M = 64 rows with few output tiles: the K loop is split over a thread-block cluster
+    and the partial tiles are summed through distributed shared memory."""
     got, exp = _case(fg, 64, 4096, 4096, 64, False, True, seed=7)
     assert_close_rms(got, exp, what="split-K")
+
+
+@pytest.mark.parametrize("M,N,K,g,relu,resid", [
+    (1, 256, 128, 64, False, True),        # one row
+    (17, 512, 1024, 64, True, True),       # rows not a multiple of 16
+    (144, 768, 512, 32, False, True),      # two row chunks (128 + 16), g 32
+    (256, 512, 640, 128, True, False),     # two full row chunks, g 128
+    (64, 256, 4096, 64, False, False),     # one tile, K split 8 ways
+    (64, 3072, 4096, 64, False, False),    # 12 tiles x 8-way K split
+])
+def test_qgemm_decode_batches(fg, M, N, K, g, relu, resid):
+    """Decode-size GEMMs (M <= 256): weight expanded into tensor memory, swap-AB."""
+    got, exp = _case(fg, M, N, K, g, relu, resid, seed=3 * M + N + K)
+    assert_close_rms(got, exp, what="decode qgemm")
 
 
 def test_qgemm_prefill_size_sampled(fg):

@@ -182,3 +182,31 @@ def test_generate_graph_replay_matches_eager(fg):
         assert all(c.length == L + T - 1 for c in caches)
     assert np.array_equal(results[0][0], results[1][0]) and np.array_equal(results[0][0], results[2][0])
     assert results[0][1] == results[1][1] == results[2][1] > 0   # same kernels, counted once each
+
+
+def test_profiling_inside_graphs_counts_every_launch(fg):
+    """With profiling on, the timing events become nodes of the recorded graphs: an eager
+    call, the capturing call and a replay each report the same launches per kernel class
+    with positive durations."""
+    import torch
+    mo, md = small_model(fg, seed=9, n_layers=2)
+    B, L, T = 2, 10, 4
+    ids = to_dev(fg_synth.token_ids(9, fg_synth.S_IDS, (B, L), mo.vocab))
+    caches = [fg.DeviceKVCache(B, mo.n_heads, mo.head_dim, L + T, 64) for _ in range(mo.n_layers)]
+    out = torch.empty((B, T), dtype=torch.int32, device="cuda")
+    ws = torch.empty((fg.fg_workspace_bytes(md, B, L, T),), dtype=torch.uint8, device="cuda")
+    fg.fg_profile_enable(True)
+    try:
+        per_call = []
+        for _ in range(3):
+            fg.fg_profile_reset()
+            fg.fg_generate(md, ids, T, caches, out_ids=out, workspace=ws)
+            per_call.append({k: fg.fg_profile_read(k) for k in range(7)})
+    finally:
+        fg.fg_profile_enable(False)
+    for k in range(7):
+        n = [c[k]["launches"] for c in per_call]
+        assert n[0] == n[1] == n[2], (k, n)
+        for c in per_call:
+            assert (c[k]["ms"] > 0) == (c[k]["launches"] > 0)
+    assert per_call[2][1]["launches"] == mo.n_layers * (T - 1)   # decode attention per layer and step
