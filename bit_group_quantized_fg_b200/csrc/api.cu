@@ -180,13 +180,11 @@ int check_layer(const fg_layer* L, int h, int* ffn) {
 // Y = [relu](X W_hat + b) [+ R] for a 4-bit weight.  With many rows (a prompt pass) each
 // weight tile is reused by M/128 row tiles, so the weight is first expanded once into an
 // fp16 copy in the workspace (an HBM-bound pass, ~1 % of the GEMM) and the tensor-core GEMM
-// then runs without dequant warps.  Decode batches (M <= 256) run the kernel that expands
-// the weight into tensor memory; the rows in between, the fused kernel that expands it into
-// shared memory.  All compute with the same fp16 values W_hat.
+// then runs without dequant warps; with fewer rows (decode batches included) the fused kernel
+// expands each weight tile into shared memory as it streams the 4-bit weight once.  Both
+// compute with the same fp16 values W_hat.
 int qlinear_run(const void* X, int64_t M, const fg_qlinear& w, const void* R, int relu, void* Y, void* ws,
                 size_t wsb, cudaStream_t s) {
-  if (qgemm_dec_supported(M, w.N, w.K, w.group))
-    return qgemm_dec_impl(X, M, w.N, w.K, w.codes, w.params, w.group, w.bias, R, relu, Y, s);
   const size_t wbytes = (size_t(w.K) * size_t(w.N) * 2 + 255) & ~size_t(255);
   if (M >= kExpandRows && ws != nullptr && wsb >= wbytes && aligned16(ws)) {
     FG_TRY(dequantize_impl(w.codes, w.params, w.K, w.N, w.group, 1, ws, s));

@@ -46,11 +46,6 @@ int num_sms();
 // fp16 tensor-core GEMM (measured break-even ~700 rows on B200).
 constexpr int64_t kExpandRows = 1024;
 
-// 4-bit GEMM for decode batches (M <= 256) with the expanded weight in tensor memory.
-bool qgemm_dec_supported(int64_t M, int N, int K, int G);
-int qgemm_dec_impl(const void* X, int64_t M, int N, int K, const void* codes, const void* params, int G,
-                   const void* bias, const void* R, int relu, void* Y, cudaStream_t s);
-
 // Device address of the flag that bounded device-side waits set when they give up.
 int* device_error_ptr();
 

@@ -50,8 +50,8 @@ def test_qgemm_matches_oracle(fg, M, N, K, g, relu, resid):
 
 
 def test_qgemm_decode_split_k(fg):
-    """M = 64 rows with few output tiles: the K loop is split over a thread-block cluster
-    and the partial tiles are summed through distributed shared memory."""
+    """M = 64 rows with few output tiles: the K loop is split and the fp32 partials are
+    reduced by the epilogue kernel."""
     got, exp = _case(fg, 64, 4096, 4096, 64, False, True, seed=7)
     assert_close_rms(got, exp, what="split-K")
 
@@ -65,7 +65,7 @@ def test_qgemm_decode_split_k(fg):
     (64, 3072, 4096, 64, False, False),    # 12 tiles x 8-way K split
 ])
 def test_qgemm_decode_batches(fg, M, N, K, g, relu, resid):
-    """Decode-size GEMMs (M <= 256): weight expanded into tensor memory, swap-AB."""
+    """Decode-size GEMMs (M <= 256): ragged rows, row tiles, group sizes, deep K splits."""
     got, exp = _case(fg, M, N, K, g, relu, resid, seed=3 * M + N + K)
     assert_close_rms(got, exp, what="decode qgemm")
 
