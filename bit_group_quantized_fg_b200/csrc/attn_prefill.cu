@@ -6,7 +6,9 @@
 // computed flash-style so the L x L scores never reach memory: one CTA per (64-query tile,
 // head, sequence), 4 warps x 16 query rows, key/value tiles of 64 staged in shared
 // memory, S = Q K^T and O += P V on mma.sync m16n8k16 (fp16 in, fp32 accumulate), fp32
-// online softmax in registers.  P is rounded to fp16 for the second product.
+// online softmax in registers.  P is rounded to fp16 for the second product.  The next
+// key tile is copied (cp.async) while the softmax and P V of this one run, the next value
+// tile while the next Q K^T runs.
 #include "fg_common.cuh"
 
 namespace fg {
@@ -38,10 +40,13 @@ __device__ __forceinline__ void cp_async16(uint32_t saddr, const void* g, bool v
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr), "l"(g), "r"(n) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) { return h2_as_u32(__floats2half2_rn(a, b)); }
 
 template <int HD>
-__global__ void __launch_bounds__(128) prefill_attn_kernel(const __half* __restrict__ qkv, int L, int nh,
+__global__ void __launch_bounds__(128, HD == 128 ? 3 : 4) prefill_attn_kernel(const __half* __restrict__ qkv, int L, int nh,
                                                            __half* __restrict__ out) {
   constexpr int LD = HD + 8;  // padded smem row (halves)
   constexpr int NKS = HD / 16;  // k-steps over head dim
@@ -70,16 +75,9 @@ __global__ void __launch_bounds__(128) prefill_attn_kernel(const __half* __restr
   cp_async_wait_all();
   __syncthreads();
 
-  uint32_t qf[NKS][4];
-  {
-    const int r = warp * 16 + (lane & 15);
-#pragma unroll
-    for (int ks = 0; ks < NKS; ++ks) {
-      const int c = ks * 16 + (lane >> 4) * 8;
-      ldsm_x4(static_cast<uint32_t>(__cvta_generic_to_shared(sQ + r * LD + c)), qf[ks][0], qf[ks][1], qf[ks][2],
-              qf[ks][3]);
-    }
-  }
+  // Q fragments are re-read from shared memory at each k-step (registers go to O and S)
+  const uint32_t q_frag_addr =
+      static_cast<uint32_t>(__cvta_generic_to_shared(sQ + (warp * 16 + (lane & 15)) * LD + (lane >> 4) * 8));
 
   float o[NDB][4];
 #pragma unroll
@@ -89,18 +87,22 @@ __global__ void __launch_bounds__(128) prefill_attn_kernel(const __half* __restr
   const int qrow0 = q0 + warp * 16 + g;  // rows qrow0 and qrow0 + 8
 
   const int n_kt = qt + 1;  // causal: key tiles 0..qt
-  for (int kt = 0; kt < n_kt; ++kt) {
-    const int k0 = kt * kKT;
-    __syncthreads();
+  auto load_tile = [&](__half* dst, int k0, int which) {  // which: 1 = K, 2 = V
     for (int i = threadIdx.x; i < kKT * (HD / 8); i += 128) {
       const int r = i / (HD / 8), c = (i % (HD / 8)) * 8;
       const int kj = k0 + r;
       const bool ok = kj < L;
-      const __half* src = base + int64_t(ok ? kj : 0) * row_stride + c;
-      cp_async16(static_cast<uint32_t>(__cvta_generic_to_shared(sK + r * LD + c)), src + h, ok);
-      cp_async16(static_cast<uint32_t>(__cvta_generic_to_shared(sV + r * LD + c)), src + 2 * h, ok);
+      const __half* src = base + int64_t(ok ? kj : 0) * row_stride + c + which * h;
+      cp_async16(static_cast<uint32_t>(__cvta_generic_to_shared(dst + r * LD + c)), src, ok);
     }
-    cp_async_wait_all();
+    cp_async_commit();
+  };
+  load_tile(sK, 0, 1);
+  load_tile(sV, 0, 2);
+  for (int kt = 0; kt < n_kt; ++kt) {
+    const int k0 = kt * kKT;
+    const bool more = kt + 1 < n_kt;
+    cp_async_wait_group<1>();  // this key tile has landed (its value tile may still be in flight)
     __syncthreads();
 
     // S = Q K^T  (16 x 64 per warp)
@@ -109,6 +111,8 @@ __global__ void __launch_bounds__(128) prefill_attn_kernel(const __half* __restr
     for (int i = 0; i < 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
 #pragma unroll
     for (int ks = 0; ks < NKS; ++ks) {
+      uint32_t qa[4];
+      ldsm_x4(q_frag_addr + ks * 32, qa[0], qa[1], qa[2], qa[3]);
 #pragma unroll
       for (int nb2 = 0; nb2 < 4; ++nb2) {  // pairs of 8-key blocks
         const int j = lane >> 3, r = lane & 7;
@@ -116,10 +120,12 @@ __global__ void __launch_bounds__(128) prefill_attn_kernel(const __half* __restr
         const int d = ks * 16 + (j & 1) * 8;
         uint32_t b0, b1, b2, b3;
         ldsm_x4(static_cast<uint32_t>(__cvta_generic_to_shared(sK + key * LD + d)), b0, b1, b2, b3);
-        mma16816(s[2 * nb2], qf[ks], b0, b1);
-        mma16816(s[2 * nb2 + 1], qf[ks], b2, b3);
+        mma16816(s[2 * nb2], qa, b0, b1);
+        mma16816(s[2 * nb2 + 1], qa, b2, b3);
       }
     }
+    __syncthreads();  // every warp is done with this key tile
+    if (more) load_tile(sK, k0 + kKT, 1);
     // scale, mask, online softmax
     float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
@@ -167,7 +173,10 @@ __global__ void __launch_bounds__(128) prefill_attn_kernel(const __half* __restr
       o[i][2] *= alpha[1];
       o[i][3] *= alpha[1];
     }
-    // O += P V
+    // O += P V (the value tile of this step must have landed)
+    if (more) cp_async_wait_group<1>();
+    else cp_async_wait_group<0>();
+    __syncthreads();
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {  // 16 keys per k-step
       uint32_t a[4];
@@ -186,6 +195,8 @@ __global__ void __launch_bounds__(128) prefill_attn_kernel(const __half* __restr
         mma16816(o[2 * db2 + 1], a, b2, b3);
       }
     }
+    __syncthreads();  // every warp is done with this value tile
+    if (more) load_tile(sV, k0 + kKT, 2);
   }
 
   // normalize and store

@@ -18,7 +18,8 @@
 //               the MN-major 128-byte-swizzled operand layout the MMA reads.
 // Other operand modes reuse the skeleton: B as a ready fp16 [K][N] tensor (MN-major, by
 // TMA) or as an fp16 [N][K] tensor (K-major by TMA, the tied LM head).  Tiles are
-// rasterized in bands of 16 M-tiles so a band of X stays in L2 while weights stream.
+// rasterized in bands of row tiles (~48 MB of X) so a band of X stays in L2 while the
+// weight streams past it.
 // With few tiles (decode batches) the K loop is split and fp32 partials are reduced by a
 // second kernel that applies the epilogue.
 #include <algorithm>
@@ -39,7 +40,6 @@ using namespace sm100;
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 64;
-constexpr int kBand = 16;
 constexpr int kABytes = BM * BK * 2;   // 16 KB
 constexpr int kBBytes = BN * BK * 2;   // 32 KB
 constexpr int kCodeBytes = BK * BN / 2; // 8 KB
@@ -70,6 +70,7 @@ struct Cfg {
 struct GemmArgs {
   int M, N, K;
   int m_tiles, n_tiles, k_blocks, splits;
+  int band;         // row tiles per rasterization band
   int total;        // m_tiles * n_tiles * splits
   int G, PB;        // group size, params per k row in a stage
   const __half* bias;
@@ -87,12 +88,12 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t) {
   TileCoord c;
   c.ks = t % a.splits;
   const int r = t / a.splits;
-  const int band_tiles = kBand * a.n_tiles;
+  const int band_tiles = a.band * a.n_tiles;
   const int bi = r / band_tiles;
   const int rr = r - bi * band_tiles;
-  const int mt_in_band = min(kBand, a.m_tiles - bi * kBand);
+  const int mt_in_band = min(a.band, a.m_tiles - bi * a.band);
   const int n = rr / mt_in_band;
-  const int m = bi * kBand + (rr - n * mt_in_band);
+  const int m = bi * a.band + (rr - n * mt_in_band);
   c.m0 = m * BM;
   c.n0 = n * BN;
   c.kb0 = int((int64_t(c.ks) * a.k_blocks) / a.splits);
@@ -109,7 +110,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base_u32 = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024 - (base_u32 & 1023)) & 1023);
-  constexpr int SB = 2;  // B-ring depth (4-bit mode)
+  constexpr int SB = C::kBStages > 0 ? C::kBStages : 1;  // B-ring depth (4-bit mode)
   uint8_t* bring = smem + C::kBRingOff;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBRingOff + C::kBStages * kBBytes);
   uint64_t* full = bars;                   // [S]  TMA stage landed
@@ -341,7 +342,9 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
     }
   } else if (MODE == B_Q4 && warp >= 8) {
     // ------------------------------------------------------------ dequant warps
-    const int dw = warp - 8;       // 0..7: k rows dw, dw+8, ..., dw+56
+    constexpr int DW = C::kDequantWarps > 0 ? C::kDequantWarps : 1;
+    constexpr int RPW = BK / DW;   // k rows per warp: dw, dw + DW, ...
+    const int dw = warp - 8;
     const int nb = lane >> 3;      // 64-wide MN block of the word
     const int ch = lane & 7;       // 16-byte chunk inside the block
     int stage = 0, bs = 0;
@@ -356,16 +359,16 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
         const uint8_t* st = smem + stage * C::kStageBytes;
         const uint32_t* codes = reinterpret_cast<const uint32_t*>(st + C::kCodeOff);
         const uint32_t* prm = reinterpret_cast<const uint32_t*>(st + C::kParamOff);
-        uint32_t w[8], p[8];
+        uint32_t w[RPW], p[RPW];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int row = dw + 8 * i;
+        for (int i = 0; i < RPW; ++i) {
+          const int row = dw + DW * i;
           w[i] = codes[row * (BN / 8) + lane];
           p[i] = prm[row * args.PB + pcol];
         }
-        uint32_t o[8][4];
+        uint32_t o[RPW][4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < RPW; ++i) {
           const __half2 pr = u32_as_h2(p[i]);
           dequant8_interleaved(w[i], __high2half2(pr), __low2half2(pr), o[i]);
         }
@@ -373,8 +376,8 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
         if (!mbar_wait(&bempty[bs], bphase ^ 1, abort_flag, &g_device_error, 64)) { ok = false; break; }
         uint8_t* bt = bring + bs * kBBytes;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int row = dw + 8 * i;  // k index inside the block
+        for (int i = 0; i < RPW; ++i) {
+          const int row = dw + DW * i;  // k index inside the block
           const int kg = row >> 3, rr = row & 7;
           uint4* dst = reinterpret_cast<uint4*>(bt + nb * 8192 + kg * 1024 + rr * 128 + ((ch ^ rr) << 4));
           *dst = make_uint4(o[i][0], o[i][1], o[i][2], o[i][3]);
@@ -581,6 +584,9 @@ int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, c
   a.n_tiles = (N + BN - 1) / BN;
   a.k_blocks = K / BK;
   a.splits = out_f32 ? 1 : pick_splits(a.m_tiles * a.n_tiles, a.k_blocks);
+  // Rasterization: bands of row tiles whose X rows (band x 128 x K fp16) take ~48 MB of the
+  // 126 MB L2 while the weight tiles stream past them; the weight is read once per band.
+  a.band = int(std::min<int64_t>(64, std::max<int64_t>(16, (int64_t(48) << 20) / (int64_t(BM) * K * 2))));
   a.total = a.m_tiles * a.n_tiles * a.splits;
   a.G = G;
   a.PB = G == 32 ? 8 : 4;

@@ -61,11 +61,16 @@ def test_decode_attention_t3_and_outliers(fg):
         assert_close_rms(to_np(out), oracle.decode_attention(q[:, :512], ref, 129), what=dist)
 
 
-def test_decode_attention_sampled_full_size(fg):
-    """Config-2 decode shape (B 64, 32 heads x 128, context 543) with sampled (b, head)
-    pairs checked against the oracle; the rest checked for finiteness."""
+@pytest.mark.parametrize("B,nh,S", [
+    (64, 32, 543),    # OPT-6.7B shape, batch 64, last decode step
+    (256, 56, 543),   # OPT-30B shape, batch 256
+    (144, 96, 543),   # OPT-175B shape, batch 144
+])
+def test_decode_attention_sampled_full_size(fg, B, nh, S):
+    """Decode attention at the configurations' full shapes (head dim 128, group 64, context
+    543): sampled sequences checked against the oracle, the rest for finiteness."""
     import torch
-    B, nh, hd, g, S = 64, 32, 128, 64, 543
+    hd, g = 128, 64
     h = nh * hd
     from fg_synth import gpu as sg
     kv = torch.empty((B * S, 2 * h), dtype=torch.float16, device="cuda")
@@ -77,13 +82,13 @@ def test_decode_attention_sampled_full_size(fg):
     out = fg.fg_decode_attention(q, 3 * h, cache)
     torch.cuda.synchronize()
     assert bool(torch.isfinite(out.float()).all())
-    qn = to_np(q)
-    for b in (0, 31, 63):
+    for b in (0, B // 2 - 1, B - 1):
+        qb = fg_synth.values(77, 2, np.arange(b * 3 * h, b * 3 * h + h), "normal", 1.0, 3 * h).reshape(1, h)
         rows = fg_synth.values(77, 1, np.arange(b * S * 2 * h, (b + 1) * S * 2 * h), "normal", 1.0, 2 * h)
         rows = rows.reshape(1, S, 2 * h)
         ref = oracle.KVCache(1, nh, hd, g, S)
         oracle.kv_append(ref, rows[:, :, :h], rows[:, :, h:], 0)
-        exp = oracle.decode_attention(qn[b:b + 1, :h], ref, S)
+        exp = oracle.decode_attention(qb, ref, S)
         assert_close_rms(to_np(out[b:b + 1]), exp, what=f"row {b}")
 
 

@@ -70,30 +70,65 @@ def test_qgemm_decode_batches(fg, M, N, K, g, relu, resid):
     assert_close_rms(got, exp, what="decode qgemm")
 
 
-def test_qgemm_prefill_size_sampled(fg):
-    """Config-2 prefill QKV shape (M 32768, N 12288, K 4096) on sampled outputs."""
+def oracle_weight_columns(seed, stream, K, N, g, cols, scale=0.02):
+    """W_hat[:, cols] (float64 [K, len(cols)]) of a seeded N(0, scale) weight [K][N], quantized
+    by the oracle group by group: only the groups holding ``cols`` are generated on the CPU."""
+    cols = np.asarray(cols)
+    out = np.empty((K, len(cols)), np.float64)
+    for gi in np.unique(cols // g):
+        c0 = int(gi) * g
+        idx = (np.arange(K)[:, None] * N + c0 + np.arange(g)[None, :]).ravel()
+        wg = fg_synth.values(seed, stream, idx, "normal", scale).reshape(K, g)
+        codes, params = oracle.quantize_pack(wg, g, axis=1)
+        wh = oracle.dequantize(codes, params, K, g, g, 1).astype(np.float64)
+        sel = np.nonzero(cols // g == gi)[0]
+        out[:, sel] = wh[:, cols[sel] - c0]
+    return out
+
+
+def _sampled_qgemm(fg, M, N, K, g, seed, rows, cols):
+    """Y = X W_hat + b at full size on the GPU (inputs from the GPU twin of the generator);
+    the oracle recomputes the sampled rows x columns from CPU-generated inputs."""
     import torch
     from fg_synth import gpu as sg
-    M, N, K, g = 32768, 12288, 4096, 64
     x = torch.empty((M, K), dtype=torch.float16, device="cuda")
-    sg.fill(x, 11, 1, "normal", 1.0)
+    sg.fill(x, seed, 1, "normal", 1.0)
     w = torch.empty((K, N), dtype=torch.float16, device="cuda")
-    sg.fill(w, 11, 2, "normal", 0.02)
+    sg.fill(w, seed, 2, "normal", 0.02)
     b = torch.empty((N,), dtype=torch.float16, device="cuda")
-    sg.fill(b, 11, 3, "normal", 0.5)
+    sg.fill(b, seed, 3, "normal", 0.5)
     lin = fg.DeviceQLinear.from_fp16(w, b, g)
     del w
     y = fg.fg_qgemm(x, lin)
     torch.cuda.synchronize()
     assert bool(torch.isfinite(y.float()).all())
+    wcols = oracle_weight_columns(seed, 2, K, N, g, cols)
+    bh = fg_synth.values(seed, 3, np.arange(N), "normal", 0.5)
+    xr = fg_synth.values(seed, 1, (rows[:, None] * K + np.arange(K)[None, :]).ravel(), "normal", 1.0).reshape(-1, K)
+    exp = (xr.astype(np.float64) @ wcols + bh[cols].astype(np.float64)).astype(np.float16)
+    return to_np(y)[rows][:, cols], exp
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (256, 21504, 7168),    # OPT-30B-shaped QKV at batch 256
+    (144, 49152, 12288),   # OPT-175B-shaped fc1 at batch 144
+])
+def test_qgemm_large_decode_sampled(fg, M, N, K):
+    """Decode GEMMs at the larger configurations' shapes, on sampled outputs."""
+    rng = np.random.default_rng(M)
+    rows = np.concatenate([[0, M - 1], rng.integers(0, M, 6)])
+    cols = np.concatenate([[0, N - 1], rng.integers(0, N, 14)])
+    got, exp = _sampled_qgemm(fg, M, N, K, 64, M + 5, rows, cols)
+    assert_close_rms(got, exp, what="sampled decode GEMM")
+
+
+def test_qgemm_prefill_size_sampled(fg):
+    """Config-2 prefill QKV shape (M 32768, N 12288, K 4096) on sampled outputs."""
+    M, N, K = 32768, 12288, 4096
     rng = np.random.default_rng(0)
     rows = np.concatenate([[0, 127, 128, M - 1], rng.integers(0, M, 12)])
     cols = np.concatenate([[0, 255, 256, N - 1], rng.integers(0, N, 28)])
-    ref_lin = oracle.QLinear(to_np(lin.codes), to_np(lin.params), to_np(b), K, N, g)
-    wcols = ref_lin.columns(cols)                      # [K, ncols] exact fp16 weights
-    xr = fg_synth.values(11, 1, (rows[:, None] * K + np.arange(K)[None, :]).ravel(), "normal", 1.0).reshape(-1, K)
-    exp = (xr.astype(np.float64) @ wcols + to_np(b)[cols].astype(np.float64)).astype(np.float16)
-    got = to_np(y)[rows][:, cols]
+    got, exp = _sampled_qgemm(fg, M, N, K, 64, 11, rows, cols)
     assert_close_rms(got, exp, what="sampled prefill GEMM")
 
 
