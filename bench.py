@@ -356,6 +356,36 @@ def kernel_case(args):
     print(json.dumps(res))
 
 
+# ---------------------------------------------------------------------------- replicas
+# N > 1: N independent replicas, one process per GPU; each generates its own batch (seeded by
+# its rank) and the only cross-rank traffic is the barrier and the max of the timings.
+def replica_env():
+    """(world, rank, local_rank) from the torchrun environment (1, 0, 0 without it)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def replica_seed(rank):
+    """Seed of a replica's prompt ids: every rank generates a different batch."""
+    return SEED + rank
+
+
+def max_over_ranks(x, device):
+    """The largest per-rank value (the slowest rank's time) over the process group, if any."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank_step, world, steps, ms_max):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank_step * world * steps / (ms_max / 1000.0)
+
+
 # ---------------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -372,9 +402,7 @@ def main():
     args = ap.parse_args()
     if args.case != "generate":
         return kernel_case(args)
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = replica_env()
     c = CFG
     config = {"workload": "OPT-6.7B-shaped decoder, 4-bit weights + 4-bit KV (group 64), batch 64 per GPU, "
                           "prompt 512, generate 32", "layers": c["n_layers"], "hidden": c["hidden"],
@@ -413,7 +441,7 @@ def main():
     from fg_synth import gpu as sg
     import fg_synth
     ids = torch.empty((B, L), dtype=torch.int32, device=dev)
-    sg.fill_ids(ids, SEED + rank, fg_synth.S_IDS, c["vocab"])
+    sg.fill_ids(ids, replica_seed(rank), fg_synth.S_IDS, c["vocab"])
     out = torch.empty((B, T), dtype=torch.int32, device=dev)
     ws = torch.empty((fg.fg_workspace_bytes(model, B, L, T),), dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
@@ -449,15 +477,10 @@ def main():
         e1.record(stream)
         barrier()
     launches = fg.fg_launch_count() - launches0
-    ms_total = e0.elapsed_time(e1)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(e0.elapsed_time(e1), dev)
     ms_step = ms_total / args.steps
     tokens_step = B * T * world
-    value = tokens_step / (ms_step / 1000.0)
+    value = job_throughput(B * T, world, args.steps, ms_total)
     prof = {fg.PROF_NAMES[k]: fg.fg_profile_read(k) for k in range(7)}
     clocks = clk.summary()
 
@@ -483,13 +506,8 @@ def main():
     fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
     breakdown = {fg.PROF_NAMES[k]: fg.fg_profile_read(k) for k in range(7)}
     fg.fg_profile_enable(False)
-    ms_e2e = e2.elapsed_time(e3)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
-    e2e_value = tokens_step * args.steps / (ms_e2e / 1000.0)
+    ms_e2e = max_over_ranks(e2.elapsed_time(e3), dev)
+    e2e_value = job_throughput(B * T, world, args.steps, ms_e2e)
 
     # ---- quantizer GB/s on a 1 GiB fp16 tensor (group 64), bytes = 2 + 0.5 + 4/64 per element
     xq = torch.empty((131072, 4096), dtype=torch.float16, device=dev)

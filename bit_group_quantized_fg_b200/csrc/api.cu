@@ -27,7 +27,7 @@ int argmax_impl(const float*, int, int, int32_t*, int64_t, cudaStream_t);
 size_t qgemm_ws_bytes(int64_t, int, int);
 size_t splitk_ws_bytes(int64_t, int, int);
 int gemm_impl(int, const void*, int64_t, int, int, const void*, const void*, int, const void*, const void*, int,
-              void*, bool, void*, size_t, cudaStream_t);
+              void*, bool, void*, size_t, cudaStream_t, bool);
 int read_device_error(int*);
 
 // ---------------------------------------------------------------- errors
@@ -183,15 +183,18 @@ int check_layer(const fg_layer* L, int h, int* ffn) {
 // then runs without dequant warps; with fewer rows (decode batches included) the fused kernel
 // expands each weight tile into shared memory as it streams the 4-bit weight once.  Both
 // compute with the same fp16 values W_hat.
+// w_ready: the weight was not written by the kernel just before this one in the stream
+// (true inside the layer calls, whose first kernel is a LayerNorm), so its tiles may be
+// requested before the previous kernel finishes.
 int qlinear_run(const void* X, int64_t M, const fg_qlinear& w, const void* R, int relu, void* Y, void* ws,
-                size_t wsb, cudaStream_t s) {
+                size_t wsb, cudaStream_t s, bool w_ready = false) {
   const size_t wbytes = (size_t(w.K) * size_t(w.N) * 2 + 255) & ~size_t(255);
   if (M >= kExpandRows && ws != nullptr && wsb >= wbytes && aligned16(ws)) {
     FG_TRY(dequantize_impl(w.codes, w.params, w.K, w.N, w.group, 1, ws, s));
     return gemm_impl(1, X, M, w.N, w.K, ws, nullptr, 0, w.bias, R, relu, Y, false,
-                     reinterpret_cast<uint8_t*>(ws) + wbytes, wsb - wbytes, s);
+                     reinterpret_cast<uint8_t*>(ws) + wbytes, wsb - wbytes, s, false);  // weight just written
   }
-  return gemm_impl(0, X, M, w.N, w.K, w.codes, w.params, w.group, w.bias, R, relu, Y, false, ws, wsb, s);
+  return gemm_impl(0, X, M, w.N, w.K, w.codes, w.params, w.group, w.bias, R, relu, Y, false, ws, wsb, s, w_ready);
 }
 
 size_t gemm_ws_for_layer(int64_t M, int h, int F) {
@@ -247,13 +250,13 @@ int decode_layer_impl(const fg_layer* layer, fg_kv_cache* cache, const void* x_i
   auto* qkvh = reinterpret_cast<__half*>(qkv);
 
   FG_TRY(layernorm_impl(x_in, B, h, layer->ln1_g, layer->ln1_b, h1, s));
-  FG_TRY(qlinear_run(h1, B, layer->qkv, nullptr, 0, qkv, gws, gws_b, s));
+  FG_TRY(qlinear_run(h1, B, layer->qkv, nullptr, 0, qkv, gws, gws_b, s, true));
   FG_TRY(kv_append_impl(cache, qkvh + h, qkvh + 2 * h, 3 * int64_t(h), 1, s));
   FG_TRY(decode_attention_impl(qkv, 3 * int64_t(h), cache, att, aws, aws_b, s));
-  FG_TRY(qlinear_run(att, B, layer->out, x_in, 0, x1, gws, gws_b, s));
+  FG_TRY(qlinear_run(att, B, layer->out, x_in, 0, x1, gws, gws_b, s, true));
   FG_TRY(layernorm_impl(x1, B, h, layer->ln2_g, layer->ln2_b, h2, s));
-  FG_TRY(qlinear_run(h2, B, layer->fc1, nullptr, 1, f, gws, gws_b, s));
-  FG_TRY(qlinear_run(f, B, layer->fc2, x1, 0, x_out, gws, gws_b, s));
+  FG_TRY(qlinear_run(h2, B, layer->fc1, nullptr, 1, f, gws, gws_b, s, true));
+  FG_TRY(qlinear_run(f, B, layer->fc2, x1, 0, x_out, gws, gws_b, s, true));
   return FG_OK;
 }
 
@@ -280,13 +283,13 @@ int prefill_layer_impl(const fg_layer* layer, fg_kv_cache* cache, void* x, int B
   auto* qkvh = reinterpret_cast<__half*>(qkv);
 
   FG_TRY(layernorm_impl(x, BL, h, layer->ln1_g, layer->ln1_b, hn, s));
-  FG_TRY(qlinear_run(hn, BL, layer->qkv, nullptr, 0, qkv, gws, gws_b, s));
+  FG_TRY(qlinear_run(hn, BL, layer->qkv, nullptr, 0, qkv, gws, gws_b, s, true));
   FG_TRY(kv_append_impl(cache, qkvh + h, qkvh + 2 * h, 3 * int64_t(h), L, s));
   FG_TRY(prefill_attention_impl(qkv, B, L, cache->n_heads, cache->head_dim, att, s));
-  FG_TRY(qlinear_run(att, BL, layer->out, x, 0, x1, gws, gws_b, s));
+  FG_TRY(qlinear_run(att, BL, layer->out, x, 0, x1, gws, gws_b, s, true));
   FG_TRY(layernorm_impl(x1, BL, h, layer->ln2_g, layer->ln2_b, hn, s));
-  FG_TRY(qlinear_run(hn, BL, layer->fc1, nullptr, 1, f, gws, gws_b, s));
-  FG_TRY(qlinear_run(f, BL, layer->fc2, x1, 0, x, gws, gws_b, s));
+  FG_TRY(qlinear_run(hn, BL, layer->fc1, nullptr, 1, f, gws, gws_b, s, true));
+  FG_TRY(qlinear_run(f, BL, layer->fc2, x1, 0, x, gws, gws_b, s, true));
   return FG_OK;
 }
 
@@ -294,7 +297,7 @@ namespace {
 size_t lm_ws(int B, int V) { return align256(size_t(B) * V * 4) + 256; }
 
 int lm_head_impl(const void* x, int B, int hidden, const void* E, int V, float* logits, int32_t* tokens,
-                 int64_t tok_stride, void* ws, size_t wsb, cudaStream_t s) {
+                 int64_t tok_stride, void* ws, size_t wsb, cudaStream_t s, bool w_ready = false) {
   if (!x || !E || !tokens) return fail(FG_ERR_INVALID_ARG, "null pointer");
   if (B <= 0 || V <= 0 || hidden <= 0 || hidden % 64) return fail(FG_ERR_SHAPE, "bad LM head shape");
   float* lg = logits;
@@ -303,7 +306,7 @@ int lm_head_impl(const void* x, int B, int hidden, const void* E, int V, float* 
     lg = reinterpret_cast<float*>(ws);
   }
   if (!aligned16(lg)) return fail(FG_ERR_ALIGN, "logits must be 16-byte aligned");
-  FG_TRY(gemm_impl(2, x, B, V, hidden, E, nullptr, 0, nullptr, nullptr, 0, lg, true, nullptr, 0, s));
+  FG_TRY(gemm_impl(2, x, B, V, hidden, E, nullptr, 0, nullptr, nullptr, 0, lg, true, nullptr, 0, s, w_ready));
   return argmax_impl(lg, B, V, tokens, tok_stride, s);
 }
 
@@ -476,7 +479,7 @@ int generate_impl(const fg_model* m, const int32_t* ids, int B, int L, int T, in
     FG_CHECK_CUDA(cudaMemcpy2DAsync(xd, size_t(h) * 2, reinterpret_cast<uint8_t*>(x) + size_t(L - 1) * h * 2,
                                     size_t(L) * h * 2, size_t(h) * 2, B, cudaMemcpyDeviceToDevice, st_));
     FG_TRY(layernorm_impl(xd, B, h, m->lnf_g, m->lnf_b, xn, st_));
-    return lm_head_impl(xn, B, h, m->embed, m->vocab, nullptr, out, T, lgw, lm_ws(B, m->vocab), st_);
+    return lm_head_impl(xn, B, h, m->embed, m->vocab, nullptr, out, T, lgw, lm_ws(B, m->vocab), st_, true);
   };
   auto decode_seq = [&](cudaStream_t st_) -> int {
     for (int j = 1; j < T; ++j) {
@@ -484,7 +487,7 @@ int generate_impl(const fg_model* m, const int32_t* ids, int B, int L, int T, in
       FG_TRY(embed_impl(out + (j - 1), B, 1, T, L + j - 1, m->embed, m->pos_embed, h, xd, st_));
       for (int l = 0; l < m->n_layers; ++l) FG_TRY(decode_layer_impl(&m->layers[l], &caches[l], xd, xd, B, lws, layer_b, st_));
       FG_TRY(layernorm_impl(xd, B, h, m->lnf_g, m->lnf_b, xn, st_));
-      FG_TRY(lm_head_impl(xn, B, h, m->embed, m->vocab, nullptr, out + j, T, lgw, lm_ws(B, m->vocab), st_));
+      FG_TRY(lm_head_impl(xn, B, h, m->embed, m->vocab, nullptr, out + j, T, lgw, lm_ws(B, m->vocab), st_, true));
     }
     return FG_OK;
   };
@@ -606,7 +609,8 @@ size_t fg_gemm_f16_workspace_bytes(int64_t M, int N, int K) { return splitk_ws_b
 
 int fg_gemm_f16(const void* X, int64_t M, const void* W, int K, int N, const void* bias, const void* R, int relu,
                 void* Y, void* workspace, size_t ws_bytes, void* stream) {
-  return gemm_impl(1, X, M, N, K, W, nullptr, 0, bias, R, relu, Y, false, workspace, ws_bytes, as_stream(stream));
+  return gemm_impl(1, X, M, N, K, W, nullptr, 0, bias, R, relu, Y, false, workspace, ws_bytes, as_stream(stream),
+                   false);
 }
 
 size_t fg_decode_attention_workspace_bytes(int B, int n_heads, int head_dim, int ctx) {

@@ -81,6 +81,7 @@ __global__ void __launch_bounds__(kThreads) decode_attn_mma_kernel(
     const __half2* __restrict__ kp, const uint8_t* __restrict__ vc, const __half2* __restrict__ vp,
     int nh, int cap, int S, int chunk_len, __half* __restrict__ out, float* __restrict__ part_ml,
     float* __restrict__ part_acc) {
+  pdl_wait();  // the previous kernel in the stream has finished (see fg_launch)
   using C = AttnMma<HD, G>;
   constexpr int NG = C::NG, KW = C::KW, KS = C::KS, MT = C::MT, DPT = C::DPT, VW = C::VW, TB = C::TB;
   __shared__ float red_v[kWarps][HD];
@@ -366,6 +367,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
                                                              const float* __restrict__ part_acc,
                                                              int n_bh, int n_chunks, int nh,
                                                              __half* __restrict__ out) {
+  pdl_wait();  // the previous kernel in the stream has finished (see fg_launch)
   const int bh = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (bh >= n_bh) return;
@@ -444,7 +446,7 @@ int decode_attention_impl(const void* q, int64_t q_stride, const fg_kv_cache* c,
   auto* kc8 = reinterpret_cast<const uint8_t*>(c->k_codes);
   auto* vc8 = reinterpret_cast<const uint8_t*>(c->v_codes);
 #define FG_ATTN_LAUNCH(HD_, G_)                                                                      \
-  decode_attn_mma_kernel<HD_, G_><<<grid, kThreads, smem, s>>>(qh, q_stride, kc8, kp, vc8, vp, nh, \
+  FG_LAUNCH("decode attention kernel", decode_attn_mma_kernel<HD_, G_>, dim3(grid), dim3(kThreads), size_t(smem), s, qh, q_stride, kc8, kp, vc8, vp, nh, \
                                                                 c->capacity, S, chunk_len, o, ml, acc)
   if (hd == 128 && G == 128) FG_ATTN_LAUNCH(128, 128);
   else if (hd == 128 && G == 64) FG_ATTN_LAUNCH(128, 64);
@@ -452,14 +454,12 @@ int decode_attention_impl(const void* q, int64_t q_stride, const fg_kv_cache* c,
   else if (hd == 64 && G == 64) FG_ATTN_LAUNCH(64, 64);
   else FG_ATTN_LAUNCH(64, 32);
 #undef FG_ATTN_LAUNCH
-  FG_CHECK_LAUNCH("decode attention kernel");
   if (nc > 1) {
     const int n_bh = B * nh;
     if (hd == 128)
-      decode_combine_kernel<128><<<(n_bh + 3) / 4, 128, 0, s>>>(ml, acc, n_bh, nc, nh, o);
+      FG_LAUNCH("decode combine kernel", decode_combine_kernel<128>, dim3((n_bh + 3) / 4), dim3(128), size_t(0), s, ml, acc, n_bh, nc, nh, o);
     else
-      decode_combine_kernel<64><<<(n_bh + 3) / 4, 128, 0, s>>>(ml, acc, n_bh, nc, nh, o);
-    FG_CHECK_LAUNCH("decode combine kernel");
+      FG_LAUNCH("decode combine kernel", decode_combine_kernel<64>, dim3((n_bh + 3) / 4), dim3(128), size_t(0), s, ml, acc, n_bh, nc, nh, o);
   }
   return FG_OK;
 }

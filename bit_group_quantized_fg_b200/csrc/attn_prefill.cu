@@ -48,6 +48,7 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) { return h2_as_u32
 template <int HD>
 __global__ void __launch_bounds__(128, HD == 128 ? 3 : 4) prefill_attn_kernel(const __half* __restrict__ qkv, int L, int nh,
                                                            __half* __restrict__ out) {
+  pdl_wait();  // the previous kernel in the stream has finished (see fg_launch)
   constexpr int LD = HD + 8;  // padded smem row (halves)
   constexpr int NKS = HD / 16;  // k-steps over head dim
   constexpr int NDB = HD / 8;   // n-blocks over head dim
@@ -231,13 +232,12 @@ int prefill_attention_impl(const void* qkv, int B, int L, int nh, int hd, void* 
       FG_CHECK_CUDA(cudaFuncSetAttribute(prefill_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)));
       set = true;
     }
-    prefill_attn_kernel<128><<<grid, 128, smem, s>>>(reinterpret_cast<const __half*>(qkv), L, nh,
+    FG_LAUNCH("prefill attention kernel", prefill_attn_kernel<128>, dim3(grid), dim3(128), size_t(smem), s, reinterpret_cast<const __half*>(qkv), L, nh,
                                                       reinterpret_cast<__half*>(out));
   } else {
-    prefill_attn_kernel<64><<<grid, 128, smem, s>>>(reinterpret_cast<const __half*>(qkv), L, nh,
+    FG_LAUNCH("prefill attention kernel", prefill_attn_kernel<64>, dim3(grid), dim3(128), size_t(smem), s, reinterpret_cast<const __half*>(qkv), L, nh,
                                                      reinterpret_cast<__half*>(out));
   }
-  FG_CHECK_LAUNCH("prefill attention kernel");
   return FG_OK;
 }
 

@@ -37,6 +37,38 @@ void count_launch();
     if (_s != FG_OK) return _s;      \
   } while (0)
 
+// Every kernel of the library is launched with programmatic stream serialization: a kernel
+// may start (prologue, loads of data no earlier kernel writes) while the previous kernel
+// in the stream finishes, and waits in pdl_wait() before it touches that kernel's results
+// or writes memory the previous kernel may still read.  Every kernel calls pdl_wait(), so
+// completion stays ordered along the stream.
+template <typename... KArgs, typename... Args>
+inline cudaError_t fg_launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+#define FG_LAUNCH(what, ...)                                  \
+  do {                                                        \
+    ::fg::count_launch();                                     \
+    cudaError_t _e = ::fg::fg_launch(__VA_ARGS__);            \
+    if (_e != cudaSuccess) return ::fg::cuda_fail(_e, what);  \
+  } while (0)
+
+// Waits until the previous kernel in the stream has completed and its writes are visible
+// (no-op for a kernel launched without programmatic serialization).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 

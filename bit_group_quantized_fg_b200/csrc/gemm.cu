@@ -71,6 +71,7 @@ struct GemmArgs {
   int M, N, K;
   int m_tiles, n_tiles, k_blocks, splits;
   int band;         // row tiles per rasterization band
+  int prefetch_w;   // weight tiles may be requested before the previous kernel completes
   int total;        // m_tiles * n_tiles * splits
   int G, PB;        // group size, params per k row in a stage
   const __half* bias;
@@ -165,31 +166,60 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
       uint32_t pend_phase[S];
 #pragma unroll
       for (int i = 0; i < S; ++i) { pend[i] = false; pend_phase[i] = 0; }
+      // the weight operand of k-block kb of tile c into stage buffer st
+      auto load_w = [&](uint8_t* st, const TileCoord& c, int kb, uint64_t* bar) {
+        if (MODE == B_Q4) {
+          tma_load_2d(st + C::kCodeOff, &tm_b, c.n0 / 2, kb * BK, bar);
+          const int px = (c.n0 / args.G) & ~3;
+          tma_load_2d(st + C::kParamOff, &tm_p, px, kb * BK, bar);
+        } else if (MODE == B_F16_MN) {
+#pragma unroll
+          for (int j = 0; j < BN / 64; ++j) tma_load_2d(st + kABytes + j * 8192, &tm_b, c.n0 + 64 * j, kb * BK, bar);
+        } else {
+          tma_load_2d(st + kABytes, &tm_b, kb * BK, c.n0, bar);
+        }
+      };
+      // Weights are never written by an earlier kernel: the first stages' weight tiles are
+      // requested before waiting for the previous kernel, whose output X may still be in
+      // the making (programmatic dependent launch).
+      int pre = 0;
+      if (args.prefetch_w && int(blockIdx.x) < args.total) {
+        const TileCoord c0 = tile_coord(args, blockIdx.x);
+        pre = min(S, c0.kb1 - c0.kb0);
+        for (int i = 0; i < pre; ++i) {
+          mbar_expect_tx(&full[i], tx);
+          load_w(smem + i * C::kStageBytes, c0, c0.kb0 + i, &full[i]);
+        }
+      }
+      pdl_wait();
+      int issued = 0;
       for (int t = blockIdx.x; t < args.total && ok; t += gridDim.x) {
         const TileCoord c = tile_coord(args, t);
-        for (int kb = c.kb0; kb < c.kb1; ++kb) {
+        for (int kb = c.kb0; kb < c.kb1; ++kb, ++issued) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, &g_device_error, 1)) { ok = false; break; }
           uint8_t* st = smem + stage * C::kStageBytes;
-          mbar_expect_tx(&full[stage], tx);
-          tma_load_2d(st, &tm_a, kb * BK, c.m0, &full[stage]);
-          if (MODE == B_Q4) {
-            tma_load_2d(st + C::kCodeOff, &tm_b, c.n0 / 2, kb * BK, &full[stage]);
-            const int px = (c.n0 / args.G) & ~3;
-            tma_load_2d(st + C::kParamOff, &tm_p, px, kb * BK, &full[stage]);
-          } else if (MODE == B_F16_MN) {
-#pragma unroll
-            for (int j = 0; j < BN / 64; ++j)
-              tma_load_2d(st + kABytes + j * 8192, &tm_b, c.n0 + 64 * j, kb * BK, &full[stage]);
-          } else {
-            tma_load_2d(st + kABytes, &tm_b, kb * BK, c.n0, &full[stage]);
+          if (issued >= pre) {
+            mbar_expect_tx(&full[stage], tx);
+            load_w(st, c, kb, &full[stage]);
           }
+          tma_load_2d(st, &tm_a, kb * BK, c.m0, &full[stage]);
           pend[stage] = true;
           pend_phase[stage] = phase;
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
       }
       if (*abort_flag) {
-        // let every copy this thread issued land before the CTA exits
+        // stages whose weight tiles were requested up front but whose X copy was never
+        // issued get it now, so that their barriers complete; then let every copy this
+        // thread issued land before the CTA exits
+        if (issued < pre) {
+          const TileCoord c0 = tile_coord(args, blockIdx.x);
+          for (int i = issued; i < pre; ++i) {
+            tma_load_2d(smem + i * C::kStageBytes, &tm_a, (c0.kb0 + i) * BK, c0.m0, &full[i]);
+            pend[i] = true;
+            pend_phase[i] = 0;
+          }
+        }
         for (int i = 0; i < S; ++i)
           if (pend[i]) mbar_wait_drain(&full[i], pend_phase[i]);
       }
@@ -403,6 +433,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
 __global__ void splitk_reduce_kernel(const float* __restrict__ P, int splits, int64_t MN, int N,
                                      const __half* __restrict__ bias, const __half* __restrict__ R,
                                      int relu, __half* __restrict__ Y) {
+  pdl_wait();  // the previous kernel in the stream has finished (see fg_launch)
   const int64_t n8 = MN / 8;
   for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += int64_t(gridDim.x) * blockDim.x) {
     float v[8];
@@ -491,8 +522,7 @@ int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& p, con
     attr_set = true;
   }
   const int grid = std::min(args.total, num_sms());
-  gemm_tc_kernel<MODE, F32><<<grid, C::kThreads, C::kSmem, s>>>(a, b, p, args);
-  FG_CHECK_LAUNCH("tcgen05 gemm kernel");
+  FG_LAUNCH("tcgen05 gemm kernel", gemm_tc_kernel<MODE, F32>, dim3(grid), dim3(C::kThreads), size_t(C::kSmem), s, a, b, p, args);
   return FG_OK;
 }
 
@@ -510,9 +540,8 @@ int splitk_reduce_launch(const float* P, int splits, int64_t M, int N, const voi
                          void* Y, cudaStream_t s) {
   const int64_t MN = M * N;
   const int grid = int(std::min<int64_t>((MN / 8 + 255) / 256, int64_t(num_sms()) * 8));
-  splitk_reduce_kernel<<<grid, 256, 0, s>>>(P, splits, MN, N, reinterpret_cast<const __half*>(bias),
+  FG_LAUNCH("split-K reduce kernel", splitk_reduce_kernel, dim3(grid), dim3(256), size_t(0), s, P, splits, MN, N, reinterpret_cast<const __half*>(bias),
                                             reinterpret_cast<const __half*>(R), relu, reinterpret_cast<__half*>(Y));
-  FG_CHECK_LAUNCH("split-K reduce kernel");
   return FG_OK;
 }
 
@@ -555,7 +584,7 @@ size_t qgemm_ws_bytes(int64_t M, int N, int K) {
 // mode: 0 = 4-bit weight W (codes/params), 1 = fp16 [K][N] weight, 2 = fp16 [N][K] weight.
 int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, const void* wparams, int G,
               const void* bias, const void* R, int relu, void* Y, bool out_f32, void* ws, size_t ws_bytes,
-              cudaStream_t s) {
+              cudaStream_t s, bool w_ready) {
   if (!X || !w || !Y) return fail(FG_ERR_INVALID_ARG, "null pointer");
   if (M < 0 || N <= 0 || K <= 0) return fail(FG_ERR_SHAPE, "bad GEMM shape");
   if (K % BK) return fail(FG_ERR_SHAPE, "K must be a multiple of 64");
@@ -594,6 +623,7 @@ int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, c
   a.R = reinterpret_cast<const __half*>(R);
   a.relu = relu;
   a.Y = Y;
+  a.prefetch_w = w_ready ? 1 : 0;
   a.partial = nullptr;
   if (a.splits > 1) {
     const size_t need = size_t(a.splits) * size_t(M) * size_t(N) * sizeof(float);

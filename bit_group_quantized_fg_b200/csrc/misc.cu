@@ -28,6 +28,7 @@ __global__ void __launch_bounds__(kLnThreads) layernorm_kernel(const uint4* __re
                                                                const uint4* __restrict__ g,
                                                                const uint4* __restrict__ bta,
                                                                uint4* __restrict__ y) {
+  pdl_wait();  // the previous kernel in the stream has finished (see fg_launch)
   __shared__ float red[4];
   const int chunks = cols / 8;
   const int64_t row = blockIdx.x;
@@ -89,6 +90,7 @@ __global__ void __launch_bounds__(kLnThreads) layernorm_kernel(const uint4* __re
 __global__ void embed_kernel(const int32_t* __restrict__ ids, int T, int ids_stride, int pos0,
                              const uint4* __restrict__ E, const uint4* __restrict__ P, int chunks,
                              int64_t n, uint4* __restrict__ out) {
+  pdl_wait();  // the previous kernel in the stream has finished (see fg_launch)
   for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
     const int64_t r = i / chunks;
     const int c = int(i - r * chunks);
@@ -109,6 +111,7 @@ __global__ void embed_kernel(const int32_t* __restrict__ ids, int T, int ids_str
 // One CTA per row of fp32 logits; ties resolve to the lowest index.
 __global__ void __launch_bounds__(512) argmax_kernel(const float* __restrict__ logits, int V,
                                                      int32_t* __restrict__ tokens, int64_t tok_stride) {
+  pdl_wait();  // the previous kernel in the stream has finished (see fg_launch)
   __shared__ float sv[16];
   __shared__ int si[16];
   const float* row = logits + int64_t(blockIdx.x) * V;
@@ -161,10 +164,9 @@ int layernorm_impl(const void* x, int64_t rows, int cols, const void* g, const v
   if (rows == 0) return FG_OK;
   if (rows > 0x7fffffff) return fail(FG_ERR_SHAPE, "too many rows");
   ProfScope ps(PROF_OTHER, s, 0.0, double(rows) * cols * 4.0);
-  layernorm_kernel<<<unsigned(rows), kLnThreads, 0, s>>>(
+  FG_LAUNCH("layernorm kernel", layernorm_kernel, dim3(unsigned(rows)), dim3(kLnThreads), size_t(0), s, 
       reinterpret_cast<const uint4*>(x), cols, reinterpret_cast<const uint4*>(g),
       reinterpret_cast<const uint4*>(b), reinterpret_cast<uint4*>(y));
-  FG_CHECK_LAUNCH("layernorm kernel");
   return FG_OK;
 }
 
@@ -179,17 +181,15 @@ int embed_impl(const int32_t* ids, int64_t B, int T, int ids_stride, int pos0, c
   if (n == 0) return FG_OK;
   ProfScope ps(PROF_OTHER, s, 0.0, double(n) * 48.0);
   const int grid = int(std::min<int64_t>((n + 255) / 256, int64_t(num_sms()) * 16));
-  embed_kernel<<<grid, 256, 0, s>>>(ids, T, ids_stride, pos0, reinterpret_cast<const uint4*>(E),
+  FG_LAUNCH("embed kernel", embed_kernel, dim3(grid), dim3(256), size_t(0), s, ids, T, ids_stride, pos0, reinterpret_cast<const uint4*>(E),
                                     reinterpret_cast<const uint4*>(P), chunks, n,
                                     reinterpret_cast<uint4*>(out));
-  FG_CHECK_LAUNCH("embed kernel");
   return FG_OK;
 }
 
 int argmax_impl(const float* logits, int B, int V, int32_t* tokens, int64_t tok_stride, cudaStream_t s) {
   if (B <= 0) return FG_OK;
-  argmax_kernel<<<B, 512, 0, s>>>(logits, V, tokens, tok_stride);
-  FG_CHECK_LAUNCH("argmax kernel");
+  FG_LAUNCH("argmax kernel", argmax_kernel, dim3(B), dim3(512), size_t(0), s, logits, V, tokens, tok_stride);
   return FG_OK;
 }
 

@@ -139,6 +139,7 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const uint4* __
                                                                  int64_t n_chunks,
                                                                  uint2* __restrict__ codes,
                                                                  __half2* __restrict__ params) {
+  pdl_wait();  // the previous kernel in the stream has finished (see fg_launch)
   constexpr int TPG = G / 16;
   const int64_t tile = int64_t(kThreads) * kUnroll;
   for (int64_t base = int64_t(blockIdx.x) * tile; base < n_chunks; base += int64_t(gridDim.x) * tile) {
@@ -171,6 +172,7 @@ __global__ void __launch_bounds__(kThreads) kv_append_kernel(
     const __half* __restrict__ k, const __half* __restrict__ v, int64_t row_stride, int T, int h,
     int hd, int cap, int pos0, int64_t n_chunks, uint2* __restrict__ kc, uint2* __restrict__ vc,
     __half2* __restrict__ kp, __half2* __restrict__ vp) {
+  pdl_wait();  // the previous kernel in the stream has finished (see fg_launch)
   constexpr int TPG = G / 16;
   const __half* src = blockIdx.y == 0 ? k : v;
   uint2* dc = blockIdx.y == 0 ? kc : vc;
@@ -220,6 +222,7 @@ __global__ void __launch_bounds__(kThreads) quantize_cols_kernel(const __half2* 
                                                                  int64_t rows, int64_t cols, int G,
                                                                  uint8_t* __restrict__ codes,
                                                                  __half2* __restrict__ params) {
+  pdl_wait();  // the previous kernel in the stream has finished (see fg_launch)
   const int64_t pairs = cols / 2;
   const int64_t p = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (p >= pairs) return;
@@ -263,6 +266,7 @@ __global__ void __launch_bounds__(kThreads) dequant_rows_kernel(const uint32_t* 
                                                                 const __half2* __restrict__ params,
                                                                 int64_t n_words,
                                                                 uint4* __restrict__ out) {
+  pdl_wait();  // the previous kernel in the stream has finished (see fg_launch)
   constexpr int WPG = G / 8;
   const int64_t tile = int64_t(kThreads) * kUnroll;
   for (int64_t base = int64_t(blockIdx.x) * tile; base < n_words; base += int64_t(gridDim.x) * tile) {
@@ -291,6 +295,7 @@ __global__ void __launch_bounds__(kThreads) dequant_cols_kernel(const uint32_t* 
                                                                 const __half2* __restrict__ params,
                                                                 int64_t rows, int64_t cols, int G,
                                                                 uint4* __restrict__ out) {
+  pdl_wait();  // the previous kernel in the stream has finished (see fg_launch)
   const int64_t words_per_row = cols / 8;
   const int64_t n_words = rows * words_per_row;
   for (int64_t c = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; c < n_words;
@@ -353,17 +358,16 @@ int quantize_pack_impl(const void* x, int64_t rows, int64_t cols, int group, int
     auto* xin = reinterpret_cast<const uint4*>(x);
     auto* cw = reinterpret_cast<uint2*>(codes);
     auto* pw = reinterpret_cast<__half2*>(params);
-    if (group == 32) quantize_rows_kernel<32><<<grid, kThreads, 0, s>>>(xin, chunks, cw, pw);
-    else if (group == 64) quantize_rows_kernel<64><<<grid, kThreads, 0, s>>>(xin, chunks, cw, pw);
-    else quantize_rows_kernel<128><<<grid, kThreads, 0, s>>>(xin, chunks, cw, pw);
+    if (group == 32) FG_LAUNCH("quantize kernel", quantize_rows_kernel<32>, dim3(grid), dim3(kThreads), size_t(0), s, xin, chunks, cw, pw);
+    else if (group == 64) FG_LAUNCH("quantize kernel", quantize_rows_kernel<64>, dim3(grid), dim3(kThreads), size_t(0), s, xin, chunks, cw, pw);
+    else FG_LAUNCH("quantize kernel", quantize_rows_kernel<128>, dim3(grid), dim3(kThreads), size_t(0), s, xin, chunks, cw, pw);
   } else {
     const int64_t pairs = cols / 2;
     dim3 grid(unsigned((pairs + kThreads - 1) / kThreads),
               unsigned(std::min<int64_t>(rows / group, 65535)));
-    quantize_cols_kernel<<<grid, kThreads, 0, s>>>(reinterpret_cast<const __half2*>(x), rows, cols,
+    FG_LAUNCH("quantize kernel", quantize_cols_kernel, dim3(grid), dim3(kThreads), size_t(0), s, reinterpret_cast<const __half2*>(x), rows, cols,
                                                    group, codes, reinterpret_cast<__half2*>(params));
   }
-  FG_CHECK_LAUNCH("quantize kernel");
   return FG_OK;
 }
 
@@ -379,14 +383,13 @@ int dequantize_impl(const uint8_t* codes, const void* params, int64_t rows, int6
   auto* o = reinterpret_cast<uint4*>(out);
   if (axis == 1) {
     const int grid = grid_for(words, int64_t(kThreads) * kUnroll);
-    if (group == 32) dequant_rows_kernel<32><<<grid, kThreads, 0, s>>>(cw, pw, words, o);
-    else if (group == 64) dequant_rows_kernel<64><<<grid, kThreads, 0, s>>>(cw, pw, words, o);
-    else dequant_rows_kernel<128><<<grid, kThreads, 0, s>>>(cw, pw, words, o);
+    if (group == 32) FG_LAUNCH("dequantize kernel", dequant_rows_kernel<32>, dim3(grid), dim3(kThreads), size_t(0), s, cw, pw, words, o);
+    else if (group == 64) FG_LAUNCH("dequantize kernel", dequant_rows_kernel<64>, dim3(grid), dim3(kThreads), size_t(0), s, cw, pw, words, o);
+    else FG_LAUNCH("dequantize kernel", dequant_rows_kernel<128>, dim3(grid), dim3(kThreads), size_t(0), s, cw, pw, words, o);
   } else {
     const int grid = grid_for(words, kThreads);
-    dequant_cols_kernel<<<grid, kThreads, 0, s>>>(cw, pw, rows, cols, group, o);
+    FG_LAUNCH("dequantize kernel", dequant_cols_kernel, dim3(grid), dim3(kThreads), size_t(0), s, cw, pw, rows, cols, group, o);
   }
-  FG_CHECK_LAUNCH("dequantize kernel");
   return FG_OK;
 }
 
@@ -417,12 +420,11 @@ int kv_append_impl(fg_kv_cache* c, const void* k, const void* v, int64_t row_str
   auto* kp = reinterpret_cast<__half2*>(c->k_params);
   auto* vp = reinterpret_cast<__half2*>(c->v_params);
   if (G == 32)
-    kv_append_kernel<32><<<grid, kThreads, 0, s>>>(K, V, row_stride, n_tokens, h, hd, c->capacity, c->len, chunks, kc, vc, kp, vp);
+    FG_LAUNCH("kv append kernel", kv_append_kernel<32>, dim3(grid), dim3(kThreads), size_t(0), s, K, V, row_stride, n_tokens, h, hd, c->capacity, c->len, chunks, kc, vc, kp, vp);
   else if (G == 64)
-    kv_append_kernel<64><<<grid, kThreads, 0, s>>>(K, V, row_stride, n_tokens, h, hd, c->capacity, c->len, chunks, kc, vc, kp, vp);
+    FG_LAUNCH("kv append kernel", kv_append_kernel<64>, dim3(grid), dim3(kThreads), size_t(0), s, K, V, row_stride, n_tokens, h, hd, c->capacity, c->len, chunks, kc, vc, kp, vp);
   else
-    kv_append_kernel<128><<<grid, kThreads, 0, s>>>(K, V, row_stride, n_tokens, h, hd, c->capacity, c->len, chunks, kc, vc, kp, vp);
-  FG_CHECK_LAUNCH("kv append kernel");
+    FG_LAUNCH("kv append kernel", kv_append_kernel<128>, dim3(grid), dim3(kThreads), size_t(0), s, K, V, row_stride, n_tokens, h, hd, c->capacity, c->len, chunks, kc, vc, kp, vp);
   c->len += n_tokens;
   return FG_OK;
 }
