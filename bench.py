@@ -96,7 +96,7 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------- model
-def build_model(fg, torch, dev):
+def build_model(fg, torch, dev, weights="4bit"):
     from fg_synth import gpu as sg
     from fg_synth import layer_stream as ls
     import fg_synth
@@ -111,7 +111,11 @@ def build_model(fg, torch, dev):
                            (fg_synth.S_W2, F, h)):
             w = torch.empty((K, N), dtype=torch.float16, device=dev)
             sg.fill(w, SEED, ls(l, kind), "normal", 0.02)
-            lins.append(fg.DeviceQLinear.from_fp16(w, torch.zeros(N, dtype=torch.float16, device=dev), g))
+            b = torch.zeros(N, dtype=torch.float16, device=dev)
+            if weights == "fp16":   # the uncompressed side of the compression contrast
+                lins.append(fg.DeviceQLinear.uncompressed(w, b))
+            else:
+                lins.append(fg.DeviceQLinear.from_fp16(w, b, g))
             del w
         layers.append(fg.DeviceLayer(ones, zeros, ones, zeros, *lins))
     E = torch.empty((c["vocab"], h), dtype=torch.float16, device=dev)
@@ -399,12 +403,15 @@ def main():
                     default="generate",
                     help="kernel-only cases sized for ncu captures (inputs larger than L2, a few GB at most)")
     ap.add_argument("--mnk", default="", help="M,N,K of the qgemm_decode case")
+    ap.add_argument("--weights", choices=["4bit", "fp16"], default="4bit",
+                    help="fp16: the same generation over uncompressed weights (compression contrast)")
     args = ap.parse_args()
     if args.case != "generate":
         return kernel_case(args)
     world, rank, local = replica_env()
     c = CFG
-    config = {"workload": "OPT-6.7B-shaped decoder, 4-bit weights + 4-bit KV (group 64), batch 64 per GPU, "
+    wdesc = "4-bit weights" if args.weights == "4bit" else "fp16 (uncompressed) weights"
+    config = {"workload": f"OPT-6.7B-shaped decoder, {wdesc} + 4-bit KV (group 64), batch 64 per GPU, "
                           "prompt 512, generate 32", "layers": c["n_layers"], "hidden": c["hidden"],
               "heads": f"{c['n_heads']}x{c['head_dim']}", "ffn": c["ffn"], "vocab": c["vocab"],
               "global_batch": c["batch"] * max(world, args.gpus if world == 1 else world),
@@ -436,7 +443,7 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
-    model, caches = build_model(fg, torch, dev)
+    model, caches = build_model(fg, torch, dev, args.weights)
     B, L, T = c["batch"], c["prompt_len"], c["gen_len"]
     from fg_synth import gpu as sg
     import fg_synth
@@ -479,7 +486,6 @@ def main():
     launches = fg.fg_launch_count() - launches0
     ms_total = max_over_ranks(e0.elapsed_time(e1), dev)
     ms_step = ms_total / args.steps
-    tokens_step = B * T * world
     value = job_throughput(B * T, world, args.steps, ms_total)
     prof = {fg.PROF_NAMES[k]: fg.fg_profile_read(k) for k in range(7)}
     clocks = clk.summary()
@@ -558,8 +564,9 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic", "config": config,
         "prefill_ms": statistics.median(t[0] for t in timings), "decode_ms": statistics.median(t[1] for t in timings),
-        "roofline": {"kernel": "tcgen05 GEMM of the prompt pass (M = 32768; 4-bit weights expanded to fp16 "
-                               "once per layer)", "bound": "tensor",
+        "roofline": {"kernel": "tcgen05 GEMM of the prompt pass (M = 32768; " +
+                               ("4-bit weights expanded to fp16 once per layer)" if args.weights == "4bit"
+                                else "uncompressed fp16 weights)"), "bound": "tensor",
                      "achieved": achieved_tf, "peak": pk["tf_sust"], "unit": "TFLOP/s",
                      "frac": achieved_tf / pk["tf_sust"], "traffic": traffic,
                      "peak_source": f"bf16_tflops_sustained of {pk['src']} peaks (fp16 and bf16 dense rates are equal)"},

@@ -31,7 +31,7 @@ class FGError(RuntimeError):
 
 class QLinear(ctypes.Structure):
     _fields_ = [("codes", c_void_p), ("params", c_void_p), ("bias", c_void_p),
-                ("K", c_int), ("N", c_int), ("group", c_int)]
+                ("K", c_int), ("N", c_int), ("group", c_int), ("w16", c_void_p)]
 
 
 class Layer(ctypes.Structure):
@@ -162,16 +162,22 @@ def fg_dequantize(codes, params, rows: int, cols: int, group: int = 64, axis: in
 class DeviceQLinear:
     """A 4-bit linear layer resident in HBM (keeps the tensors alive for the C struct)."""
 
-    def __init__(self, codes, params, bias, K: int, N: int, group: int = 64):
-        self.codes, self.params, self.bias = codes, params, bias
+    def __init__(self, codes, params, bias, K: int, N: int, group: int = 64, w16=None):
+        self.codes, self.params, self.bias, self.w16 = codes, params, bias, w16
         self.K, self.N, self.group = K, N, group
-        self.c = QLinear(_ptr(codes), _ptr(params), _ptr(bias), K, N, group)
+        self.c = QLinear(_ptr(codes), _ptr(params), _ptr(bias), K, N, group, _ptr(w16))
 
     @staticmethod
     def from_fp16(w, bias, group: int = 64, stream=None) -> "DeviceQLinear":
         K, N = w.shape
         codes, params = fg_quantize_pack(w, group, 1, stream=stream)
         return DeviceQLinear(codes, params, bias, K, N, group)
+
+    @staticmethod
+    def uncompressed(w, bias) -> "DeviceQLinear":
+        """The same layer over the fp16 weight itself (no compression)."""
+        K, N = w.shape
+        return DeviceQLinear(None, None, bias, K, N, 64, w16=w)
 
 
 class DeviceLayer:

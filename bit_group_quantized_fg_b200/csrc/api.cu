@@ -160,7 +160,7 @@ struct Carver {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 int check_qlinear(const fg_qlinear& w, int K, int N, const char* name) {
-  if (!w.codes || !w.params) return fail(FG_ERR_INVALID_ARG, "%s: null weight", name);
+  if (!w.w16 && (!w.codes || !w.params)) return fail(FG_ERR_INVALID_ARG, "%s: null weight", name);
   if (w.K != K || w.N != N) return fail(FG_ERR_SHAPE, "%s: weight is %dx%d, expected %dx%d", name, w.K, w.N, K, N);
   return FG_OK;
 }
@@ -188,6 +188,8 @@ int check_layer(const fg_layer* L, int h, int* ffn) {
 // requested before the previous kernel finishes.
 int qlinear_run(const void* X, int64_t M, const fg_qlinear& w, const void* R, int relu, void* Y, void* ws,
                 size_t wsb, cudaStream_t s, bool w_ready = false) {
+  if (w.w16)  // uncompressed weight: the fp16 GEMM over it directly
+    return gemm_impl(1, X, M, w.N, w.K, w.w16, nullptr, 0, w.bias, R, relu, Y, false, ws, wsb, s, w_ready);
   const size_t wbytes = (size_t(w.K) * size_t(w.N) * 2 + 255) & ~size_t(255);
   if (M >= kExpandRows && ws != nullptr && wsb >= wbytes && aligned16(ws)) {
     FG_TRY(dequantize_impl(w.codes, w.params, w.K, w.N, w.group, 1, ws, s));

@@ -79,12 +79,17 @@ int fg_dequantize(const uint8_t* codes, const void* params, int64_t rows, int64_
 /* A linear layer Y = X W + b whose weight W [K][N] (math convention, N contiguous) is
  * stored 4-bit with groups of `group` along N (the output channel):
  *   codes  uint8 [K][N/2], params half2 [K][N/group], bias fp16 [N] (may be NULL).
- * This is exactly fg_quantize_pack(W, K, N, group, axis=1). */
+ * This is exactly fg_quantize_pack(W, K, N, group, axis=1).
+ * w16: when not NULL the layer uses this uncompressed fp16 weight [K][N] instead (codes
+ * and params are then ignored and may be NULL; N % 256 == 0).  The "FlexGen" README
+ * mirror's benchmark table contrasts FlexGen with and without compression; this is the
+ * uncompressed side, running through the same layer and generation calls. */
 typedef struct {
   const uint8_t* codes;
   const void* params;
   const void* bias;
   int K, N, group;
+  const void* w16;
 } fg_qlinear;
 
 /* One OPT decoder block (pre-LayerNorm, MHA, ReLU FFN).  qkv: [h][3h] with output
@@ -134,9 +139,10 @@ int fg_kv_append(fg_kv_cache* cache, const void* k, const void* v, int64_t row_s
 
 /* Dequant-fused GEMM on the tensor cores: Y[M][N] = [relu](X[M][K] W_hat + b) [+ R].
  * X fp16 [M][K] (row stride K), R fp16 [M][N] or NULL, Y fp16 [M][N].  W_hat is the
- * fg_dequantize of the weight (exact fp16), products accumulate in fp32.
- * K % 64 == 0, N % 128 == 0, group in {32, 64, 128}.  `workspace` may be NULL when
- * fg_qgemm_workspace_bytes(M, N, K) is 0. */
+ * fg_dequantize of the weight (exact fp16; W->w16 itself when set), products accumulate
+ * in fp32.  K % 64 == 0, N % 256 == 0, N % (4 * group) == 0, group in {32, 64, 128}.
+ * `workspace` may be NULL when fg_qgemm_workspace_bytes(M, N, K) is 0; with M >= 1024 and
+ * enough workspace the 4-bit weight is first expanded to fp16 inside it. */
 size_t fg_qgemm_workspace_bytes(int64_t M, int N, int K);
 int fg_qgemm(const void* X, int64_t M, const fg_qlinear* W, const void* R, int relu, void* Y,
              void* workspace, size_t ws_bytes, void* stream);

@@ -26,11 +26,11 @@ from .quant import (quantize_groups, dequantize_groups, pack_nibbles, unpack_nib
                     quantize_pack, dequantize, storage_bytes)
 from .decoder import (layernorm, qlinear, linear_fp16, prefill_attention, decode_attention,
                       kv_append, cache_dequant, cache_values, decode_layer, prefill_layer, generate, embed,
-                      lm_head_argmax, QLinear, QLayer, KVCache, Model)
+                      lm_head_argmax, QLinear, Linear16, QLayer, KVCache, Model)
 
 __all__ = [
     "quantize_groups", "dequantize_groups", "pack_nibbles", "unpack_nibbles",
     "quantize_pack", "dequantize", "storage_bytes", "layernorm", "qlinear", "linear_fp16",
     "prefill_attention", "decode_attention", "kv_append", "cache_dequant", "cache_values", "decode_layer",
-    "prefill_layer", "generate", "embed", "lm_head_argmax", "QLinear", "QLayer", "KVCache", "Model",
+    "prefill_layer", "generate", "embed", "lm_head_argmax", "QLinear", "Linear16", "QLayer", "KVCache", "Model",
 ]

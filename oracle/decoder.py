@@ -88,6 +88,25 @@ class QLinear:
         return exact.astype(np.float16).astype(np.float64)
 
 
+@dataclass
+class Linear16:
+    """An uncompressed linear layer: the fp16 weight [K][N] itself stands where W_hat does
+    ("FlexGen" README mirror, benchmark table: FlexGen without compression)."""
+    w16: np.ndarray             # fp16 [K, N]
+    bias: np.ndarray            # fp16 [N]
+
+    @property
+    def K(self) -> int:
+        return self.w16.shape[0]
+
+    @property
+    def N(self) -> int:
+        return self.w16.shape[1]
+
+    def weight(self) -> np.ndarray:
+        return np.asarray(self.w16, np.float16).astype(np.float64)
+
+
 def qlinear(a16: np.ndarray, lin: QLinear, relu: bool = False,
             residual16: Optional[np.ndarray] = None) -> np.ndarray:
     """fp16( [relu](a @ W_hat + b) [+ residual] ), float64 in between."""

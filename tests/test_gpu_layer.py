@@ -24,8 +24,9 @@ def fg():
     return m
 
 
-def make_layer(seed, l, h, F, g=64, wscale=0.02, ln_random=False):
-    """Oracle and device copies of one decoder layer from seeded fp16 tensors."""
+def make_layer(seed, l, h, F, g=64, wscale=0.02, ln_random=False, uncompressed=False):
+    """Oracle and device copies of one decoder layer from seeded fp16 tensors (with
+    ``uncompressed`` the fp16 weights are used as they are, on both sides)."""
     def t(kind, shape, dist="normal", scale=wscale):
         return fg_synth.tensor(seed, ls(l, kind), shape, dist, scale)
     if ln_random:
@@ -39,14 +40,17 @@ def make_layer(seed, l, h, F, g=64, wscale=0.02, ln_random=False):
     for wk, bk, K, N in ws:
         w = t(wk, (K, N))
         b = t(bk, (N,), scale=0.02)
-        o_lins.append(oracle.QLinear.from_fp16(w, b, g))
+        o_lins.append(oracle.Linear16(w, b) if uncompressed else oracle.QLinear.from_fp16(w, b, g))
         d_lins.append((w, b, K, N))
     ol = oracle.QLayer(*ln, *o_lins)
     return ol, ln, d_lins
 
 
-def to_device_layer(fg, ln, d_lins, g=64):
-    lins = [fg.DeviceQLinear.from_fp16(to_dev(w), to_dev(b), g) for (w, b, K, N) in d_lins]
+def to_device_layer(fg, ln, d_lins, g=64, uncompressed=False):
+    if uncompressed:
+        lins = [fg.DeviceQLinear.uncompressed(to_dev(w), to_dev(b)) for (w, b, K, N) in d_lins]
+    else:
+        lins = [fg.DeviceQLinear.from_fp16(to_dev(w), to_dev(b), g) for (w, b, K, N) in d_lins]
     return fg.DeviceLayer(*[to_dev(x) for x in ln], *lins)
 
 
@@ -105,13 +109,13 @@ def test_config1_layer_prefill_then_decode(fg, ln_random):
     assert dcache.length == L + steps
 
 
-def small_model(fg, seed=5, n_layers=2, h=256, nh=4, F=1024, V=1000, max_pos=64, g=64):
+def small_model(fg, seed=5, n_layers=2, h=256, nh=4, F=1024, V=1000, max_pos=64, g=64, uncompressed=False):
     hd = h // nh
     layers_o, layers_d = [], []
     for l in range(n_layers):
-        ol, ln, d_lins = make_layer(seed, l, h, F, g, wscale=0.05, ln_random=True)
+        ol, ln, d_lins = make_layer(seed, l, h, F, g, wscale=0.05, ln_random=True, uncompressed=uncompressed)
         layers_o.append(ol)
-        layers_d.append(to_device_layer(fg, ln, d_lins, g))
+        layers_d.append(to_device_layer(fg, ln, d_lins, g, uncompressed))
     E = fg_synth.tensor(seed, fg_synth.S_EMBED, (V, h), "normal", 0.5)
     P = fg_synth.tensor(seed, fg_synth.S_POS, (max_pos, h), "normal", 0.1)
     lnf_g = np.ones(h, np.float16)
@@ -210,3 +214,31 @@ def test_profiling_inside_graphs_counts_every_launch(fg):
         for c in per_call:
             assert (c[k]["ms"] > 0) == (c[k]["launches"] > 0)
     assert per_call[2][1]["launches"] == mo.n_layers * (T - 1)   # decode attention per layer and step
+
+
+def test_uncompressed_weights_layer_and_generate(fg):
+    """The fp16-weight side of the compression contrast: the same layer and generation calls
+    over uncompressed weights (the KV cache stays 4-bit) against the oracle with W itself."""
+    import torch
+    h, F, nh, g = 256, 1024, 4, 64
+    ol, ln, d_lins = make_layer(21, 0, h, F, g, wscale=0.05, ln_random=True, uncompressed=True)
+    dl = to_device_layer(fg, ln, d_lins, g, uncompressed=True)
+    B, L = 3, 20
+    pc = fg.DeviceKVCache(B, nh, h // nh, L + 2, g)
+    oc = oracle.KVCache(B, nh, h // nh, g, L + 2)
+    x = fg_synth.tensor(21, 1, (B, L, h), "normal", 1.0)
+    y = fg.fg_prefill_layer(dl, pc, to_dev(x.reshape(B * L, h)), B, L)
+    torch.cuda.synchronize()
+    yo = oracle.prefill_layer(ol, oc, x)
+    assert_close_rms(to_np(y).reshape(B, L, h), yo, what="uncompressed prefill layer")
+    xd = fg_synth.tensor(21, 2, (B, h), "normal", 1.0)
+    yd = fg.fg_decode_layer(dl, pc, to_dev(xd))
+    torch.cuda.synchronize()
+    assert_close_rms(to_np(yd), oracle.decode_layer(ol, oc, xd), what="uncompressed decode layer")
+    mo, md = small_model(fg, seed=6, uncompressed=True)
+    ids = fg_synth.token_ids(6, fg_synth.S_IDS, (4, 16), mo.vocab)
+    caches = [fg.DeviceKVCache(4, mo.n_heads, mo.head_dim, 24, 64) for _ in range(mo.n_layers)]
+    out, _ = fg.fg_generate(md, to_dev(ids), 8, caches)
+    torch.cuda.synchronize()
+    exp, logits = oracle.generate(mo, ids, 8, return_logits=True)
+    assert compare_tokens(to_np(out), exp, logits) >= 0.99

@@ -248,3 +248,19 @@ def test_two_position_attention_is_logistic_of_scaled_score():
     qkv[0, 1, 2 * hd:] = 1.0
     outp = oracle.prefill_attention(qkv, 1, hd).astype(np.float64)
     assert np.all(np.abs(outp[0, 1] - expect) <= 2 ** -11)
+
+
+def test_linear16_is_the_plain_product():
+    """The uncompressed layer uses the fp16 weight itself: an identity weight returns
+    x + b exactly, and a weight on the fp16 grid gives the exact product rounded once."""
+    h = 64
+    x = fg_synth.tensor(3, 1, (5, h), "normal", 1.0)
+    b = fg_synth.tensor(3, 2, (h,), "normal", 0.5)
+    eye = np.eye(h, dtype=np.float16)
+    y = oracle.qlinear(x, oracle.Linear16(eye, b))
+    assert np.array_equal(y, (x.astype(np.float64) + b.astype(np.float64)).astype(np.float16))
+    w = (np.arange(h * 8).reshape(h, 8) % 7 - 3).astype(np.float16)   # small integers
+    xi = (np.arange(5 * h).reshape(5, h) % 5 - 2).astype(np.float16)
+    y2 = oracle.qlinear(xi, oracle.Linear16(w, np.zeros(8, np.float16)), relu=True)
+    ref = np.maximum(xi.astype(np.int64) @ w.astype(np.int64), 0).astype(np.float16)
+    assert np.array_equal(y2, ref)
