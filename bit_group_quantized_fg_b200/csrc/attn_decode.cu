@@ -18,7 +18,7 @@
 namespace fg {
 namespace {
 
-constexpr int kWarps = 4;
+constexpr int kWarps = 2;
 constexpr int kThreads = kWarps * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
