@@ -533,6 +533,30 @@ def main():
     q_gbs = xq.numel() * (2 + 0.5 + 4 / 64) / (q_ms * 1e-3) / 1e9
     del xq, codes, params
 
+    # ---- decode attention GB/s at the last decode step's shape (B 64, 32 x 128, context 543,
+    # 160 MB of 4-bit cache, larger than L2), timed on its own
+    S_att = L + T - 1
+    h = c["hidden"]
+    kvsrc = torch.empty((B * S_att, 2 * h), dtype=torch.float16, device=dev)
+    sg.fill(kvsrc, SEED, 3, "normal", 1.0)
+    qa = torch.empty((B, 3 * h), dtype=torch.float16, device=dev)
+    sg.fill(qa, SEED, 4, "normal", 1.0)
+    acache = fg.DeviceKVCache(B, c["n_heads"], c["head_dim"], S_att, c["group"], dev)
+    fg.fg_kv_append(acache, kvsrc, kvsrc[:, h:], 2 * h, S_att)
+    del kvsrc
+    aout = torch.empty((B, h), dtype=torch.float16, device=dev)
+    for _ in range(3):
+        fg.fg_decode_attention(qa, 3 * h, acache, out=aout)
+    e4.record(stream)
+    for _ in range(reps):
+        fg.fg_decode_attention(qa, 3 * h, acache, out=aout)
+    e5.record(stream)
+    torch.cuda.synchronize()
+    att_ms = e4.elapsed_time(e5) / reps
+    att_bytes = B * c["n_heads"] * S_att * 2.0 * (c["head_dim"] / 2 + 4.0 * c["head_dim"] / c["group"]) + 4.0 * B * h
+    att_gbs = att_bytes / (att_ms * 1e-3) / 1e9
+    del acache, qa, aout
+
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -572,8 +596,9 @@ def main():
                      "peak_source": f"bf16_tflops_sustained of {pk['src']} peaks (fp16 and bf16 dense rates are equal)"},
         "quantizer": {"GB/s": q_gbs, "frac": q_gbs / pk["hbm"], "peak_GB/s": pk["hbm"],
                       "tensor": "1 GiB fp16 (131072 x 4096), group 64"},
-        "decode_attention": {"GB/s": da["bytes"] / (da["ms"] * 1e-3) / 1e9 if da["ms"] else None,
-                             "frac": (da["bytes"] / (da["ms"] * 1e-3) / 1e9) / pk["hbm"] if da["ms"] else None},
+        "decode_attention": {"GB/s": att_gbs, "frac": att_gbs / pk["hbm"], "peak_GB/s": pk["hbm"],
+                             "shape": f"B {B}, {c['n_heads']} x {c['head_dim']}, context {S_att}, group {c['group']}",
+                             "in_step_GB/s": da["bytes"] / (da["ms"] * 1e-3) / 1e9 if da["ms"] else None},
         "kernels": kernels,
         "kernels_note": "one extra replayed step with every kernel class timed (outside the timed region)",
         "clocks": clocks,
