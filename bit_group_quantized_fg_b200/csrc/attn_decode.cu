@@ -34,15 +34,17 @@ __device__ __forceinline__ uint4 ldg_v4(const uint4* p) {
 // The same attention with both contractions on mma.sync (m16n8k16, fp16 in, fp32 out), so
 // that the codes are only unpacked, never multiplied on the FMA pipe.  A warp takes blocks
 // of 16 positions.
-//   scores:  D[t][n] = sum over the dims d of group n of q_d (64 + c_td)   (A = codes,
-//            B = q masked per group): a code becomes the exact fp16 64 + c by putting the
-//            nibble into mantissa bits 4-7 of 64.0 (the smallest offset with an exact
-//            integer step there, which keeps the cancellation below small); K dims are taken
-//            in any order that A and B agree on.
-//            score_t = sum_n s_tn (D[t][n] - 64 Q_n) + mn_tn Q_n, Q_n = sum q_d over the group.
+//   scores:  D[t][n] = sum over the dims d of group n of q_d (o_d + c_td)   (A = codes,
+//            B = q masked per group): a code becomes an exact fp16 o + c by putting the
+//            nibble into the mantissa of 1024.0 (low nibbles, bits 0-3: o = 1024) or of 64.0
+//            (high nibbles, bits 4-7: o = 64); K dims are taken in any order that A and B
+//            agree on.  score_t = sum_n s_tn (D[t][n] - O_n) + mn_tn Q_n, with
+//            O_n = sum q_d o_d and Q_n = sum q_d over the group.
 //   values:  E[d][n] = sum_t w_tn (64 + c_td) with w_tn = fp16(p_t s_tn) (A = codes with
 //            pairs of positions per register, B = w), and
 //            out_d = (sum_t p_t mn_tn + E[d][n] - 64 sum_t w_tn) / sum_t p_t, n = group(d).
+//            Here both nibbles use o = 64 (low nibbles shifted up): the offset sum grows with
+//            the number of positions, and the small offset keeps its cancellation small.
 // Thread (g = lane/4, q4 = lane%4) holds positions g and g + 8 of a block for the scores and
 // dims DPT*g .. DPT*g + DPT-1 for the values (DPT = HD/8).
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -54,13 +56,13 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// The four fp16 pairs (64 + c) of one code word (dims 8w .. 8w+7): P0 = dims (0, 2),
-// P1 = (4, 6) from the low nibbles (moved up into bits 4-7), P2 = (1, 3), P3 = (5, 7) from the
-// high nibbles.
+// The four fp16 pairs (o + c) of one code word (dims 8w .. 8w+7): P0 = dims (0, 2),
+// P1 = (4, 6) from the low nibbles (o = 1024), P2 = (1, 3), P3 = (5, 7) from the high nibbles
+// (o = 64).
 __device__ __forceinline__ void code_pairs(uint32_t w, uint32_t (&P)[4]) {
-  const uint32_t x = (w << 4) & 0xF0F0F0F0u, y = w & 0xF0F0F0F0u;
-  P[0] = __byte_perm(x, 0x54545454u, 0x4140);
-  P[1] = __byte_perm(x, 0x54545454u, 0x4342);
+  const uint32_t x = w & 0x0F0F0F0Fu, y = w & 0xF0F0F0F0u;
+  P[0] = __byte_perm(x, 0x64646464u, 0x4140);
+  P[1] = __byte_perm(x, 0x64646464u, 0x4342);
   P[2] = __byte_perm(y, 0x54545454u, 0x4140);
   P[3] = __byte_perm(y, 0x54545454u, 0x4342);
 }
@@ -119,7 +121,7 @@ __global__ void __launch_bounds__(kThreads) decode_attn_mma_kernel(
     for (int n = 0; n < NG; ++n) {
       if (d / G == n) {
         Qn[n] += qd;
-        On[n] += qd * 64.f;
+        On[n] += qd * ((d & 1) ? 64.f : 1024.f);
       }
     }
   }

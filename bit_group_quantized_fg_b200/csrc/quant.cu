@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const uint4* __
 // Rows r = b*T + t of k (blockIdx.y == 0) or v (== 1); h valid values per row, quantized in
 // chunks of 16 along the hidden dimension.  The group of head `head` lands at cache
 // position pos0 + t.
-template <int G>
+template <int G, int U>
 __global__ void __launch_bounds__(kThreads) kv_append_kernel(
     const __half* __restrict__ k, const __half* __restrict__ v, int64_t row_stride, int T, int h,
     int hd, int cap, int pos0, int64_t n_chunks, uint2* __restrict__ kc, uint2* __restrict__ vc,
@@ -179,11 +179,11 @@ __global__ void __launch_bounds__(kThreads) kv_append_kernel(
   __half2* dp = blockIdx.y == 0 ? kp : vp;
   const int chunks_per_row = h / 16;
   const int nh = h / hd;
-  const int64_t tile = int64_t(kThreads) * kUnroll;
+  const int64_t tile = int64_t(kThreads) * U;
   for (int64_t base = int64_t(blockIdx.x) * tile; base < n_chunks; base += int64_t(gridDim.x) * tile) {
-    uint4 va[kUnroll], vb[kUnroll];
+    uint4 va[U], vb[U];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+    for (int u = 0; u < U; ++u) {
       const int64_t c = base + u * kThreads + threadIdx.x;
       if (c < n_chunks) {
         const int64_t row = c / chunks_per_row;
@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(kThreads) kv_append_kernel(
       }
     }
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+    for (int u = 0; u < U; ++u) {
       const int64_t c = base + u * kThreads + threadIdx.x;
       GroupQ q = quantize_chunk16<TPG>(va[u], vb[u]);
       if (c < n_chunks) {
@@ -412,7 +412,10 @@ int kv_append_impl(fg_kv_cache* c, const void* k, const void* v, int64_t row_str
   if (n_tokens == 0) return FG_OK;
   const int64_t chunks = int64_t(c->B) * n_tokens * (h / 16);
   ProfScope ps(PROF_QUANT, s, 0.0, double(chunks) * 16 * 2 * (2.0 + 0.5 + 4.0 / G));
-  dim3 grid(unsigned(grid_for(chunks, int64_t(kThreads) * kUnroll)), 2);
+  // few chunks (a decode step's tokens): one chunk per thread and more CTAs, so the
+  // latency of the loads is spread over the SMs instead of queueing in a few CTAs
+  const bool small = chunks < int64_t(num_sms()) * kThreads * 2;
+  dim3 grid(unsigned(grid_for(chunks, int64_t(kThreads) * (small ? 1 : kUnroll))), 2);
   auto* K = reinterpret_cast<const __half*>(k);
   auto* V = reinterpret_cast<const __half*>(v);
   auto* kc = reinterpret_cast<uint2*>(c->k_codes);
@@ -420,11 +423,11 @@ int kv_append_impl(fg_kv_cache* c, const void* k, const void* v, int64_t row_str
   auto* kp = reinterpret_cast<__half2*>(c->k_params);
   auto* vp = reinterpret_cast<__half2*>(c->v_params);
   if (G == 32)
-    FG_LAUNCH("kv append kernel", kv_append_kernel<32>, dim3(grid), dim3(kThreads), size_t(0), s, K, V, row_stride, n_tokens, h, hd, c->capacity, c->len, chunks, kc, vc, kp, vp);
+    FG_LAUNCH("kv append kernel", (small ? kv_append_kernel<32, 1> : kv_append_kernel<32, kUnroll>), dim3(grid), dim3(kThreads), size_t(0), s, K, V, row_stride, n_tokens, h, hd, c->capacity, c->len, chunks, kc, vc, kp, vp);
   else if (G == 64)
-    FG_LAUNCH("kv append kernel", kv_append_kernel<64>, dim3(grid), dim3(kThreads), size_t(0), s, K, V, row_stride, n_tokens, h, hd, c->capacity, c->len, chunks, kc, vc, kp, vp);
+    FG_LAUNCH("kv append kernel", (small ? kv_append_kernel<64, 1> : kv_append_kernel<64, kUnroll>), dim3(grid), dim3(kThreads), size_t(0), s, K, V, row_stride, n_tokens, h, hd, c->capacity, c->len, chunks, kc, vc, kp, vp);
   else
-    FG_LAUNCH("kv append kernel", kv_append_kernel<128>, dim3(grid), dim3(kThreads), size_t(0), s, K, V, row_stride, n_tokens, h, hd, c->capacity, c->len, chunks, kc, vc, kp, vp);
+    FG_LAUNCH("kv append kernel", (small ? kv_append_kernel<128, 1> : kv_append_kernel<128, kUnroll>), dim3(grid), dim3(kThreads), size_t(0), s, K, V, row_stride, n_tokens, h, hd, c->capacity, c->len, chunks, kc, vc, kp, vp);
   c->len += n_tokens;
   return FG_OK;
 }
