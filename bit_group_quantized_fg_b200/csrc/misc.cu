@@ -86,6 +86,75 @@ __global__ void __launch_bounds__(kLnThreads) layernorm_kernel(const uint4* __re
   }
 }
 
+// One warp per row for hidden sizes up to 4096 (multiples of 256): the row stays in
+// registers as fp16 (CPL 16-byte chunks per lane, a compile-time count so that every load
+// of the row is issued before the first is used) and both statistics are warp shuffles, so
+// no block barrier sits on the path.  Same fp32 two-pass statistics as above.
+constexpr int kLnWarpMaxChunks = 16;
+constexpr int kLnWarpRows = 8;  // rows (warps) per CTA
+
+template <int CPL>
+__global__ void __launch_bounds__(kLnWarpRows * 32) layernorm_warp_kernel(const uint4* __restrict__ x, int64_t rows,
+                                                                           const uint4* __restrict__ g,
+                                                                           const uint4* __restrict__ bta,
+                                                                           uint4* __restrict__ y) {
+  pdl_wait();  // the previous kernel in the stream has finished (see fg_launch)
+  const int lane = threadIdx.x & 31;
+  const int64_t row = int64_t(blockIdx.x) * kLnWarpRows + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  constexpr int cols = CPL * 256;  // CPL chunks of 8 values per lane
+  const uint4* xr = x + row * (cols / 8);
+  uint4 v[CPL];
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) v[i] = __ldg(xr + i * 32 + lane);  // all loads in flight at once
+  float sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) {
+    const __half2* h = reinterpret_cast<const __half2*>(&v[i]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __half22float2(h[j]);
+      sum += f.x + f.y;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float mean = sum / float(cols);
+  float sq = 0.f;
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) {
+    const __half2* h = reinterpret_cast<const __half2*>(&v[i]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __half22float2(h[j]);
+      const float d0 = f.x - mean, d1 = f.y - mean;
+      sq = fmaf(d0, d0, sq);
+      sq = fmaf(d1, d1, sq);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  const float rstd = 1.0f / sqrtf(sq / float(cols) + 1e-5f);
+#pragma unroll
+  for (int i = 0; i < CPL; ++i) {
+    const int c = i * 32 + lane;
+    const uint4 gr = __ldg(g + c), br = __ldg(bta + c);
+    const __half2* xh = reinterpret_cast<const __half2*>(&v[i]);
+    const __half2* gh = reinterpret_cast<const __half2*>(&gr);
+    const __half2* bh = reinterpret_cast<const __half2*>(&br);
+    uint4 o;
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __half22float2(xh[j]), gg = __half22float2(gh[j]), bb = __half22float2(bh[j]);
+      const float a = fmaf((f.x - mean) * rstd, gg.x, bb.x);
+      const float b = fmaf((f.y - mean) * rstd, gg.y, bb.y);
+      ow[j] = h2_as_u32(__floats2half2_rn(a, b));
+    }
+    y[row * (cols / 8) + c] = o;
+  }
+}
+
 // x[r] = fp16(E[ids[r]] + P[pos0 + r % T]); __hadd2 rounds the exact sum once.
 __global__ void embed_kernel(const int32_t* __restrict__ ids, int T, int ids_stride, int pos0,
                              const uint4* __restrict__ E, const uint4* __restrict__ P, int chunks,
@@ -164,6 +233,18 @@ int layernorm_impl(const void* x, int64_t rows, int cols, const void* g, const v
   if (rows == 0) return FG_OK;
   if (rows > 0x7fffffff) return fail(FG_ERR_SHAPE, "too many rows");
   ProfScope ps(PROF_OTHER, s, 0.0, double(rows) * cols * 4.0);
+  if (cols % 256 == 0 && cols / 256 <= kLnWarpMaxChunks) {
+    using K = void (*)(const uint4*, int64_t, const uint4*, const uint4*, uint4*);
+    static const K table[kLnWarpMaxChunks] = {
+        layernorm_warp_kernel<1>,  layernorm_warp_kernel<2>,  layernorm_warp_kernel<3>,  layernorm_warp_kernel<4>,
+        layernorm_warp_kernel<5>,  layernorm_warp_kernel<6>,  layernorm_warp_kernel<7>,  layernorm_warp_kernel<8>,
+        layernorm_warp_kernel<9>,  layernorm_warp_kernel<10>, layernorm_warp_kernel<11>, layernorm_warp_kernel<12>,
+        layernorm_warp_kernel<13>, layernorm_warp_kernel<14>, layernorm_warp_kernel<15>, layernorm_warp_kernel<16>};
+    FG_LAUNCH("layernorm kernel", table[cols / 256 - 1], dim3(unsigned((rows + kLnWarpRows - 1) / kLnWarpRows)),
+              dim3(kLnWarpRows * 32), size_t(0), s, reinterpret_cast<const uint4*>(x), rows,
+              reinterpret_cast<const uint4*>(g), reinterpret_cast<const uint4*>(b), reinterpret_cast<uint4*>(y));
+    return FG_OK;
+  }
   FG_LAUNCH("layernorm kernel", layernorm_kernel, dim3(unsigned(rows)), dim3(kLnThreads), size_t(0), s, 
       reinterpret_cast<const uint4*>(x), cols, reinterpret_cast<const uint4*>(g),
       reinterpret_cast<const uint4*>(b), reinterpret_cast<uint4*>(y));

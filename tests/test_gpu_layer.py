@@ -62,7 +62,7 @@ def test_layernorm(fg):
     y = fg.fg_layernorm(to_dev(x), to_dev(g), to_dev(b))
     torch.cuda.synchronize()
     assert_close_rms(to_np(y), oracle.layernorm(x, g, b), tol=2e-3, what="layernorm")
-    for h in (768, 7168, 12288):
+    for h in (256, 768, 2048, 7168, 12288):   # one warp per row up to 4096, a CTA per row above
         x = fg_synth.tensor(2, h, (5, h), "t3", 1.0)
         y = fg.fg_layernorm(to_dev(x), to_dev(np.ones(h, np.float16)), to_dev(np.zeros(h, np.float16)))
         torch.cuda.synchronize()
