@@ -94,12 +94,59 @@ def test_decode_attention_sampled_full_size(fg, B, nh, S):
         print(f"B {B} nh {nh} S {S} row {b}: max|err| / RMS = {err / rms:.2e}")
 
 
-@pytest.mark.parametrize("B,L,nh,hd", [(4, 32, 12, 64), (2, 100, 2, 128), (1, 200, 3, 64), (2, 64, 1, 128)])
-def test_prefill_attention_matches_oracle(fg, B, L, nh, hd):
+@pytest.mark.parametrize("B,L,nh,hd,scale", [
+    (4, 32, 12, 64, 1.0), (2, 100, 2, 128, 1.0), (1, 200, 3, 64, 1.0), (2, 64, 1, 128, 1.0),
+    (3, 129, 1, 128, 1.0),   # one query past a tile edge
+    (2, 300, 2, 128, 1.0),   # three query tiles, ragged tail
+    (1, 512, 2, 128, 3.0),   # wide scores: the running maximum is raised from tile to tile
+    (2, 257, 2, 64, 3.0),
+])
+def test_prefill_attention_matches_oracle(fg, B, L, nh, hd, scale):
     import torch
     h = nh * hd
-    qkv = fg_synth.tensor(L, nh, (B, L, 3 * h), "normal", 1.0)
+    qkv = fg_synth.tensor(L, nh, (B, L, 3 * h), "normal", scale)
     out = fg.fg_prefill_attention(to_dev(qkv.reshape(B * L, 3 * h)), B, L, nh, hd)
     torch.cuda.synchronize()
     exp = oracle.prefill_attention(qkv, nh, hd)
-    assert_close_rms(to_np(out).reshape(B, L, h), exp, what="prefill attention")
+    err, rms = assert_close_rms(to_np(out).reshape(B, L, h), exp, what="prefill attention")
+    print(f"B {B} L {L} nh {nh} hd {hd} scale {scale}: max|err| / RMS = {err / rms:.2e}")
+
+
+def test_prefill_attention_spike_in_late_tile(fg):
+    """A key far later than the first tile that matches every query much better than the
+    rest: each row's maximum jumps at that tile and earlier contributions must vanish."""
+    import torch
+    B, L, nh, hd = 1, 400, 1, 128
+    qkv = fg_synth.tensor(5, 5, (B, L, 3 * hd), "normal", 0.5).astype(np.float64)
+    qkv[0, :, :hd] = np.abs(qkv[0, :, :hd]) + 0.5          # queries in the positive orthant
+    qkv[0, 300, hd:2 * hd] = 4.0                            # key 300: score ~ 4 * sum(q) / sqrt(hd)
+    qkv = qkv.astype(np.float16)
+    out = fg.fg_prefill_attention(to_dev(qkv.reshape(L, 3 * hd)), B, L, nh, hd)
+    torch.cuda.synchronize()
+    exp = oracle.prefill_attention(qkv, nh, hd)
+    assert_close_rms(to_np(out).reshape(B, L, hd), exp, what="late spike")
+
+
+def test_prefill_attention_sampled_full_size(fg):
+    """The prompt pass of the OPT-6.7B-shaped workload (B 64, L 512, 32 heads x 128): the
+    projections are drawn on the device, sampled (sequence, head) pairs are recomputed by
+    the oracle from the same seeded values, every output is checked for finiteness."""
+    import torch
+    from fg_synth import gpu as sg
+    B, L, nh, hd = 64, 512, 32, 128
+    h = nh * hd
+    qkv = torch.empty((B * L, 3 * h), dtype=torch.float16, device="cuda")
+    sg.fill(qkv, 91, 4, "normal", 1.0)
+    out = fg.fg_prefill_attention(qkv, B, L, nh, hd)
+    torch.cuda.synchronize()
+    assert bool(torch.isfinite(out.float()).all())
+    cols = np.arange(hd)
+    for b, j in ((0, 0), (37, 11), (63, 31)):
+        rows = np.arange(b * L, (b + 1) * L, dtype=np.int64)[:, None]
+        idx = np.concatenate([rows * 3 * h + j * hd + cols, rows * 3 * h + h + j * hd + cols,
+                              rows * 3 * h + 2 * h + j * hd + cols], axis=1)
+        part = fg_synth.values(91, 4, idx.reshape(-1), "normal", 1.0).reshape(1, L, 3 * hd)
+        exp = oracle.prefill_attention(part, 1, hd)
+        got = to_np(out[b * L:(b + 1) * L, j * hd:(j + 1) * hd]).reshape(1, L, hd)
+        err, rms = assert_close_rms(got, exp, what=f"sequence {b} head {j}")
+        print(f"B {B} L {L} sequence {b} head {j}: max|err| / RMS = {err / rms:.2e}")
