@@ -227,6 +227,8 @@ def kernel_case(args):
     gemm_f16         the QKV slice over an fp16 weight; lm_head: [N][K] weight, fp32 logits
     gemm_prefill     one layer's four prompt-pass GEMMs at M 32768 over fp16 weights
     decode_attention config-2 decode step: B 64, 32 heads x 128, context 543 (160 MB of cache)
+    prefill_attention the prompt pass's causal attention of one layer: B 64, L 512, 32 x 128
+                     (805 MB of projections, 268 MB out)
     quantize         1 GiB fp16 tensor [131072 x 4096], group 64
     Runs `--warmup` untimed and `--steps` timed launches and prints their mean time."""
     import torch
@@ -320,6 +322,14 @@ def kernel_case(args):
         out = torch.empty((B, h), dtype=torch.float16, device=dev)
         run = lambda: fg.fg_decode_attention(q, 3 * h, cache, out=out)
         work = {"bytes": B * nh * S * 2.0 * (hd / 2 + 4.0 * hd / 64) + 4.0 * B * h}
+    elif args.case == "prefill_attention":
+        B, L, nh, hd = 64, 512, 32, 128
+        h = nh * hd
+        qkv = torch.empty((B * L, 3 * h), dtype=torch.float16, device=dev)
+        sg.fill(qkv, SEED, 5, "normal", 1.0)
+        out = torch.empty((B * L, h), dtype=torch.float16, device=dev)
+        run = lambda: fg.fg_prefill_attention(qkv, B, L, nh, hd, out=out)
+        work = {"flops": 4.0 * B * nh * L * (L + 1) / 2.0 * hd}
     else:
         x = torch.empty((131072, 4096), dtype=torch.float16, device=dev)
         sg.fill(x, SEED, 7, "normal", 0.02)
@@ -399,7 +409,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", choices=["generate", "qgemm", "qgemm_decode", "gemm_f16", "gemm_prefill", "lm_head",
-                                       "decode_attention", "quantize"],
+                                       "decode_attention", "prefill_attention", "quantize"],
                     default="generate",
                     help="kernel-only cases sized for ncu captures (inputs larger than L2, a few GB at most)")
     ap.add_argument("--mnk", default="", help="M,N,K of the qgemm_decode case")

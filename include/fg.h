@@ -184,9 +184,9 @@ int fg_decode_attention_noalloc(const void* q, int64_t q_stride, const fg_kv_cac
 /* Causal prefill attention on unquantized fp16 projections: qkv fp16 [B*L][3h]
  * (q | k | v), out fp16 [B*L][h].  "FlexGen" README mirror: prompt processing time is
  * part of the throughput metric.  head_dim 64 or 128 (FG_ERR_UNSUPPORTED otherwise); qkv
- * and out 16-byte aligned (FG_ERR_ALIGN); B*L below 2^31 (FG_ERR_SHAPE).  qkv must be
- * readable for 128 rows past each sequence's start (rows past B*L are not read: the copy
- * engine fills them with zeros).  Every wait inside the kernel is bounded (about 2 s);
+ * and out 16-byte aligned (FG_ERR_ALIGN); B*L below 2^31 (FG_ERR_SHAPE).  Nothing outside
+ * the [B*L][3h] qkv rows is read (tiles that reach past row B*L are filled with zeros by
+ * the copy engine).  Every wait inside the kernel is bounded (about 2 s);
  * one that gives up leaves the output unwritten and records a device-side error that the
  * next fg_generate reports as FG_ERR_CUDA. */
 int fg_prefill_attention(const void* qkv, int B, int L, int n_heads, int head_dim, void* out,
