@@ -14,154 +14,207 @@ namespace fg {
 namespace {
 
 // ---------------------------------------------------------------------------------------
-// On the 5th-generation tensor cores.  One CTA of 4 warps per
-// (128-query tile, head, sequence); thread r of the CTA owns query row q0 + r.
-//   TMA       Q tile [128 x HD] once, key and value tiles [128 x HD] per step, straight
-//             from the interleaved projection rows (128-byte swizzle, 64-column boxes).
-//   S         = Q K^T: HD/16 x tcgen05.mma M128 N128 K16 into TMEM columns [0, 128).
-//   softmax   each thread loads its row of S (fp32), applies the scale and the causal
-//             mask, and writes P = 2^(s - m) as fp16 pairs over the first 64 columns of S
-//             (TMEM lane r, column c = keys 2c, 2c+1: the A layout the MMA reads).
-//   O         += P V: 8 x tcgen05.mma M128 N=HD K16 with A from TMEM, V (MN-major) from
-//             shared memory, accumulating in TMEM columns [128, 128 + HD).
+// On the 5th-generation tensor cores.  One CTA of 5 warps per (128-query tile, head,
+// sequence); thread r of warps 0-3 owns query row q0 + r, warp 4 issues every copy and MMA.
+//   TMA       Q tile [128 x HD] once; key and value tiles [64 x HD], two of each in flight,
+//             straight from the interleaved projection rows (128-byte swizzle, 64-column boxes).
+//   S_j       = Q K_j^T: HD/16 x tcgen05.mma M128 N64 K16 into one of two 64-column TMEM
+//             buffers, so Q K_{j+1}^T can run while the softmax of tile j does.
+//   softmax   each thread loads its row of S_j (fp32), applies the causal mask, and writes
+//             P = 2^(s/sqrt(hd) log2 e - m) as fp16 pairs over the first 32 columns of the
+//             same buffer (TMEM lane r, column c = keys 2c, 2c+1: the A layout the MMA reads).
+//   O         += P_j V_j: 4 x tcgen05.mma M128 N=HD K16 with A from TMEM and V (MN-major)
+//             from shared memory, accumulating in TMEM columns [128, 128 + HD).
 // The running maximum m of a row is only raised when a new score exceeds it by more than
-// 2^8 (then O and the running sum are rescaled by 2^(m_old - m_new)); otherwise P is taken
-// against the stale maximum, at most 256, which fp16 and the fp32 sums hold exactly as
-// well.  The result is the same softmax: numerator and denominator share the maximum.
-// One thread issues all copies and MMAs; the next key tile is copied while the softmax
-// runs, the next value tile while the next Q K^T and softmax run.  Two CTAs fit on an SM
-// (96 KB of shared memory and 256 TMEM columns each), so one CTA's softmax overlaps the
-// other's MMAs.  Every wait is bounded; a wait that gives up raises the device error flag,
-// and the CTA drains its copies and MMAs before it frees TMEM and exits.
-constexpr int kTQ = 128;       // queries per CTA (MMA M)
-constexpr int kTK = 128;       // keys per step (MMA N of Q K^T, K of P V)
-constexpr int kBox = 128 * 128;  // one [128 rows x 64 fp16] swizzled box
+// 2^8 (then O and the running sum are rescaled by 2^(m_old - m_new), after the previous
+// P V has completed); otherwise P is taken against the stale maximum, at most 256, which
+// fp16 and the fp32 sums hold exactly as well.  The result is the same softmax: numerator
+// and denominator share the maximum.  Two CTAs fit on an SM (96 KB of shared memory and
+// 256 TMEM columns each).  Every wait is bounded; a wait that gives up raises the device
+// error flag, and the CTA drains its copies and MMAs before it frees TMEM and exits.
+constexpr int kTQ = 128;         // queries per CTA (MMA M)
+constexpr int kTK = 64;          // keys per tile (MMA N of Q K^T, K of P V)
+constexpr int kBox = 64 * 128;   // one [64 rows x 64 fp16] swizzled box (8 KB)
 
 template <int HD>
 struct TcAttnCfg {
-  static constexpr int NB = HD / 64;                 // 64-column boxes per tile
-  static constexpr int kTileBytes = NB * kBox;
-  static constexpr int kOffQ = 0, kOffK = kTileBytes, kOffV = 2 * kTileBytes;
-  static constexpr int kOffBar = 3 * kTileBytes;
-  static constexpr int kSmem = kOffBar + 64 + 1024;  // barriers + alignment slack
-  static constexpr uint32_t kTmemCols = 256;         // S/P [0, 128), O [128, 128 + HD)
+  static constexpr int NB = HD / 64;                  // 64-column boxes across the head dim
+  static constexpr int kQBytes = NB * 2 * kBox;      // [NB][128 rows][64]
+  static constexpr int kKVBytes = NB * kBox;         // [NB][64 rows][64]
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kQBytes;               // two key buffers
+  static constexpr int kOffV = kQBytes + 2 * kKVBytes;  // two value buffers
+  static constexpr int kOffBar = kQBytes + 4 * kKVBytes;
+  static constexpr int kSmem = kOffBar + 128 + 1024;  // barriers + alignment slack
+  static constexpr uint32_t kTmemCols = 256;          // S/P 2 x 64, O [128, 128 + HD)
+  static constexpr int kThreads = 160;
 };
 
 template <int HD>
-__global__ void __launch_bounds__(128, 2)
+__global__ void __launch_bounds__(160, 2)
     prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm, int L, int nh, __half* __restrict__ out,
                            int* __restrict__ err_flag) {
   using namespace sm100;
   using C = TcAttnCfg<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  uint8_t* sQ = smem + C::kOffQ;
-  uint8_t* sK = smem + C::kOffK;
-  uint8_t* sV = smem + C::kOffV;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* bar_k = bars + 0;   // Q (first step) and key tile landed
-  uint64_t* bar_v = bars + 1;   // value tile landed
-  uint64_t* bar_s = bars + 2;   // S = Q K^T complete
-  uint64_t* bar_o = bars + 3;   // O += P V complete
-  uint64_t* bar_d = bars + 4;   // drain on abort
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 6);
+  uint64_t* kfull = bars + 0;   // [2] key tile (and, first, Q) landed
+  uint64_t* vfull = bars + 2;   // [2] value tile landed
+  uint64_t* sfull = bars + 4;   // [2] S_j = Q K_j^T complete
+  uint64_t* pfull = bars + 6;   // [2] P_j written (one arrival per softmax warp)
+  uint64_t* ofull = bars + 8;   // O += P_j V_j complete (one phase per tile)
+  uint64_t* bar_d = bars + 9;   // drain on abort
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 11);
 
-  const int warp = threadIdx.x >> 5;
-  const int nqt = gridDim.x;
-  const int qt = nqt - 1 - blockIdx.x;  // heavy (late) tiles first
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = gridDim.x - 1 - blockIdx.x;  // heavy (late) tiles first
   const int head = blockIdx.y, b = blockIdx.z;
   const int q0 = qt * kTQ;
   const int h = nh * HD;
-  const int row0 = b * L;  // first projection row of this sequence
-  const int n_kt = qt + 1;  // causal: key tiles 0..qt
+  const int row0 = b * L;            // first projection row of this sequence
+  const int n_kt = 2 * (qt + 1);     // causal: key tiles 0 .. q0 + 127
+  const int kt_diag = 2 * qt;        // tiles from here on need the causal mask
 
   pdl_wait();  // the projections come from the previous kernel in the stream
   if (threadIdx.x == 0) {
     prefetch_tmap(&tm);
-    for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < 10; ++i) mbar_init(&bars[i], (i == 6 || i == 7) ? 4 : 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0) tmem_alloc(tmem_slot, C::kTmemCols);
+  if (warp == 4) tmem_alloc(tmem_slot, C::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + 128;
-  const uint32_t lane_off = uint32_t(warp * 32) << 16;
+  const uint32_t tO = tmem + 128;
 
-  // copies issued / completions waited, per barrier (thread 0 only), for the abort drain
-  int k_issued = 0, v_issued = 0, k_done = 0, v_done = 0, mma_open = 0;
-  if (threadIdx.x == 0) {
-    mbar_expect_tx(bar_k, 2 * C::kTileBytes);
-    for (int bb = 0; bb < C::NB; ++bb) {
-      tma_load_2d(sQ + bb * kBox, &tm, head * HD + 64 * bb, row0 + q0, bar_k);
-      tma_load_2d(sK + bb * kBox, &tm, h + head * HD + 64 * bb, row0, bar_k);
-    }
-    mbar_expect_tx(bar_v, C::kTileBytes);
-    for (int bb = 0; bb < C::NB; ++bb) tma_load_2d(sV + bb * kBox, &tm, 2 * h + head * HD + 64 * bb, row0, bar_v);
-    k_issued = v_issued = 1;
-  }
-
-  constexpr uint32_t idesc_qk = idesc_f16_f32(kTQ, kTK, false);
-  constexpr uint32_t idesc_pv = idesc_f16_f32(kTQ, HD, true);
-  const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-  const float sl2 = 1.4426950408889634f * rsqrtf(float(HD));  // log2(e) / sqrt(hd)
-  const int qi = q0 + threadIdx.x;
-  float m_run = -INFINITY, l_run = 0.f;
-  bool ok = true;
-
-  for (int kt = 0; kt < n_kt; ++kt) {
-    const uint32_t ph = kt & 1;
-    // ---- S = Q K^T
-    if (threadIdx.x == 0 && ok) {
-      ok = mbar_wait(bar_k, ph, abort_flag, err_flag, 0x100);
-      if (ok) {
-        k_done++;
+  if (warp == 4) {
+    // ------------------------------------------------------------ copies and MMAs
+    if (lane == 0) {
+      const uint32_t q_addr = smem_u32(smem + C::kOffQ);
+      const uint32_t k_addr = smem_u32(smem + C::kOffK), v_addr = smem_u32(smem + C::kOffV);
+      constexpr uint32_t idesc_qk = idesc_f16_f32(kTQ, kTK, false);
+      constexpr uint32_t idesc_pv = idesc_f16_f32(kTQ, HD, true);
+      // tiles whose copies were issued / waited for, in tile order (for the abort drain)
+      int k_iss = 0, k_wt = 0, v_iss = 0, v_wt = 0;
+      bool ok = true;
+      auto load_k = [&](int j, int extra_bytes) {  // key tile j into buffer j & 1
+        const int bb = j & 1;
+        mbar_expect_tx(&kfull[bb], C::kKVBytes + extra_bytes);  // the one arrival of this phase
+        for (int x = 0; x < C::NB; ++x)
+          tma_load_2d(smem + C::kOffK + bb * C::kKVBytes + x * kBox, &tm, h + head * HD + 64 * x, row0 + j * kTK,
+                      &kfull[bb]);
+        k_iss++;
+      };
+      auto load_v = [&](int j) {
+        const int bb = j & 1;
+        mbar_expect_tx(&vfull[bb], C::kKVBytes);
+        for (int x = 0; x < C::NB; ++x)
+          tma_load_2d(smem + C::kOffV + bb * C::kKVBytes + x * kBox, &tm, 2 * h + head * HD + 64 * x,
+                      row0 + j * kTK, &vfull[bb]);
+        v_iss++;
+      };
+      auto issue_qk = [&](int j) {  // waits for key tile j, S_j into buffer j & 1
+        const int bb = j & 1;
+        if (!mbar_wait(&kfull[bb], (j >> 1) & 1, abort_flag, err_flag, 0x100)) return false;
+        k_wt++;
         tc_fence_after();
+        const uint32_t kb = k_addr + bb * C::kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-          mma_f16_ss(tS, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
-                     idesc_qk, kk > 0);
+          mma_f16_ss(tmem + 64 * bb, smem_desc_sw128(q_addr + (kk >> 2) * (2 * kBox) + (kk & 3) * 32, 16, 1024),
+                     smem_desc_sw128(kb + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024), idesc_qk, kk > 0);
         }
-        mma_commit(bar_s);
-        mma_open++;
+        mma_commit(&sfull[bb]);
+        return true;
+      };
+      // Q rides on the first key tile's barrier (its bytes counted in that phase's expect_tx)
+      load_k(0, C::kQBytes);
+      for (int x = 0; x < C::NB; ++x)
+        for (int r = 0; r < 2; ++r)
+          tma_load_2d(smem + C::kOffQ + x * 2 * kBox + r * kBox, &tm, head * HD + 64 * x, row0 + q0 + 64 * r,
+                      &kfull[0]);
+      load_v(0);
+      load_k(1, 0);  // n_kt >= 2
+      load_v(1);
+      ok = issue_qk(0) && issue_qk(1);
+      for (int j = 0; j < n_kt && ok; ++j) {
+        const int bb = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        // S_j complete: its key buffer is free for tile j + 2
+        if (!(ok = mbar_wait(&sfull[bb], ph, abort_flag, err_flag, 0x200))) break;
+        if (j + 2 < n_kt) load_k(j + 2, 0);
+        if (!(ok = mbar_wait(&pfull[bb], ph, abort_flag, err_flag, 0x400))) break;
+        if (!(ok = mbar_wait(&vfull[bb], ph, abort_flag, err_flag, 0x800))) break;
+        v_wt++;
+        tc_fence_after();
+        const uint32_t vb = v_addr + bb * C::kKVBytes;
+#pragma unroll
+        for (int kk = 0; kk < kTK / 16; ++kk)
+          mma_f16_ts(tO, tmem + 64 * bb + 8 * kk, smem_desc_sw128(vb + kk * 2048, kBox, 1024), idesc_pv,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(ofull);
+        if (j + 2 < n_kt) {
+          // P_j and the value tile are read once P V completes: then S_j's buffer and the
+          // value buffer take tile j + 2
+          if (!(ok = mbar_wait(ofull, j & 1, abort_flag, err_flag, 0x1000))) break;
+          load_v(j + 2);
+          if (!(ok = issue_qk(j + 2))) break;
+        }
+      }
+      if (!ok) {
+        // drain: copies still in flight, then every MMA issued so far
+        for (; k_wt < k_iss; ++k_wt) mbar_wait_drain(&kfull[k_wt & 1], (k_wt >> 1) & 1);
+        for (; v_wt < v_iss; ++v_wt) mbar_wait_drain(&vfull[v_wt & 1], (v_wt >> 1) & 1);
+        mma_commit(bar_d);
+        mbar_wait_drain(bar_d, 0);
       }
     }
-    if (ok) ok = mbar_wait(bar_s, ph, abort_flag, err_flag, 0x200);
-    ok = __all_sync(0xffffffffu, ok);
-    if (threadIdx.x == 0 && ok) {
-      mma_open--;
-      if (kt + 1 < n_kt) {  // the key tile is free: fetch the next one under the softmax
-        mbar_expect_tx(bar_k, C::kTileBytes);
-        for (int bb = 0; bb < C::NB; ++bb)
-          tma_load_2d(sK + bb * kBox, &tm, h + head * HD + 64 * bb, row0 + (kt + 1) * kTK, bar_k);
-        k_issued++;
-      }
-    }
-    // ---- softmax on this thread's row
-    if (ok) {
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax and epilogue
+    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    const float sl2 = 1.4426950408889634f * rsqrtf(float(HD));  // log2(e) / sqrt(hd)
+    const int qi = q0 + threadIdx.x;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kt; ++j) {
+      const int bb = j & 1;
+      ok = mbar_wait(&sfull[bb], (j >> 1) & 1, abort_flag, err_flag, 0x2000);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld_32x32b_x32(tS + lane_off + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
+      const uint32_t ts = tmem + 64 * bb + lane_off;
+      uint32_t sr[64];
+      tmem_ld_32x32b_x32(ts, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld_32x32b_x32(ts + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_ld_wait();
-      const int k0 = kt * kTK;
-      const bool diag = kt == qt;
       float mx = -INFINITY;
+      if (j >= kt_diag) {
+        const int last = qi - j * kTK;  // keys of this tile with index <= last are visible
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        float v = __uint_as_float(sr[c]) * sl2;
-        if (diag && k0 + c > qi) v = -INFINITY;
-        sr[c] = __float_as_uint(v);
-        mx = fmaxf(mx, v);
+        for (int c = 0; c < 64; ++c) {
+          const float v = c <= last ? __uint_as_float(sr[c]) * sl2 : -INFINITY;
+          sr[c] = __float_as_uint(v);
+          mx = fmaxf(mx, v);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float v = __uint_as_float(sr[c]) * sl2;
+          sr[c] = __float_as_uint(v);
+          mx = fmaxf(mx, v);
+        }
       }
       // raise the running maximum only when it grew by more than 8 (p <= 2^8 otherwise)
       const bool raise = mx > m_run + 8.f;
-      if (__any_sync(0xffffffffu, raise && kt > 0)) {
+      if (__any_sync(0xffffffffu, raise && j > 0)) {
+        // O is rescaled after P_{j-1} V_{j-1} has landed in it
+        ok = mbar_wait(ofull, (j - 1) & 1, abort_flag, err_flag, 0x4000);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
         const float alpha = raise ? exp2f(m_run - mx) : 1.f;
 #pragma unroll
         for (int c = 0; c < HD / 32; ++c) {
@@ -174,91 +227,58 @@ __global__ void __launch_bounds__(128, 2)
         }
       }
       if (raise) {
-        l_run *= (kt > 0) ? exp2f(m_run - mx) : 0.f;
+        l_run *= (j > 0) ? exp2f(m_run - mx) : 0.f;
         m_run = mx;
       }
       float ls = 0.f;
-      uint32_t pr[64];
+      uint32_t pr[32];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
+      for (int c = 0; c < 32; ++c) {
         const float p0 = exp2f(__uint_as_float(sr[2 * c]) - m_run);
         const float p1 = exp2f(__uint_as_float(sr[2 * c + 1]) - m_run);
         ls += p0 + p1;
         pr[c] = h2_as_u32(__floats2half2_rn(p0, p1));
       }
       l_run += ls;
-      tmem_st_32x32b_x32(tS + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&pr[0]));
-      tmem_st_32x32b_x32(tS + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&pr[32]));
+      tmem_st_32x32b_x32(ts, pr);
       tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pfull[bb]);
     }
-    tc_fence_before();
-    __syncthreads();
-    ok = ok && !*abort_flag;
-    // ---- O += P V
-    if (threadIdx.x == 0 && ok) {
+    // epilogue: O / l to fp16
+    if (ok) ok = mbar_wait(ofull, (n_kt - 1) & 1, abort_flag, err_flag, 0x8000);
+    if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
-      ok = mbar_wait(bar_v, ph, abort_flag, err_flag, 0x400);
-      if (ok) {
-        v_done++;
+      const float inv = 1.f / l_run;
+      __half* dst = out + (int64_t(row0) + qi) * h + head * HD;
 #pragma unroll
-        for (int kk = 0; kk < kTK / 16; ++kk)
-          mma_f16_ts(tO, tS + 8 * kk, smem_desc_sw128(v_addr + kk * 2048, kBox, 1024), idesc_pv,
-                     (kt > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar_o);
-        mma_open++;
-        // P and the value tile are read once P V completes: then S may be overwritten
-        ok = mbar_wait(bar_o, ph, abort_flag, err_flag, 0x800);
-        if (ok) {
-          mma_open--;
-          if (kt + 1 < n_kt) {
-            mbar_expect_tx(bar_v, C::kTileBytes);
-            for (int bb = 0; bb < C::NB; ++bb)
-              tma_load_2d(sV + bb * kBox, &tm, 2 * h + head * HD + 64 * bb, row0 + (kt + 1) * kTK, bar_v);
-            v_issued++;
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld_32x32b_x32(tO + lane_off + 32 * c, o);
+        tmem_ld_wait();
+        if (qi < L) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint4 w;
+            w.x = h2_as_u32(__floats2half2_rn(__uint_as_float(o[8 * e + 0]) * inv, __uint_as_float(o[8 * e + 1]) * inv));
+            w.y = h2_as_u32(__floats2half2_rn(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv));
+            w.z = h2_as_u32(__floats2half2_rn(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv));
+            w.w = h2_as_u32(__floats2half2_rn(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv));
+            reinterpret_cast<uint4*>(dst + 32 * c)[e] = w;
           }
         }
       }
     }
   }
-
-  // ---- epilogue: O / l to fp16
-  if (ok) ok = mbar_wait(bar_o, (n_kt - 1) & 1, abort_flag, err_flag, 0x1000);
-  ok = __all_sync(0xffffffffu, ok);
-  if (ok) {
-    tc_fence_after();
-    const float inv = 1.f / l_run;
-    __half* dst = out + (int64_t(row0) + qi) * h + head * HD;
-#pragma unroll
-    for (int c = 0; c < HD / 32; ++c) {
-      uint32_t o[32];
-      tmem_ld_32x32b_x32(tO + lane_off + 32 * c, o);
-      tmem_ld_wait();
-      if (qi < L) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          uint4 w;
-          w.x = h2_as_u32(__floats2half2_rn(__uint_as_float(o[8 * e + 0]) * inv, __uint_as_float(o[8 * e + 1]) * inv));
-          w.y = h2_as_u32(__floats2half2_rn(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv));
-          w.z = h2_as_u32(__floats2half2_rn(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv));
-          w.w = h2_as_u32(__floats2half2_rn(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv));
-          reinterpret_cast<uint4*>(dst + 32 * c)[e] = w;
-        }
-      }
-    }
-  }
-  // ---- abort drain: wait (bounded) for this CTA's copies and MMAs still in flight
-  if (threadIdx.x == 0 && !ok) {
-    for (; k_done < k_issued; ++k_done) mbar_wait_drain(bar_k, k_done & 1);
-    for (; v_done < v_issued; ++v_done) mbar_wait_drain(bar_v, v_done & 1);
-    if (mma_open > 0) {
-      mma_commit(bar_d);
-      mbar_wait_drain(bar_d, 0);
-    }
-  }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, C::kTmemCols);
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
 }
+
 }  // namespace
 
 int make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t inner,
@@ -274,7 +294,7 @@ int prefill_attention_impl(const void* qkv, int B, int L, int nh, int hd, void* 
   ProfScope ps(PROF_PREFILL_ATTN, s, flops, double(B) * L * nh * hd * 2.0 * 4.0);
   const uint64_t h = uint64_t(nh) * hd;
   CUtensorMap tm;
-  FG_TRY(make_map_2d(&tm, qkv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, 3 * h, uint64_t(B) * L, 3 * h * 2, 64, kTQ,
+  FG_TRY(make_map_2d(&tm, qkv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, 3 * h, uint64_t(B) * L, 3 * h * 2, 64, kTK,
                      CU_TENSOR_MAP_SWIZZLE_128B));
   int* err = device_error_ptr();
   if (!err) return fail(FG_ERR_CUDA, "device error flag unavailable");
@@ -286,7 +306,7 @@ int prefill_attention_impl(const void* qkv, int B, int L, int nh, int hd, void* 
                                          TcAttnCfg<128>::kSmem));
       set = true;
     }
-    FG_LAUNCH("prefill attention kernel", prefill_attn_tc_kernel<128>, grid, dim3(128), size_t(TcAttnCfg<128>::kSmem),
+    FG_LAUNCH("prefill attention kernel", prefill_attn_tc_kernel<128>, grid, dim3(TcAttnCfg<128>::kThreads), size_t(TcAttnCfg<128>::kSmem),
               s, tm, L, nh, reinterpret_cast<__half*>(out), err);
   } else {
     static bool set = false;
@@ -295,7 +315,7 @@ int prefill_attention_impl(const void* qkv, int B, int L, int nh, int hd, void* 
                                          TcAttnCfg<64>::kSmem));
       set = true;
     }
-    FG_LAUNCH("prefill attention kernel", prefill_attn_tc_kernel<64>, grid, dim3(128), size_t(TcAttnCfg<64>::kSmem),
+    FG_LAUNCH("prefill attention kernel", prefill_attn_tc_kernel<64>, grid, dim3(TcAttnCfg<64>::kThreads), size_t(TcAttnCfg<64>::kSmem),
               s, tm, L, nh, reinterpret_cast<__half*>(out), err);
   }
   return FG_OK;
