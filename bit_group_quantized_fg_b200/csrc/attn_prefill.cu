@@ -77,14 +77,47 @@ __global__ void __launch_bounds__(160, 2)
   const int n_kt = 2 * (qt + 1);     // causal: key tiles 0 .. q0 + 127
   const int kt_diag = 2 * qt;        // tiles from here on need the causal mask
 
+  const bool issuer = warp == 4 && lane == 0;
+  // tiles whose copies were issued / waited for, in tile order (issuer only; abort drain)
+  int k_iss = 0, k_wt = 0, v_iss = 0, v_wt = 0;
+  auto load_k = [&](int j, int extra_bytes) {  // key tile j into buffer j & 1
+    const int bb = j & 1;
+    mbar_expect_tx(&kfull[bb], C::kKVBytes + extra_bytes);  // the one arrival of this phase
+    for (int x = 0; x < C::NB; ++x)
+      tma_load_2d(smem + C::kOffK + bb * C::kKVBytes + x * kBox, &tm, h + head * HD + 64 * x, row0 + j * kTK,
+                  &kfull[bb]);
+    k_iss++;
+  };
+  auto load_v = [&](int j) {
+    const int bb = j & 1;
+    mbar_expect_tx(&vfull[bb], C::kKVBytes);
+    for (int x = 0; x < C::NB; ++x)
+      tma_load_2d(smem + C::kOffV + bb * C::kKVBytes + x * kBox, &tm, 2 * h + head * HD + 64 * x, row0 + j * kTK,
+                  &vfull[bb]);
+    v_iss++;
+  };
+
   pdl_wait();  // the projections come from the previous kernel in the stream
-  if (threadIdx.x == 0) {
+  if (issuer) {
+    // barriers, then the first copies at once: their latency overlaps the TMEM allocation
     prefetch_tmap(&tm);
     for (int i = 0; i < 10; ++i) mbar_init(&bars[i], (i == 6 || i == 7) ? 4 : 1);
     *abort_flag = 0;
     fence_barrier_init();
+    // Q rides on the first key tile's barrier (its bytes counted in that phase's expect_tx)
+    load_k(0, C::kQBytes);
+    for (int x = 0; x < C::NB; ++x)
+      for (int r = 0; r < 2; ++r)
+        tma_load_2d(smem + C::kOffQ + x * 2 * kBox + r * kBox, &tm, head * HD + 64 * x, row0 + q0 + 64 * r,
+                    &kfull[0]);
+    load_v(0);
+    load_k(1, 0);  // n_kt >= 2
+    load_v(1);
   }
-  if (warp == 4) tmem_alloc(tmem_slot, C::kTmemCols);
+  if (warp == 4) {
+    __syncwarp();  // the warp-wide allocation after lane 0's copies
+    tmem_alloc(tmem_slot, C::kTmemCols);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -98,25 +131,7 @@ __global__ void __launch_bounds__(160, 2)
       const uint32_t k_addr = smem_u32(smem + C::kOffK), v_addr = smem_u32(smem + C::kOffV);
       constexpr uint32_t idesc_qk = idesc_f16_f32(kTQ, kTK, false);
       constexpr uint32_t idesc_pv = idesc_f16_f32(kTQ, HD, true);
-      // tiles whose copies were issued / waited for, in tile order (for the abort drain)
-      int k_iss = 0, k_wt = 0, v_iss = 0, v_wt = 0;
       bool ok = true;
-      auto load_k = [&](int j, int extra_bytes) {  // key tile j into buffer j & 1
-        const int bb = j & 1;
-        mbar_expect_tx(&kfull[bb], C::kKVBytes + extra_bytes);  // the one arrival of this phase
-        for (int x = 0; x < C::NB; ++x)
-          tma_load_2d(smem + C::kOffK + bb * C::kKVBytes + x * kBox, &tm, h + head * HD + 64 * x, row0 + j * kTK,
-                      &kfull[bb]);
-        k_iss++;
-      };
-      auto load_v = [&](int j) {
-        const int bb = j & 1;
-        mbar_expect_tx(&vfull[bb], C::kKVBytes);
-        for (int x = 0; x < C::NB; ++x)
-          tma_load_2d(smem + C::kOffV + bb * C::kKVBytes + x * kBox, &tm, 2 * h + head * HD + 64 * x,
-                      row0 + j * kTK, &vfull[bb]);
-        v_iss++;
-      };
       auto issue_qk = [&](int j) {  // waits for key tile j, S_j into buffer j & 1
         const int bb = j & 1;
         if (!mbar_wait(&kfull[bb], (j >> 1) & 1, abort_flag, err_flag, 0x100)) return false;
@@ -131,15 +146,6 @@ __global__ void __launch_bounds__(160, 2)
         mma_commit(&sfull[bb]);
         return true;
       };
-      // Q rides on the first key tile's barrier (its bytes counted in that phase's expect_tx)
-      load_k(0, C::kQBytes);
-      for (int x = 0; x < C::NB; ++x)
-        for (int r = 0; r < 2; ++r)
-          tma_load_2d(smem + C::kOffQ + x * 2 * kBox + r * kBox, &tm, head * HD + 64 * x, row0 + q0 + 64 * r,
-                      &kfull[0]);
-      load_v(0);
-      load_k(1, 0);  // n_kt >= 2
-      load_v(1);
       ok = issue_qk(0) && issue_qk(1);
       for (int j = 0; j < n_kt && ok; ++j) {
         const int bb = j & 1;
