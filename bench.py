@@ -220,6 +220,146 @@ def cpu_baseline_line(args, steps, warmup):
 
 
 # ---------------------------------------------------------------------------- kernel-only cases
+def time_launches(run, steps, warmup):
+    """(ms per launch from a replayed CUDA graph of `steps` launches, ms per eager launch)."""
+    import torch
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    ms_eager = e0.elapsed_time(e1) / max(steps, 1)
+    # device time per launch: the same launches recorded into a CUDA graph and replayed, so
+    # the host's per-call cost (Python, argument checks) cannot leave the GPU idle in between
+    graph = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream()
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(graph, stream=cs, capture_error_mode="thread_local"):
+        for _ in range(steps):
+            run()
+    graph.replay()
+    torch.cuda.synchronize()
+    e0.record()
+    graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del graph
+    return e0.elapsed_time(e1) / max(steps, 1), ms_eager
+
+
+def sweep_case(args):
+    """The measurement sweep of the quantizer, the dequantizer, decode attention and the
+    4-bit GEMM over sizes, group sizes, value distributions, batches and contexts (one JSON
+    line per point; each point is `--steps` launches replayed from a CUDA graph after
+    `--warmup` eager ones).  Points whose bytes fit in L2 (126 MB) say so: their rate is an
+    L2 rate, not an HBM one."""
+    import torch
+    import bit_group_quantized_fg_b200 as fg
+    from fg_synth import gpu as sg
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    L2 = 126e6
+
+    def emit(kind, point, ms, work):
+        res = {"sweep": kind, **point, "ms_per_launch": round(ms, 5)}
+        if "bytes" in work:
+            res["GB/s"] = round(work["bytes"] / (ms * 1e-3) / 1e9, 1)
+            res["l2_resident"] = work["bytes"] < L2 and not work.get("streamed", False)
+        if "flops" in work:
+            res["TFLOP/s"] = round(work["flops"] / (ms * 1e-3) / 1e12, 1)
+        print(json.dumps(res), flush=True)
+
+    # quantize / dequantize: rows of 4096 (grouped along the row), fp16 in
+    cols = 4096
+    points = [(mb, 64, "normal", 0.02) for mb in (1, 16, 256, 1024, 4096)]
+    points += [(1024, g, "normal", 0.02) for g in (32, 128)]
+    points += [(1024, 64, d, sc) for d, sc in (("uniform", 1.0), ("t3", 1.0), ("outlier", 1.0))]
+    for mb, g, dist, sc in points:
+        rows = mb * (1 << 20) // (2 * cols)
+        x = torch.empty((rows, cols), dtype=torch.float16, device=dev)
+        sg.fill(x, SEED, 30, dist, sc)
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+        params = torch.empty((rows, cols // g, 2), dtype=torch.float16, device=dev)
+        y = torch.empty_like(x)
+        n = x.numel()
+        bytes_ = n * (2 + 0.5 + 4.0 / g)
+        pt = {"MB": mb, "group": g, "dist": dist}
+        ms, _ = time_launches(lambda: fg.fg_quantize_pack(x, g, 1, codes, params), args.steps, args.warmup)
+        emit("quantize", pt, ms, {"bytes": bytes_})
+        ms, _ = time_launches(lambda: fg.fg_dequantize(codes, params, rows, cols, g, 1, y), args.steps, args.warmup)
+        emit("dequantize", pt, ms, {"bytes": bytes_})
+        del x, codes, params, y
+        torch.cuda.empty_cache()
+
+    # decode attention over a 4-bit cache (head dim 128, group 64); the codes and params are
+    # drawn directly (every byte is a valid pair of codes), so no fp16 cache is ever built
+    hd, g = 128, 64
+    att = [(B, S, 32) for B in (1, 8, 64, 144, 256) for S in (128, 512, 2048, 8192)]
+    att += [(256, 543, 56), (144, 543, 96), (256, 8192, 96)]
+    for B, S, nh in att:
+        h = nh * hd
+        cache = fg.DeviceKVCache(B, nh, hd, S, g, dev)
+        for t, st in ((cache.k_codes, 40), (cache.v_codes, 41)):
+            sg.fill(t.view(torch.float16), SEED, st, "uniform", 1.0)
+        for t, st in ((cache.k_params, 42), (cache.v_params, 43)):
+            sg.fill(t, SEED, st, "uniform", 0.1)
+        cache.c.len = S
+        q = torch.empty((B, 3 * h), dtype=torch.float16, device=dev)
+        sg.fill(q, SEED, 44, "normal", 1.0)
+        out = torch.empty((B, h), dtype=torch.float16, device=dev)
+        wsb = fg.lib().fg_decode_attention_workspace_bytes(B, nh, hd, S)
+        ws = torch.empty((max(wsb, 16),), dtype=torch.uint8, device=dev)
+        ms, _ = time_launches(lambda: fg.fg_decode_attention(q, 3 * h, cache, out=out, workspace=ws),
+                              args.steps, args.warmup)
+        emit("decode_attention", {"B": B, "S": S, "heads": nh},
+             ms, {"bytes": B * nh * S * 2.0 * (hd / 2 + 4.0 * hd / g) + 4.0 * B * h})
+        del cache, q, out, ws
+        torch.cuda.empty_cache()
+
+    # 4-bit GEMM (group 64): the OPT-6.7B projections at decode batches and the prompt pass,
+    # and the OPT-30B / OPT-175B decode shapes.  Weight copies used in turn exceed the L2,
+    # so every launch streams its weight from HBM as a decode step does (one weight re-read
+    # launch after launch runs slower at the larger shapes: 0.26 vs 0.14 ms at 256 x 21504
+    # x 7168, where 87 MB of codes only partly stay in the L2)
+    h = 4096
+    shapes = [(M, N, K) for M in (64, 144, 256, 32768)
+              for N, K in ((3 * h, h), (h, h), (4 * h, h), (h, 4 * h))]
+    shapes += [(256, 3 * 7168, 7168), (144, 4 * 12288, 12288)]
+    lins = {}
+    for M, N, K in shapes:
+        if (N, K) not in lins:
+            lins.clear()
+            torch.cuda.empty_cache()
+            copies = max(2, int(-(-256e6 // (N * K * (0.5 + 4 / 64)))))
+            w = torch.empty((K, N), dtype=torch.float16, device=dev)
+            lins[(N, K)] = []
+            for i in range(copies):
+                sg.fill(w, SEED, 50 + i, "normal", 0.02)
+                lins[(N, K)].append(
+                    fg.DeviceQLinear.from_fp16(w, torch.zeros(N, dtype=torch.float16, device=dev), 64))
+            del w
+        ring = lins[(N, K)]
+        x = torch.empty((M, K), dtype=torch.float16, device=dev)
+        sg.fill(x, SEED, 51, "normal", 1.0)
+        y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        wsb = fg.fg_qgemm_workspace_bytes(M, N, K)
+        ws = torch.empty((max(wsb, 16),), dtype=torch.uint8, device=dev)
+        it = [0]
+
+        def run_gemm():
+            fg.fg_qgemm(x, ring[it[0] % len(ring)], Y=y, workspace=ws)
+            it[0] += 1
+        ms, _ = time_launches(run_gemm, args.steps, args.warmup)
+        emit("qgemm", {"M": M, "N": N, "K": K}, ms,
+             {"flops": 2.0 * M * N * K, "bytes": N * K * (0.5 + 4.0 / 64) + 2.0 * M * (K + N),
+              "streamed": True})
+        del x, y, ws
+
+
 def kernel_case(args):
     """One kernel class on its own (for ncu captures and micro-measurements):
     qgemm            prompt-pass QKV slice: M 16384, N 12288, K 4096, group 64 (X 134 MB)
@@ -338,31 +478,7 @@ def kernel_case(args):
         params = torch.empty((131072, 64, 2), dtype=torch.float16, device=dev)
         run = lambda: fg.fg_quantize_pack(x, 64, 1, codes, params)
         work = {"bytes": x.numel() * (2 + 0.5 + 4 / 64)}
-    for _ in range(args.warmup):
-        run()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        run()
-    e1.record()
-    torch.cuda.synchronize()
-    ms_eager = e0.elapsed_time(e1) / max(args.steps, 1)
-    # device time per launch: the same launches recorded into a CUDA graph and replayed, so
-    # the host's per-call cost (Python, argument checks) cannot leave the GPU idle in between
-    graph = torch.cuda.CUDAGraph()
-    cs = torch.cuda.Stream()
-    cs.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.graph(graph, stream=cs, capture_error_mode="thread_local"):
-        for _ in range(args.steps):
-            run()
-    graph.replay()
-    torch.cuda.synchronize()
-    e0.record()
-    graph.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / max(args.steps, 1)
+    ms, ms_eager = time_launches(run, args.steps, args.warmup)
     res = {"case": args.case, "ms_per_launch": ms, "ms_per_launch_eager": ms_eager}
     if "flops" in work:
         res["TFLOP/s"] = work["flops"] / (ms * 1e-3) / 1e12
@@ -410,13 +526,15 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", choices=["generate", "qgemm", "qgemm_decode", "gemm_f16", "gemm_prefill", "lm_head",
-                                       "decode_attention", "prefill_attention", "quantize"],
+                                       "decode_attention", "prefill_attention", "quantize", "sweep"],
                     default="generate",
                     help="kernel-only cases sized for ncu captures (inputs larger than L2, a few GB at most)")
     ap.add_argument("--mnk", default="", help="M,N,K of the qgemm_decode case")
     ap.add_argument("--weights", choices=["4bit", "fp16"], default="4bit",
                     help="fp16: the same generation over uncompressed weights (compression contrast)")
     args = ap.parse_args()
+    if args.case == "sweep":
+        return sweep_case(args)
     if args.case != "generate":
         return kernel_case(args)
     world, rank, local = replica_env()
