@@ -9,7 +9,11 @@
 // Both contractions run on the tensor cores (mma.sync) over codes that are only unpacked
 // into exact fp16 (offset + code) values, with the per-group {min, scale} applied to the
 // fp32 results.  Softmax is fp32 with exp2 (scores scaled by log2(e)/sqrt(hd)); warps and
-// chunks are merged with the usual (max, sum, acc) rescaling.
+// chunks are merged with the usual (max, sum, acc) rescaling.  The small mma.sync tile, not
+// tcgen05, because each (sequence, head) has a single query row: the contractions are
+// matrix-vector products over streamed codes (about 3.6 FLOP per byte), so a 128-row tcgen05
+// tile would hold one useful row; the MMA only takes the multiply-adds off the FMA pipe, and
+// HBM stays the bound.
 #include <algorithm>
 #include <mutex>
 
