@@ -81,3 +81,17 @@ def test_workspace_size_queries(fg):
     assert lib.fg_decode_layer_workspace_bytes(4096, 16384, 32, 64, 544) > 0
     assert lib.fg_prefill_layer_workspace_bytes(768, 3072, 4, 32) > 0
     assert lib.fg_lm_head_workspace_bytes(64, 50272) >= 64 * 50272 * 4
+
+
+def test_prefill_attention_and_layernorm_checks(fg):
+    lib = fg.lib()
+    fake = 0x10000
+    assert lib.fg_prefill_attention(None, 2, 64, 4, 128, fake, None) == -1
+    assert lib.fg_prefill_attention(fake, 0, 64, 4, 128, fake, None) == -2
+    assert lib.fg_prefill_attention(fake, 2, 64, 4, 96, fake, None) == -6          # head_dim 96
+    assert lib.fg_prefill_attention(fake, 1 << 16, 1 << 15, 4, 128, fake, None) == -2  # B*L >= 2^31
+    assert lib.fg_prefill_attention(fake + 8, 2, 64, 4, 128, fake, None) == -3
+    assert lib.fg_layernorm(fake, 4, 100, fake, fake, fake, None) == -2            # cols % 8
+    assert lib.fg_layernorm(fake, 4, 16384, fake, fake, fake, None) == -6          # above 12288
+    assert lib.fg_layernorm(fake + 4, 4, 4096, fake, fake, fake, None) == -3
+    assert lib.fg_layernorm(fake, 0, 4096, fake, fake, fake, None) == 0             # no rows: no launch
