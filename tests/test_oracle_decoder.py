@@ -5,8 +5,8 @@ known without the oracle's own formula: LayerNorm statistics and affine behaviou
 linear layers with weights exactly on the 4-bit grid, attention with one position /
 equal keys / a dominant key / causal independence / permutation invariance, a layer with
 zero weights (output = input + out bias + fc2 bias), the generate loop's position
-schedule with zero layers and a hand-built embedding, argmax ties, and batch-row
-independence.  The readings are those of the OPT decoder block named by the FlexGen
+schedule with zero layers and a hand-built embedding, argmax ties, batch-row
+independence, the tied LM head on one-hot inputs, and the KV cache layout on grid values.  The readings are those of the OPT decoder block named by the FlexGen
 README mirror's benchmark table (OPT-6.7B/30B/175B, input 512, output 32).
 """
 import numpy as np
@@ -264,3 +264,46 @@ def test_linear16_is_the_plain_product():
     y2 = oracle.qlinear(xi, oracle.Linear16(w, np.zeros(8, np.float16)), relu=True)
     ref = np.maximum(xi.astype(np.int64) @ w.astype(np.int64), 0).astype(np.float16)
     assert np.array_equal(y2, ref)
+
+
+# ---------------------------------------------------------------- LM head and cache layout
+def test_tied_lm_head_reads_embedding_rows():
+    """logits = x E^T over an [V][h] embedding: a one-hot x at feature i returns column i
+    of E, one logit per vocabulary row (a transposed operand cannot produce [V] logits from
+    a non-square E, nor these values)."""
+    V, h = 7, 4
+    E = f16(np.arange(V * h).reshape(V, h) * 0.25 - 3.0)
+    for i in range(h):
+        x = np.zeros((1, h), np.float16)
+        x[0, i] = 1.0
+        logits = oracle.linear_fp16(x, E)
+        assert logits.shape == (1, V)
+        assert np.array_equal(logits[0], E[:, i].astype(np.float64))
+    x = f16([[1.0, -2.0, 0.5, 4.0]])
+    assert np.array_equal(oracle.linear_fp16(x, E)[0],
+                          np.array([sum(float(x[0, k]) * float(E[n, k]) for k in range(h)) for n in range(V)]))
+
+
+def test_kv_append_places_heads_and_positions():
+    """Tokens appended at positions pos..pos+T-1 land, head by head, at those positions of
+    their (sequence, head) rows; values on the 4-bit grid (min + code * 2^-3 with codes 0..15
+    in every group) come back exactly; other positions stay empty."""
+    B, nh, hd, g, cap, T, pos = 2, 3, 64, 32, 9, 3, 4
+    h = nh * hd
+    rng = np.random.default_rng(5)
+    codes = np.tile(np.arange(16), h // 16 * B * T).reshape(B, T, h)
+    codes = rng.permuted(codes.reshape(-1, g), axis=1).reshape(B, T, h)   # 0..15 in each group
+    mins = rng.integers(-8, 8, size=(B, T, h // g)).repeat(g, axis=2) * 0.5
+    k = f16(mins + codes * 0.125)
+    v = f16(-mins + codes * 0.25)
+    cache = KVCache(B, nh, hd, g, cap)
+    oracle.kv_append(cache, k, v, pos)
+    for b in range(B):
+        for j in range(nh):
+            kk = oracle.cache_values(cache, "k", b, j, cap)
+            vv = oracle.cache_values(cache, "v", b, j, cap)
+            for t in range(T):
+                assert np.array_equal(kk[pos + t], k[b, t, j * hd:(j + 1) * hd].astype(np.float64))
+                assert np.array_equal(vv[pos + t], v[b, t, j * hd:(j + 1) * hd].astype(np.float64))
+            untouched = [p for p in range(cap) if not pos <= p < pos + T]
+            assert not cache.k_codes[b, j, untouched].any() and not cache.v_params[b, j, untouched].any()
