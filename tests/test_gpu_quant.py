@@ -136,3 +136,25 @@ def test_kv_append_bit_exact(fg, hd, g):
     with pytest.raises(fg.FGError):
         fg.fg_kv_append(cache, dev[:, h:], dev[:, 2 * h:], 3 * h, T + 1)   # 9 + 8 > 16 (rejected before launch)
     assert cache.length == 9
+
+
+@pytest.mark.slow
+def test_pack_beyond_2pow31_elements_sampled(fg):
+    """A tensor of 2^31 + 2^18 fp16 elements (4 GiB + 512 KiB): rows on both sides of
+    element 2^31 against the oracle, codes, params and dequantized values bit for bit."""
+    import torch
+    from fg_synth import gpu as sg
+    rows, cols = 524288 + 64, 4096
+    x = torch.empty((rows, cols), dtype=torch.float16, device="cuda")
+    sg.fill(x, 6, 3, "normal", 0.02)
+    codes, params = fg.fg_quantize_pack(x, 64, 1)
+    d = fg.fg_dequantize(codes, params, rows, cols, 64, 1)
+    torch.cuda.synchronize()
+    for r in [0, 524287, 524288, rows - 1]:
+        xr = fg_synth.values(6, 3, np.arange(r * cols, (r + 1) * cols), "normal", 0.02)[None, :]
+        assert np.array_equal(to_np(x[r:r + 1]).view(np.uint16), xr.view(np.uint16))
+        c_ref, p_ref = oracle.quantize_pack(xr, 64, 1)
+        assert np.array_equal(to_np(codes[r:r + 1]), c_ref)
+        assert np.array_equal(to_np(params[r:r + 1]).view(np.uint16), p_ref.view(np.uint16))
+        d_ref = oracle.dequantize(c_ref, p_ref, 1, cols, 64, 1)
+        assert np.array_equal(to_np(d[r:r + 1]).view(np.uint16), d_ref.view(np.uint16))
