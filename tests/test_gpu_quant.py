@@ -158,3 +158,39 @@ def test_pack_beyond_2pow31_elements_sampled(fg):
         assert np.array_equal(to_np(params[r:r + 1]).view(np.uint16), p_ref.view(np.uint16))
         d_ref = oracle.dequantize(c_ref, p_ref, 1, cols, 64, 1)
         assert np.array_equal(to_np(d[r:r + 1]).view(np.uint16), d_ref.view(np.uint16))
+
+
+def _kv_rows(seed, stream, b, T, h, part):
+    """K (part 1) or V (part 2) rows of sequence b of a [B*T][3h] projection tensor drawn
+    with fg_synth (the CPU twin of the values the GPU generator wrote)."""
+    rows = np.arange(b * T, (b + 1) * T, dtype=np.int64)[:, None]
+    idx = rows * 3 * h + part * h + np.arange(h, dtype=np.int64)[None, :]
+    return fg_synth.values(seed, stream, idx.reshape(-1), "normal", 1.0).reshape(T, h)
+
+
+def test_kv_append_prompt_size_sampled(fg):
+    """A prompt pass's append (16 sequences x 512 tokens x 32 heads of 128, 2.1 M chunks, the
+    path the full-size prompt takes) at cache offset 3: sampled sequences bit-exact against
+    the oracle, untouched positions still empty."""
+    import torch
+    from fg_synth import gpu as sg
+    B, T, nh, hd, g, off = 16, 512, 32, 128, 64, 3
+    h = nh * hd
+    qkv = torch.empty((B * T, 3 * h), dtype=torch.float16, device="cuda")
+    sg.fill(qkv, 44, 9, "normal", 1.0)
+    cache = fg.DeviceKVCache(B, nh, hd, T + 8, g)
+    cache.length = off
+    fg.fg_kv_append(cache, qkv[:, h:], qkv[:, 2 * h:], 3 * h, T)
+    torch.cuda.synchronize()
+    assert cache.length == off + T
+    for b in (0, 7, B - 1):
+        k = _kv_rows(44, 9, b, T, h, 1)
+        v = _kv_rows(44, 9, b, T, h, 2)
+        ref = oracle.KVCache(1, nh, hd, g, T + 8)
+        oracle.kv_append(ref, k[None], v[None], off)
+        sl = slice(off, off + T)
+        assert np.array_equal(to_np(cache.k_codes[b, :, sl]), ref.k_codes[0, :, sl])
+        assert np.array_equal(to_np(cache.v_codes[b, :, sl]), ref.v_codes[0, :, sl])
+        assert np.array_equal(to_np(cache.k_params[b, :, sl]).view(np.uint16), ref.k_params[0, :, sl].view(np.uint16))
+        assert np.array_equal(to_np(cache.v_params[b, :, sl]).view(np.uint16), ref.v_params[0, :, sl].view(np.uint16))
+        assert not to_np(cache.k_codes[b, :, :off]).any() and not to_np(cache.v_codes[b, :, off + T:]).any()
