@@ -1,17 +1,26 @@
 """Throughput benchmark: greedy generation over 4-bit weights and a 4-bit KV cache.
 
-Workload (one "step"): an OPT-6.7B-shaped decoder (32 layers, hidden 4096, 32 heads x 128,
-FFN 16384, vocab 50272, learned positions), random fp16 init ~ N(0, 0.02) compressed to
-4 bits in groups of 64 along each weight's output channel, batch 64, prompt 512 token ids
-uniform over the vocabulary, 32 generated tokens (1 from the prompt pass + 31 decode steps)
-- the metric of the FlexGen README mirror's benchmark table: generated tokens / (prompt
-time + generation time).  Synthetic, seeded data (no checkpoints or datasets).
+Workloads (one "step" = one whole generation; synthetic, seeded data, random-init weights
+~ N(0, 0.02) compressed to 4 bits in groups of 64 along each weight's output channel; the
+metric of the FlexGen README mirror's benchmark table: generated tokens / (prompt time +
+generation time), input length 512, output length 32):
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  c3 (default)  OPT-30B-shaped decoder: 48 layers, hidden 7168, 56 heads x 128, FFN 28672,
+                vocab 50272, batch 256, prompt 512 uniform token ids, 32 generated tokens
+                (1 from the prompt pass + 31 decode steps); all state resident in HBM.
+  c2            OPT-6.7B-shaped decoder: 32 layers, hidden 4096, 32 x 128, FFN 16384,
+                batch 64, otherwise as c3.
+  c4            OPT-175B-shaped 12-layer slice: hidden 12288, 96 x 128, FFN 49152, batch
+                144 (the arXiv 2303.06865 abstract's effective batch), prompt 512 hidden
+                states ~ N(0, 1), 32 decode steps with N(0, 1) inputs; no embedding or LM
+                head.  Timed through the layer calls; tokens/s of the slice are reported
+                per layer and extrapolated to 96 layers (x 12/96).
+
+    python bench.py [--config c2|c3|c4] [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 N > 1 runs N independent replicas (one process per GPU, launched by torchrun): the batch
-dimension shards with no exchange step, so each rank generates its own batch of 64
-(weak scaling) and the value is all ranks' tokens divided by the slowest rank's time.
+dimension shards with no exchange step, so each rank generates its own batch (weak
+scaling) and the value is all ranks' tokens divided by the slowest rank's time.
 `--impl reference` times the CPU oracle on a bounded sample of the same workload.
 Prints one JSON line (rank 0).
 """
@@ -30,9 +39,46 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "generated tokens/s at 1 B200 (prefill+decode) vs roofline; quantizer GB/s"
-CFG = dict(model="OPT-6.7B-shaped 32-layer decoder", n_layers=32, hidden=4096, n_heads=32, head_dim=128,
-           ffn=16384, vocab=50272, max_pos=2048, group=64, batch=64, prompt_len=512, gen_len=32)
+CONFIGS = {
+    "c2": dict(kind="generate", model="OPT-6.7B-shaped 32-layer decoder", n_layers=32, hidden=4096, n_heads=32,
+               head_dim=128, ffn=16384, vocab=50272, max_pos=2048, group=64, batch=64, prompt_len=512,
+               gen_len=32),
+    "c3": dict(kind="generate", model="OPT-30B-shaped 48-layer decoder", n_layers=48, hidden=7168, n_heads=56,
+               head_dim=128, ffn=28672, vocab=50272, max_pos=2048, group=64, batch=256, prompt_len=512,
+               gen_len=32),
+    "c4": dict(kind="slice", model="OPT-175B-shaped 12-layer slice", n_layers=12, full_layers=96, hidden=12288,
+               n_heads=96, head_dim=128, ffn=49152, vocab=0, max_pos=0, group=64, batch=144, prompt_len=512,
+               gen_len=32),
+}
+DEFAULT_CONFIG = "c3"
+CFG = CONFIGS[DEFAULT_CONFIG]
 SEED = 1234
+
+
+def use_config(name):
+    """Select the workload the module-level helpers use."""
+    global CFG
+    CFG = CONFIGS[name]
+    return CFG
+
+
+def tokens_per_step(c):
+    """Generated tokens of one step: B x gen_len (for the slice: one per sequence and decode step)."""
+    return c["batch"] * c["gen_len"]
+
+
+def weight_bytes_4bit(c):
+    h, F = c["hidden"], c["ffn"]
+    return c["n_layers"] * (h * 3 * h + h * h + 2 * h * F) * (0.5 + 4.0 / c["group"])
+
+
+def describe(c, wdesc):
+    if c["kind"] == "slice":
+        return (f"{c['model']} ({c['n_layers']} of {c['full_layers']} layers), {wdesc} + 4-bit KV (group "
+                f"{c['group']}), batch {c['batch']} per GPU, prompt {c['prompt_len']}, {c['gen_len']} decode steps; "
+                f"value extrapolated to {c['full_layers']} layers (no embedding / LM head)")
+    return (f"{c['model']}, {wdesc} + 4-bit KV (group {c['group']}), batch {c['batch']} per GPU, "
+            f"prompt {c['prompt_len']}, generate {c['gen_len']}")
 
 
 def peaks():
@@ -118,14 +164,16 @@ def build_model(fg, torch, dev, weights="4bit"):
                 lins.append(fg.DeviceQLinear.from_fp16(w, b, g))
             del w
         layers.append(fg.DeviceLayer(ones, zeros, ones, zeros, *lins))
+    caches = [fg.DeviceKVCache(c["batch"], c["n_heads"], c["head_dim"], c["prompt_len"] + c["gen_len"], g, dev)
+              for _ in range(c["n_layers"])]
+    if c["kind"] == "slice":   # a stack of layers, no embedding or LM head
+        return layers, caches
     E = torch.empty((c["vocab"], h), dtype=torch.float16, device=dev)
     sg.fill(E, SEED, fg_synth.S_EMBED, "normal", 0.02)
     P = torch.empty((c["max_pos"], h), dtype=torch.float16, device=dev)
     sg.fill(P, SEED, fg_synth.S_POS, "normal", 0.02)
     model = fg.DeviceModel(c["n_layers"], h, c["n_heads"], c["head_dim"], F, c["vocab"], c["max_pos"], g, E, P,
                            ones, zeros, layers)
-    caches = [fg.DeviceKVCache(c["batch"], c["n_heads"], c["head_dim"], c["prompt_len"] + c["gen_len"], g, dev)
-              for _ in range(c["n_layers"])]
     return model, caches
 
 
@@ -146,77 +194,114 @@ def synth_host(stream, shape, dist="normal", scale=1.0):
     return fg_synth.tensor(SEED, stream, shape, dist, scale)
 
 
+def params_per_layer(c):
+    h, F = c["hidden"], c["ffn"]
+    return h * 3 * h + h * h + 2 * h * F
+
+
 def oracle_sample():
-    """Time the CPU oracle on a bounded sample: one sequence through one decoder layer's
-    prompt pass (512 tokens), one decode step at context 528 (the mid-point of the 31
-    decode steps) and one LM-head token, at the OPT-6.7B shapes; returns the seconds of
-    each part (weights are generated and quantized before the clock starts)."""
+    """The C++ CPU oracle on a bounded sample of the workload: one sequence through one
+    decoder layer's prompt pass over its first `n_prompt` tokens, one decode step of that
+    layer at context L + T/2 (the middle of the decode steps) and, for a full decoder, one
+    LM-head token.  Weights are generated and quantized by the oracle before the clock
+    starts.  Returns run(n_prompt) -> seconds of (prompt sample, decode step, LM head)."""
     import numpy as np
     import fg_synth
     import oracle
     from fg_synth import layer_stream as ls
     c = CFG
-    h, F, g, L = c["hidden"], c["ffn"], c["group"], c["prompt_len"]
+    h, F, g, L, T = c["hidden"], c["ffn"], c["group"], c["prompt_len"], c["gen_len"]
     nh, hd = c["n_heads"], c["head_dim"]
     lins = []
     for kind, K, N in ((fg_synth.S_WQKV, h, 3 * h), (fg_synth.S_WO, h, h), (fg_synth.S_W1, h, F),
                        (fg_synth.S_W2, F, h)):
         w = synth_host(ls(0, kind), (K, N), "normal", 0.02)
         lin = oracle.QLinear.from_fp16(w, np.zeros(N, np.float16), g)
-        lin.weight()
+        lin.weight16()
         lins.append(lin)
+        del w
     ones, zeros = np.ones(h, np.float16), np.zeros(h, np.float16)
     layer = oracle.QLayer(ones, zeros, ones, zeros, *lins)
-    E = synth_host(fg_synth.S_EMBED, (c["vocab"], h), "normal", 0.02)
-    P = synth_host(fg_synth.S_POS, (c["max_pos"], h), "normal", 0.02)
-    model = oracle.Model(1, h, nh, hd, F, c["vocab"], c["max_pos"], g, E, P, ones, zeros, [layer])
-    ids = fg_synth.token_ids(SEED, fg_synth.S_IDS, (1, L), c["vocab"])
+    model = None
+    if c["kind"] == "generate":
+        E = synth_host(fg_synth.S_EMBED, (c["vocab"], h), "normal", 0.02)
+        P = synth_host(fg_synth.S_POS, (c["max_pos"], h), "normal", 0.02)
+        model = oracle.Model(1, h, nh, hd, F, c["vocab"], c["max_pos"], g, E, P, ones, zeros, [layer])
+    x_prompt = fg_synth.tensor(SEED, fg_synth.S_HIDDEN, (1, L, h), "normal", 1.0)
+    x_dec = fg_synth.tensor(SEED, fg_synth.S_DECODE_X, (1, h), "normal", 1.0)
+    ctx = L + T // 2
 
-    def run():
-        cache = oracle.KVCache(1, nh, hd, g, L + c["gen_len"])
+    def run(n_prompt):
+        cache = oracle.KVCache(1, nh, hd, g, max(ctx, n_prompt) + 1)
         t0 = time.perf_counter()
-        x = oracle.prefill_layer(layer, cache, oracle.embed(model, ids, 0))
+        oracle.prefill_layer(layer, cache, x_prompt[:, :n_prompt])
         t1 = time.perf_counter()
-        cache.length = 528 - 1 if L + c["gen_len"] > 528 else cache.length
-        xd = oracle.decode_layer(layer, cache, x[:, -1, :])
+        cache.length = ctx - 1           # attend over ctx positions (the cache holds valid codes)
+        xd = oracle.decode_layer(layer, cache, x_dec)
         t2 = time.perf_counter()
-        oracle.lm_head_argmax(model, xd)
+        if model is not None:
+            oracle.lm_head_argmax(model, xd)
         t3 = time.perf_counter()
         return t1 - t0, t2 - t1, t3 - t2
     return run
 
 
 def oracle_rate(t_pf, t_dec, t_lm):
-    """Extrapolated tokens/s of the whole workload from one sample (sequences independent:
-    B sequences x n_layers x (prompt + T-1 decode steps) + T LM-head tokens per sequence)."""
+    """Extrapolated tokens/s of the whole workload from one sample (sequences independent,
+    so B sequences take B times one sequence's time for B times its tokens): a full decoder
+    runs n_layers x (prompt pass + T-1 decode steps) + T LM-head tokens per sequence; the
+    slice runs full_layers x (prompt pass + T decode steps), its value extrapolated to the
+    full depth like the GPU's."""
     c = CFG
-    per_seq = c["n_layers"] * (t_pf + (c["gen_len"] - 1) * t_dec) + c["gen_len"] * t_lm
-    return c["batch"] * c["gen_len"] / (c["batch"] * per_seq)
+    if c["kind"] == "slice":
+        per_seq = c["full_layers"] * (t_pf + c["gen_len"] * t_dec)
+    else:
+        per_seq = c["n_layers"] * (t_pf + (c["gen_len"] - 1) * t_dec) + c["gen_len"] * t_lm
+    return c["gen_len"] / per_seq
 
 
-def blas_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
-    except Exception:
-        return os.cpu_count() or 1
-
-
-def cpu_baseline_line(args, steps, warmup):
-    run = oracle_sample()
+def oracle_measure(run, n_prompt, steps, warmup):
+    """Median seconds of the sample parts; the prompt-pass sample scaled to the full prompt
+    (linear in tokens: the projections and FFN, ~99 % of a prompt pass's arithmetic at
+    L = 512, are per token; attention's share is undercounted by this scaling)."""
     for _ in range(warmup):
-        run()
-    ts = [run() for _ in range(steps)]
-    t_pf = statistics.median(t[0] for t in ts)
-    t_dec = statistics.median(t[1] for t in ts)
-    t_lm = statistics.median(t[2] for t in ts)
+        run(n_prompt)
+    ts = [run(n_prompt) for _ in range(steps)]
+    scale = CFG["prompt_len"] / n_prompt
+    return (statistics.median(t[0] for t in ts) * scale, statistics.median(t[1] for t in ts),
+            statistics.median(t[2] for t in ts), ts)
+
+
+def cpu_baseline_line(args, steps, warmup, single_thread=True):
+    """cpu_baseline of the bench line: the C++ oracle with OpenMP over rows on every host core
+    (the value), and single-threaded (reported beside it)."""
+    import oracle
+    c = CFG
+    P = params_per_layer(c)
+    n_omp = max(4, min(64, int(40e9 / P)))     # ~40 GMAC of prompt-pass sample with all cores
+    n_one = max(2, min(64, int(5e9 / P)))      # ~5 GMAC single-threaded
+    run = oracle_sample()
+    cores = oracle.threads(os.cpu_count() or 1)
+    t_pf, t_dec, t_lm, ts = oracle_measure(run, n_omp, steps, warmup)
     rate = oracle_rate(t_pf, t_dec, t_lm)
-    sample = (f"oracle on 1 sequence x 1 layer: prompt pass 512 tokens ({t_pf:.2f} s), one decode step at "
-              f"context 528 ({t_dec:.2f} s), one LM-head token ({t_lm:.2f} s); extrapolated to 64 sequences x "
-              f"32 layers x (prompt + 31 decode steps) + 32 LM-head tokens")
-    return {"value": rate, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle", "sample": sample,
-            "sample_seconds": sum(ts[-1])}
+    seconds = sum(sum(t) for t in ts)
+    lm = f", one LM-head token ({t_lm:.2f} s)" if c["kind"] == "generate" else ""
+    sample = (f"C++ oracle (OpenMP over rows, {cores} threads) on 1 sequence x 1 layer: prompt pass over "
+              f"{n_omp} of {c['prompt_len']} tokens scaled to {c['prompt_len']} ({t_pf:.2f} s), one decode step "
+              f"at context {c['prompt_len'] + c['gen_len'] // 2} ({t_dec:.2f} s){lm}; extrapolated to "
+              f"{c['batch']} sequences x {c.get('full_layers', c['n_layers'])} layers")
+    out = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample,
+           "sample_seconds": seconds}
+    if single_thread:
+        oracle.threads(1)
+        s_pf, s_dec, s_lm, ts1 = oracle_measure(run, n_one, 1, 0)
+        out["single_thread"] = {"value": oracle_rate(s_pf, s_dec, s_lm), "cores": 1,
+                                "sample": f"prompt pass over {n_one} tokens scaled to {c['prompt_len']} "
+                                          f"({s_pf:.2f} s), decode step ({s_dec:.2f} s)"
+                                          + (f", LM head ({s_lm:.2f} s)" if c["kind"] == "generate" else "")}
+        out["sample_seconds"] += sum(sum(t) for t in ts1)
+        oracle.threads(cores)
+    return out
 
 
 # ---------------------------------------------------------------------------- kernel-only cases
@@ -518,12 +603,172 @@ def job_throughput(tokens_per_rank_step, world, steps, ms_max):
 
 
 # ---------------------------------------------------------------------------- main
+def run_generate(args, fg, torch, dev, stream, world, rank, barrier):
+    """The timed generations of a full decoder (c2, c3) through fg_generate."""
+    from fg_synth import gpu as sg
+    import fg_synth
+    c = CFG
+    model, caches = build_model(fg, torch, dev, args.weights)
+    B, L, T = c["batch"], c["prompt_len"], c["gen_len"]
+    ids = torch.empty((B, L), dtype=torch.int32, device=dev)
+    sg.fill_ids(ids, replica_seed(rank), fg_synth.S_IDS, c["vocab"])
+    out = torch.empty((B, T), dtype=torch.int32, device=dev)
+    ws = torch.empty((fg.fg_workspace_bytes(model, B, L, T),), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+
+    # The roofline kernel (the prompt-pass GEMM) is timed by CUDA events from the warm-up on:
+    # the library records them as nodes of its CUDA graphs (first call eager, second
+    # captured, later ones replayed), so the timed steps replay graphs that carry them.
+    # Only that kernel class is timed here; the per-kernel breakdown comes from one more,
+    # separately profiled step after the timed regions.
+    fg.fg_profile_select([0])
+    fg.fg_profile_enable(True)
+    for _ in range(args.warmup):
+        fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
+    # ---- timed region: device-resident inputs
+    fg.fg_profile_reset()
+    launches0 = fg.fg_launch_count()
+    timings = []
+    barrier()
+    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else 0) as clk:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            _, tm = fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
+            timings.append((tm.prefill_ms, tm.decode_ms))
+        e1.record(stream)
+        barrier()
+    launches = fg.fg_launch_count() - launches0
+    ms_total = max_over_ranks(e0.elapsed_time(e1), dev)
+    prof = fg.fg_profile_read(0)
+    clocks = clk.summary()
+
+    # ---- e2e: host buffers through the public API, copies inside the timed region (the
+    # prompt ids go host -> the same device buffer, so the recorded graphs stay valid)
+    ids_host = ids.cpu().pin_memory()
+    out_host = torch.empty((B, T), dtype=torch.int32).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+    barrier()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(e2e_steps):
+        ids.copy_(ids_host, non_blocking=True)
+        fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
+        out_host.copy_(out, non_blocking=True)
+    e3.record(stream)
+    barrier()
+    ms_e2e = max_over_ranks(e2.elapsed_time(e3), dev)
+
+    # ---- per-kernel breakdown: every kernel class timed, one replayed step (not timed above)
+    fg.fg_profile_select(None)
+    for _ in range(2):   # eager, then captured with the new timing nodes
+        fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
+    fg.fg_profile_reset()
+    fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
+    breakdown = {fg.PROF_NAMES[k]: fg.fg_profile_read(k) for k in range(7)}
+    fg.fg_profile_enable(False)
+    del model, caches, ws
+    torch.cuda.empty_cache()
+    return dict(ms_total=ms_total, ms_e2e=ms_e2e, e2e_steps=e2e_steps, timings=timings, prof=prof,
+                breakdown=breakdown, clocks=clocks, launches=launches,
+                h2d=B * L * 4, d2h=B * T * 4)
+
+
+def run_slice(args, fg, torch, dev, stream, world, rank, barrier):
+    """The timed steps of a layer slice (c4) through fg_prefill_layer / fg_decode_layer: the
+    prompt pass over B x L hidden states, then gen_len decode steps of one new token per
+    sequence, every layer in turn.  Launched eagerly (the host issues ~120 launches per
+    decode step, far ahead of the GPU's ~10 ms of work per step)."""
+    from fg_synth import gpu as sg
+    import fg_synth
+    c = CFG
+    layers, caches = build_model(fg, torch, dev, args.weights)
+    B, L, T, h, F = c["batch"], c["prompt_len"], c["gen_len"], c["hidden"], c["ffn"]
+    x0 = torch.empty((B * L, h), dtype=torch.float16, device=dev)
+    sg.fill(x0, replica_seed(rank), fg_synth.S_HIDDEN, "normal", 1.0)
+    xdec = torch.empty((T, B, h), dtype=torch.float16, device=dev)
+    sg.fill(xdec, replica_seed(rank), fg_synth.S_DECODE_X, "normal", 1.0)
+    x = torch.empty_like(x0)
+    xa = torch.empty((B, h), dtype=torch.float16, device=dev)
+    wsb = max(fg.lib().fg_prefill_layer_workspace_bytes(h, F, B, L),
+              fg.lib().fg_decode_layer_workspace_bytes(h, F, c["n_heads"], B, L + T))
+    ws = torch.empty((wsb,), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+
+    def step(prompt, dec_inputs, marks=None):
+        x.copy_(prompt, non_blocking=True)
+        for cache in caches:
+            cache.length = 0
+        for layer, cache in zip(layers, caches):
+            fg.fg_prefill_layer(layer, cache, x, B, L, workspace=ws)
+        if marks is not None:
+            marks.record(stream)
+        for j in range(T):
+            cur = dec_inputs[j]
+            for layer, cache in zip(layers, caches):
+                fg.fg_decode_layer(layer, cache, cur, x_out=xa, workspace=ws)
+                cur = xa
+        return xa
+
+    fg.fg_profile_select([0])
+    fg.fg_profile_enable(True)
+    for _ in range(args.warmup):
+        step(x0, xdec)
+    fg.fg_profile_reset()
+    launches0 = fg.fg_launch_count()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else 0) as clk:
+        for a, m, b in ev:
+            a.record(stream)
+            step(x0, xdec, m)
+            b.record(stream)
+        barrier()
+    launches = fg.fg_launch_count() - launches0
+    ms_total = max_over_ranks(ev[0][0].elapsed_time(ev[-1][2]), dev)
+    timings = [(a.elapsed_time(m), m.elapsed_time(b)) for a, m, b in ev]
+    prof = fg.fg_profile_read(0)
+    clocks = clk.summary()
+
+    # ---- e2e: the prompt's hidden states and the decode inputs from pinned host memory, the
+    # last hidden states back to the host, every step inside the timed region
+    x0_host = x0.cpu().pin_memory()
+    xdec_host = xdec.cpu().pin_memory()
+    xdec_dev = torch.empty_like(xdec)
+    out_host = torch.empty((B, h), dtype=torch.float16).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+    barrier()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(e2e_steps):
+        xdec_dev.copy_(xdec_host, non_blocking=True)
+        y = step(x0_host, xdec_dev)
+        out_host.copy_(y, non_blocking=True)
+    e3.record(stream)
+    barrier()
+    ms_e2e = max_over_ranks(e2.elapsed_time(e3), dev)
+
+    fg.fg_profile_select(None)
+    fg.fg_profile_reset()
+    step(x0, xdec)
+    breakdown = {fg.PROF_NAMES[k]: fg.fg_profile_read(k) for k in range(7)}
+    fg.fg_profile_enable(False)
+    del layers, caches, ws, x, x0, xdec, xdec_dev
+    torch.cuda.empty_cache()
+    return dict(ms_total=ms_total, ms_e2e=ms_e2e, e2e_steps=e2e_steps, timings=timings, prof=prof,
+                breakdown=breakdown, clocks=clocks, launches=launches,
+                h2d=(B * L + T * B) * h * 2, d2h=B * h * 2)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", choices=sorted(CONFIGS), default=DEFAULT_CONFIG,
+                    help="c3: OPT-30B batch 256 (default); c2: OPT-6.7B batch 64; c4: OPT-175B 12-layer slice, batch 144")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", choices=["generate", "qgemm", "qgemm_decode", "gemm_f16", "gemm_prefill", "lm_head",
                                        "decode_attention", "prefill_attention", "quantize", "sweep"],
@@ -537,24 +782,26 @@ def main():
         return sweep_case(args)
     if args.case != "generate":
         return kernel_case(args)
+    c = use_config(args.config)
     world, rank, local = replica_env()
-    c = CFG
     wdesc = "4-bit weights" if args.weights == "4bit" else "fp16 (uncompressed) weights"
-    config = {"workload": f"OPT-6.7B-shaped decoder, {wdesc} + 4-bit KV (group 64), batch 64 per GPU, "
-                          "prompt 512, generate 32", "layers": c["n_layers"], "hidden": c["hidden"],
-              "heads": f"{c['n_heads']}x{c['head_dim']}", "ffn": c["ffn"], "vocab": c["vocab"],
+    config = {"workload": describe(c, wdesc), "name": args.config, "layers": c["n_layers"], "hidden": c["hidden"],
+              "heads": f"{c['n_heads']}x{c['head_dim']}", "ffn": c["ffn"], "vocab": c["vocab"] or None,
               "global_batch": c["batch"] * max(world, args.gpus if world == 1 else world),
               "prompt_len": c["prompt_len"], "gen_len": c["gen_len"], "group": c["group"],
               "parallelism": f"replicas x{max(world, 1)} (batch-sharded, no exchange)",
-              "l2": "inputs larger than L2 (3.6 GB of 4-bit weights + 5 GB KV cache per step)"}
+              "l2": f"inputs larger than L2 ({weight_bytes_4bit(c) / 1e9:.1f} GB of 4-bit weights and the KV "
+                    f"cache read every decode step)"}
+    if c["kind"] == "slice":
+        config["full_layers"] = c["full_layers"]
 
     if args.impl == "reference":
         if rank != 0:
             return
         steps, warmup = args.steps, args.warmup
-        cb = cpu_baseline_line(args, steps, warmup)
+        cb = cpu_baseline_line(args, steps, warmup, single_thread=False)
         line = {"metric": METRIC, "value": cb["value"], "unit": "tokens/s", "n_gpus": world, "steps": steps,
-                "warmup": warmup, "ms_per_step": 1000.0 * c["batch"] * c["gen_len"] / cb["value"],
+                "warmup": warmup, "ms_per_step": 1000.0 * tokens_per_step(c) / cb["value"],
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": config, "impl": "reference",
                 "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
@@ -572,15 +819,6 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
-    model, caches = build_model(fg, torch, dev, args.weights)
-    B, L, T = c["batch"], c["prompt_len"], c["gen_len"]
-    from fg_synth import gpu as sg
-    import fg_synth
-    ids = torch.empty((B, L), dtype=torch.int32, device=dev)
-    sg.fill_ids(ids, replica_seed(rank), fg_synth.S_IDS, c["vocab"])
-    out = torch.empty((B, T), dtype=torch.int32, device=dev)
-    ws = torch.empty((fg.fg_workspace_bytes(model, B, L, T),), dtype=torch.uint8, device=dev)
-    torch.cuda.synchronize()
 
     def barrier():
         if world > 1:
@@ -588,63 +826,17 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
 
-    # The roofline kernel (the prompt-pass GEMM) is timed by CUDA events from the warm-up on:
-    # the library records them as nodes of its CUDA graphs (first call eager, second
-    # captured, later ones replayed), so the timed steps replay graphs that carry them.
-    # Only that kernel class is timed here; the per-kernel breakdown comes from one more,
-    # separately profiled step after the timed regions.
-    fg.fg_profile_select([0])
-    fg.fg_profile_enable(True)
-    for _ in range(args.warmup):
-        fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
-    # ---- timed region: device-resident inputs
-    fg.fg_profile_reset()
-    launches0 = fg.fg_launch_count()
-    timings = []
-    barrier()
-    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local) as clk:
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        torch.cuda.nvtx.range_push("timed_steps")
-        for _ in range(args.steps):
-            _, tm = fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
-            timings.append((tm.prefill_ms, tm.decode_ms))
-        torch.cuda.nvtx.range_pop()
-        e1.record(stream)
-        barrier()
-    launches = fg.fg_launch_count() - launches0
-    ms_total = max_over_ranks(e0.elapsed_time(e1), dev)
-    ms_step = ms_total / args.steps
-    value = job_throughput(B * T, world, args.steps, ms_total)
-    prof = {fg.PROF_NAMES[k]: fg.fg_profile_read(k) for k in range(7)}
-    clocks = clk.summary()
-
-    # ---- e2e: host buffers through the public API, copies inside the timed region (the
-    # prompt ids go host -> the same device buffer, so the recorded graphs stay valid)
-    ids_host = ids.cpu().pin_memory()
-    out_host = torch.empty((B, T), dtype=torch.int32).pin_memory()
-    barrier()
-    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2.record(stream)
-    for _ in range(args.steps):
-        ids.copy_(ids_host, non_blocking=True)
-        fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
-        out_host.copy_(out, non_blocking=True)
-    e3.record(stream)
-    barrier()
-
-    # ---- per-kernel breakdown: every kernel class timed, one replayed step (not timed above)
-    fg.fg_profile_select(None)
-    for _ in range(2):   # eager, then captured with the new timing nodes
-        fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
-    fg.fg_profile_reset()
-    fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
-    breakdown = {fg.PROF_NAMES[k]: fg.fg_profile_read(k) for k in range(7)}
-    fg.fg_profile_enable(False)
-    ms_e2e = max_over_ranks(e2.elapsed_time(e3), dev)
-    e2e_value = job_throughput(B * T, world, args.steps, ms_e2e)
+    runner = run_slice if c["kind"] == "slice" else run_generate
+    r = runner(args, fg, torch, dev, stream, world, rank, barrier)
+    B, L, T = c["batch"], c["prompt_len"], c["gen_len"]
+    scale = c["n_layers"] / c["full_layers"] if c["kind"] == "slice" else 1.0
+    ms_step = r["ms_total"] / args.steps
+    slice_value = job_throughput(tokens_per_step(c), world, args.steps, r["ms_total"])
+    value = slice_value * scale
+    e2e_value = job_throughput(tokens_per_step(c), world, r["e2e_steps"], r["ms_e2e"]) * scale
 
     # ---- quantizer GB/s on a 1 GiB fp16 tensor (group 64), bytes = 2 + 0.5 + 4/64 per element
+    from fg_synth import gpu as sg
     xq = torch.empty((131072, 4096), dtype=torch.float16, device=dev)
     sg.fill(xq, SEED, 7, "normal", 0.02)
     codes = torch.empty((131072, 2048), dtype=torch.uint8, device=dev)
@@ -662,17 +854,18 @@ def main():
     q_gbs = xq.numel() * (2 + 0.5 + 4 / 64) / (q_ms * 1e-3) / 1e9
     del xq, codes, params
 
-    # ---- decode attention GB/s at the last decode step's shape (B 64, 32 x 128, context 543,
-    # 160 MB of 4-bit cache, larger than L2), timed on its own
+    # ---- decode attention GB/s at the last decode step's shape of this workload (larger
+    # than L2), timed on its own
     S_att = L + T - 1
-    h = c["hidden"]
-    kvsrc = torch.empty((B * S_att, 2 * h), dtype=torch.float16, device=dev)
-    sg.fill(kvsrc, SEED, 3, "normal", 1.0)
+    h, nh, hd, g = c["hidden"], c["n_heads"], c["head_dim"], c["group"]
+    acache = fg.DeviceKVCache(B, nh, hd, S_att, g, dev)
     qa = torch.empty((B, 3 * h), dtype=torch.float16, device=dev)
     sg.fill(qa, SEED, 4, "normal", 1.0)
-    acache = fg.DeviceKVCache(B, c["n_heads"], c["head_dim"], S_att, c["group"], dev)
+    kvsrc = torch.empty((B * S_att, 2 * h), dtype=torch.float16, device=dev)   # 4 GB at c3
+    sg.fill(kvsrc, SEED, 3, "normal", 1.0)
     fg.fg_kv_append(acache, kvsrc, kvsrc[:, h:], 2 * h, S_att)
     del kvsrc
+    torch.cuda.empty_cache()
     aout = torch.empty((B, h), dtype=torch.float16, device=dev)
     for _ in range(3):
         fg.fg_decode_attention(qa, 3 * h, acache, out=aout)
@@ -682,7 +875,7 @@ def main():
     e5.record(stream)
     torch.cuda.synchronize()
     att_ms = e4.elapsed_time(e5) / reps
-    att_bytes = B * c["n_heads"] * S_att * 2.0 * (c["head_dim"] / 2 + 4.0 * c["head_dim"] / c["group"]) + 4.0 * B * h
+    att_bytes = B * nh * S_att * 2.0 * (hd / 2 + 4.0 * hd / g) + 4.0 * B * h
     att_gbs = att_bytes / (att_ms * 1e-3) / 1e9
     del acache, qa, aout
 
@@ -694,14 +887,14 @@ def main():
         return
 
     pk = peaks()
-    g = prof["gemm_prefill"]
-    g_ms = g["ms"] / max(g["launches"], 1)
-    g_flops = g["flops"] / max(g["launches"], 1)
+    prof, breakdown = r["prof"], r["breakdown"]
+    g_ms = prof["ms"] / max(prof["launches"], 1)
+    g_flops = prof["flops"] / max(prof["launches"], 1)
     achieved_tf = g_flops / (g_ms * 1e-3) / 1e12 if g_ms > 0 else 0.0
     traffic = None
     tfile = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tfile):
-        traffic = json.load(open(tfile)).get("gemm_prefill_bytes_per_launch")
+        traffic = json.load(open(tfile)).get(f"gemm_prefill_bytes_per_launch_{args.config}")
     da = breakdown["decode_attention"]
     kernels = {}
     for name, p in breakdown.items():
@@ -712,33 +905,40 @@ def main():
             if p["bytes"] and p["ms"]:
                 d["GB/s"] = p["bytes"] / (p["ms"] * 1e-3) / 1e9
             kernels[name] = d
+    M_pf = B * L
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic", "config": config,
-        "prefill_ms": statistics.median(t[0] for t in timings), "decode_ms": statistics.median(t[1] for t in timings),
-        "roofline": {"kernel": "tcgen05 GEMM of the prompt pass (M = 32768; " +
+        "prefill_ms": statistics.median(t[0] for t in r["timings"]),
+        "decode_ms": statistics.median(t[1] for t in r["timings"]),
+        "roofline": {"kernel": f"tcgen05 GEMM of the prompt pass (M = {M_pf}; " +
                                ("4-bit weights expanded to fp16 once per layer)" if args.weights == "4bit"
                                 else "uncompressed fp16 weights)"), "bound": "tensor",
                      "achieved": achieved_tf, "peak": pk["tf_sust"], "unit": "TFLOP/s",
                      "frac": achieved_tf / pk["tf_sust"], "traffic": traffic,
+                     "flop_per_launch": g_flops, "ms_per_launch": g_ms,
                      "peak_source": f"bf16_tflops_sustained of {pk['src']} peaks (fp16 and bf16 dense rates are equal)"},
         "quantizer": {"GB/s": q_gbs, "frac": q_gbs / pk["hbm"], "peak_GB/s": pk["hbm"],
                       "tensor": "1 GiB fp16 (131072 x 4096), group 64"},
         "decode_attention": {"GB/s": att_gbs, "frac": att_gbs / pk["hbm"], "peak_GB/s": pk["hbm"],
-                             "shape": f"B {B}, {c['n_heads']} x {c['head_dim']}, context {S_att}, group {c['group']}",
+                             "shape": f"B {B}, {nh} x {hd}, context {S_att}, group {g}",
                              "in_step_GB/s": da["bytes"] / (da["ms"] * 1e-3) / 1e9 if da["ms"] else None},
         "kernels": kernels,
-        "kernels_note": "one extra replayed step with every kernel class timed (outside the timed region)",
-        "clocks": clocks,
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": B * L * 4,
-                "d2h_bytes_per_step": B * T * 4},
-        "gpu_launches": launches,
+        "kernels_note": "one extra step with every kernel class timed (outside the timed region)",
+        "clocks": r["clocks"],
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"], "steps": r["e2e_steps"]},
+        "gpu_launches": r["launches"],
     }
+    if c["kind"] == "slice":
+        line["slice"] = {"tokens_per_s_12_layers": slice_value, "per_layer_tokens_per_s": slice_value * c["n_layers"],
+                         "extrapolation": f"value = slice tokens/s x {c['n_layers']}/{c['full_layers']} "
+                                          "(per-layer time constant; embedding and LM head excluded)"}
     if world == 1 and not args.no_cpu_baseline:
         try:
             cb = cpu_baseline_line(args, 1, 0)
-            line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+            line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample", "single_thread")}
         except Exception as ex:  # the baseline is informative only
             line["cpu_baseline"] = {"value": None, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
                                     "sample": f"failed: {ex}"}

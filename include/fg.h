@@ -175,7 +175,8 @@ int fg_decode_attention(const void* q, int64_t q_stride, const fg_kv_cache* cach
  *  - A shape whose partials need more than 4 MiB (fg_decode_attention_workspace_bytes tells)
  *    is rejected with FG_ERR_WORKSPACE before any launch.
  *  - The first call on a device looks up the array's address with that device current; make
- *    that first call before any stream capture.
+ *    that first call before any stream capture.  The address is kept for the life of the
+ *    process: after cudaDeviceReset on a device, do not call this function on that device again.
  *  - All calls share the array.  Each call writes every partial it reads, so nothing carries
  *    over between calls, but calls that overlap on the GPU (other streams or threads) race. */
 int fg_decode_attention_noalloc(const void* q, int64_t q_stride, const fg_kv_cache* cache,

@@ -3,8 +3,14 @@
 TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports, calls or links this
 package; only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
 ``--impl reference`` legs of ``bench.py`` use it.  It shares no code with the CUDA
-library: it is a plain, slow restatement of what the path computes, written with numpy
-(float32 where the definition fixes IEEE single precision, float64 elsewhere).
+library.
+
+The oracle is a plain, slow C++17 program, ``fg_oracle.cpp`` (built with g++ into
+``liboracle.so``, ``-O2 -ffp-contract=off -fno-fast-math``, OpenMP over independent
+rows): its own fp16 rounding, the quantizer in IEEE single precision, the decoder in
+double precision with fp16 at the storage points.  The Python modules ``quant.py`` and
+``decoder.py`` only marshal numpy buffers into it.  ``numpy_ref/`` holds a second,
+independent restatement in numpy, kept only as a cross-check of the C++ one.
 
 Sources (pages of the subject, cited by page title and section):
 
@@ -19,9 +25,10 @@ Sources (pages of the subject, cited by page title and section):
   compressing weights and the attention cache to 4 bits.
 
 The pages give no formula, group size, rounding mode or layout; the readings this
-oracle takes where they are silent are listed in the module docstrings of
-``quant.py`` and ``decoder.py``.
+oracle takes where they are silent are listed at the top of ``fg_oracle.cpp`` and in
+the module docstrings of ``quant.py`` and ``decoder.py``.
 """
+from ._lib import build, threads
 from .quant import (quantize_groups, dequantize_groups, pack_nibbles, unpack_nibbles,
                     quantize_pack, dequantize, storage_bytes)
 from .decoder import (layernorm, qlinear, linear_fp16, prefill_attention, decode_attention,
@@ -29,6 +36,7 @@ from .decoder import (layernorm, qlinear, linear_fp16, prefill_attention, decode
                       lm_head_argmax, QLinear, Linear16, QLayer, KVCache, Model)
 
 __all__ = [
+    "build", "threads",
     "quantize_groups", "dequantize_groups", "pack_nibbles", "unpack_nibbles",
     "quantize_pack", "dequantize", "storage_bytes", "layernorm", "qlinear", "linear_fp16",
     "prefill_attention", "decode_attention", "kv_append", "cache_dequant", "cache_values", "decode_layer",

@@ -1,57 +1,57 @@
-"""Oracle for the OPT-shaped decoder over 4-bit weights and a 4-bit KV cache
+"""The OPT-shaped decoder over 4-bit weights and a 4-bit KV cache: the oracle's decoder
 (test infrastructure only).
+
+Every value here is computed by the C++ oracle (``fg_oracle.cpp``: LayerNorm, the linear
+layer, prefill and decode attention, the KV append, the layers, the embedding, the LM head
+and the generation loop); this module holds the model state as numpy arrays and shapes
+buffers for those calls.
 
 The pages name the model family and workload only: OPT-6.7B/30B/175B generation with
 input length 512 and output length 32, throughput = generated tokens / (prompt time +
 generation time) ("FlexGen" README mirror, benchmark table and its workload/metric
 notes), with weights and attention cache compressed to 4 bits (same page, key features;
-arXiv 2303.06865 record, abstract).  The block structure is the standard OPT decoder
-block (pre-LayerNorm, multi-head causal attention, ReLU FFN, learned positions, tied
-LM head).  Readings taken where the pages are silent:
+arXiv 2303.06865 record, abstract).  The block is the standard OPT decoder block
+(pre-LayerNorm, multi-head causal attention, ReLU FFN, learned positions, tied LM head).
+Readings taken where the pages are silent (D1-D7 in the C++ file):
 
-* Math convention Y = X @ W + b with W stored [in][out] (out contiguous) and quantized
-  in groups along `out` (see ``quant.py``); Q, K and V come from one [h, 3h] projection,
-  columns ordered q | k | v, head j owning columns j*hd .. (j+1)*hd-1 of each part.
-* Storage precision points (the values the GPU path keeps in memory) are fp16: the
-  residual stream, LayerNorm outputs, projection outputs, attention outputs, the
-  dequantized weights and K/V.  Between those points this oracle computes in float64.
-* LayerNorm eps = 1e-5, statistics over the hidden dimension.
+* Y = X @ W + b with W stored [in][out] (out contiguous) and quantized in groups along
+  `out`; Q, K and V come from one [h, 3h] projection, columns q | k | v, head j owning
+  columns j*hd .. (j+1)*hd-1 of each part.
+* fp16 at the storage points (residual stream, LayerNorm outputs, projection outputs,
+  attention outputs, the dequantized weights and K/V), float64 in between.
+* LayerNorm eps = 1e-5 inside the square root, population variance over the hidden dim.
 * Attention scale 1/sqrt(hd).  Prefill attention uses this pass's unquantized fp16 K/V;
   every token's K and V is then appended to the 4-bit cache in groups of g along the
-  hidden dimension (g divides hd).  A decode step appends the new token first and then
-  attends over all cached positions 0..len (the new one included).  Decode attention
-  consumes the value each code stands for, mn + code*s, exactly (no second rounding to
-  fp16); the softmax and the weighted sum are float64 here, fp32 on the GPU.
+  hidden dimension.  A decode step appends the new token first and then attends over
+  positions 0..len (the new one included), consuming the exact values mn + code*s.
 * Embedding x = fp16(E[id] + P[pos]) (one rounding), positions 0..L-1 for the prompt and
   L+j-1 for the j-th generated token; no position offset.
-* LM head logits = LN_f(x) @ E^T with the tied fp16 embedding (not quantized); greedy
-  token = argmax, ties to the lowest id.
-* Output length T counts the token produced by the prefill: T tokens = 1 from the
-  prefill + T-1 decode steps.
+* LM head logits = LN_f(x) @ E^T with the tied fp16 embedding; greedy token = argmax,
+  ties to the lowest id.
+* T output tokens = 1 from the prompt pass + T-1 decode steps.
 """
 from __future__ import annotations
 
+import ctypes
 from dataclasses import dataclass, field
 from typing import List, Optional
 
 import numpy as np
 
+from . import _lib
+from ._lib import f16, lib, p
 from .quant import quantize_pack, dequantize
 
 LN_EPS = 1e-5
 
 
-def _f64(a):
-    return np.asarray(a).astype(np.float64)
-
-
 def layernorm(x16: np.ndarray, g16: np.ndarray, b16: np.ndarray, eps: float = LN_EPS) -> np.ndarray:
     """y = (x - mean) / sqrt(var + eps) * gamma + beta over the last axis -> fp16."""
-    x = _f64(x16)
-    mu = x.mean(axis=-1, keepdims=True)
-    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
-    y = (x - mu) / np.sqrt(var + eps) * _f64(g16) + _f64(b16)
-    return y.astype(np.float16)
+    x = f16(x16)
+    h = x.shape[-1]
+    y = np.empty_like(x)
+    lib().orc_layernorm(p(x), x.size // h, h, p(f16(g16)), p(f16(b16)), float(eps), p(y))
+    return y
 
 
 @dataclass
@@ -63,29 +63,38 @@ class QLinear:
     K: int
     N: int
     group: int = 64
-    _w: Optional[np.ndarray] = field(default=None, repr=False)
+    _w16: Optional[np.ndarray] = field(default=None, repr=False)
 
     @staticmethod
     def from_fp16(w16: np.ndarray, b16: np.ndarray, group: int = 64) -> "QLinear":
         K, N = w16.shape
         codes, params = quantize_pack(w16, group, axis=1)
-        return QLinear(codes, params, np.asarray(b16, np.float16), K, N, group)
+        return QLinear(codes, params, f16(b16), K, N, group)
+
+    def weight16(self) -> np.ndarray:
+        """W_hat as fp16 [K, N] (the oracle's dequantization of the stored weight)."""
+        if self._w16 is None:
+            self._w16 = dequantize(self.codes, self.params, self.K, self.N, self.group, 1)
+        return self._w16
 
     def weight(self) -> np.ndarray:
-        """Dequantized weight as float64 [K, N] (the exact fp16 values)."""
-        if self._w is None:
-            self._w = dequantize(self.codes, self.params, self.K, self.N, self.group, 1).astype(np.float64)
-        return self._w
+        """W_hat as float64 [K, N] (the exact fp16 values)."""
+        return self.weight16().astype(np.float64)
 
     def columns(self, cols) -> np.ndarray:
-        """Dequantized columns ``cols`` only, float64 [K, len(cols)] (for sampled checks)."""
+        """Dequantized columns ``cols`` only, float64 [K, len(cols)]; only the groups holding
+        them are dequantized (for sampled checks of large weights)."""
         cols = np.asarray(cols)
-        p = np.asarray(self.params, np.float16)
-        q_lo_hi = self.codes[:, cols // 2]
-        q = np.where(cols % 2 == 0, q_lo_hi & 0x0F, q_lo_hi >> 4).astype(np.float64)
-        grp = p[:, cols // self.group, :]
-        exact = q * grp[..., 1].astype(np.float64) + grp[..., 0].astype(np.float64)
-        return exact.astype(np.float16).astype(np.float64)
+        g = self.group
+        out = np.empty((self.K, len(cols)), np.float64)
+        for gi in np.unique(cols // g):
+            gi = int(gi)
+            codes = np.ascontiguousarray(self.codes[:, gi * g // 2:(gi + 1) * g // 2])
+            params = np.ascontiguousarray(np.asarray(self.params, np.float16).reshape(self.K, -1, 2)[:, gi])
+            wg = dequantize(codes, params, self.K, g, g, 1)
+            sel = np.nonzero(cols // g == gi)[0]
+            out[:, sel] = wg[:, cols[sel] - gi * g].astype(np.float64)
+        return out
 
 
 @dataclass
@@ -103,24 +112,35 @@ class Linear16:
     def N(self) -> int:
         return self.w16.shape[1]
 
+    def weight16(self) -> np.ndarray:
+        return f16(self.w16)
+
     def weight(self) -> np.ndarray:
-        return np.asarray(self.w16, np.float16).astype(np.float64)
+        return self.weight16().astype(np.float64)
 
 
-def qlinear(a16: np.ndarray, lin: QLinear, relu: bool = False,
-            residual16: Optional[np.ndarray] = None) -> np.ndarray:
-    """fp16( [relu](a @ W_hat + b) [+ residual] ), float64 in between."""
-    acc = _f64(a16) @ lin.weight() + _f64(lin.bias)
-    if relu:
-        acc = np.maximum(acc, 0.0)
-    if residual16 is not None:
-        acc = acc + _f64(residual16)
-    return acc.astype(np.float16)
+def qlinear(a16: np.ndarray, lin, relu: bool = False, residual16: Optional[np.ndarray] = None) -> np.ndarray:
+    """fp16( [relu](a @ W_hat + b) [+ residual] ), float64 in between (QLinear or Linear16)."""
+    a = f16(a16)
+    K = a.shape[-1]
+    M = a.size // K
+    W = lin.weight16()
+    assert W.shape == (K, lin.N)
+    r = None if residual16 is None else f16(residual16).reshape(M, lin.N)
+    y = np.empty(a.shape[:-1] + (lin.N,), np.float16)
+    lib().orc_linear(p(a), M, K, p(W), K, lin.N, p(None if lin.bias is None else f16(lin.bias)), int(relu), p(r),
+                     p(y))
+    return y
 
 
 def linear_fp16(a16: np.ndarray, w_nk16: np.ndarray) -> np.ndarray:
     """a @ W^T for an fp16 weight stored [N][K]; float64 result (logits)."""
-    return _f64(a16) @ _f64(w_nk16).T
+    a = f16(a16)
+    E = f16(w_nk16)
+    M, K = a.shape
+    out = np.empty((M, E.shape[0]), np.float64)
+    lib().orc_linear_nk(p(a), M, p(E), E.shape[0], K, p(out))
+    return out
 
 
 @dataclass
@@ -129,10 +149,10 @@ class QLayer:
     ln1_b: np.ndarray
     ln2_g: np.ndarray
     ln2_b: np.ndarray
-    qkv: QLinear
-    out: QLinear
-    fc1: QLinear
-    fc2: QLinear
+    qkv: object
+    out: object
+    fc1: object
+    fc2: object
 
 
 @dataclass
@@ -159,118 +179,103 @@ class KVCache:
             self.k_params = np.zeros((B, nh, cap, hd // g, 2), np.float16)
             self.v_params = np.zeros((B, nh, cap, hd // g, 2), np.float16)
 
+    def c(self) -> _lib.Cache:
+        """The C view of this cache (pointers into the numpy arrays)."""
+        return _lib.Cache(p(self.k_codes), p(self.v_codes), p(self.k_params), p(self.v_params), self.B,
+                          self.n_heads, self.head_dim, self.group, self.capacity, self.length)
+
 
 def kv_append(cache: KVCache, k16: np.ndarray, v16: np.ndarray, pos: int) -> None:
     """Quantize tokens' K and V rows ([B, T, h] or [B, h]) into positions pos.. of the cache."""
-    k16 = np.asarray(k16, np.float16)
-    v16 = np.asarray(v16, np.float16)
-    if k16.ndim == 2:
-        k16, v16 = k16[:, None, :], v16[:, None, :]
-    B, T, h = k16.shape
-    nh, hd, g = cache.n_heads, cache.head_dim, cache.group
+    k = f16(k16)
+    v = f16(v16)
+    if k.ndim == 2:
+        k, v = k[:, None, :], v[:, None, :]
+    B, T, h = k.shape
     if pos + T > cache.capacity:
         raise ValueError("KV cache capacity exceeded")
-    for src, codes_dst, params_dst in ((k16, cache.k_codes, cache.k_params),
-                                       (v16, cache.v_codes, cache.v_params)):
-        codes, params = quantize_pack(src.reshape(B * T, h), g, axis=1)
-        codes_dst[:, :, pos:pos + T, :] = codes.reshape(B, T, nh, hd // 2).transpose(0, 2, 1, 3)
-        params_dst[:, :, pos:pos + T] = params.reshape(B, T, nh, hd // g, 2).transpose(0, 2, 1, 3, 4)
+    c = cache.c()
+    assert lib().orc_kv_append(ctypes.byref(c), p(k), p(v), h, T, pos) == 0
 
 
 def cache_dequant(cache: KVCache, which: str, b: int, head: int, S: int) -> np.ndarray:
     """Dequantized K or V of one (sequence, head) for positions 0..S-1, fp16 [S, hd]
     (the storage form, as fg_dequantize would write it)."""
-    codes = (cache.k_codes if which == "k" else cache.v_codes)[b, head, :S]
-    params = (cache.k_params if which == "k" else cache.v_params)[b, head, :S]
-    return dequantize(codes, params.reshape(-1, 2), S, cache.head_dim, cache.group, 1)
+    codes = np.ascontiguousarray((cache.k_codes if which == "k" else cache.v_codes)[b, head, :S])
+    params = np.ascontiguousarray((cache.k_params if which == "k" else cache.v_params)[b, head, :S])
+    return dequantize(codes, params, S, cache.head_dim, cache.group, 1)
 
 
 def cache_values(cache: KVCache, which: str, b: int, head: int, S: int) -> np.ndarray:
-    """Exact values mn + code*s of one (sequence, head), positions 0..S-1, float64 [S, hd].
-
-    This is what attention consumes: the value the 4-bit code stands for, without a
-    second rounding to fp16 (the product and sum are exact in float64)."""
-    codes = (cache.k_codes if which == "k" else cache.v_codes)[b, head, :S]
-    params = (cache.k_params if which == "k" else cache.v_params)[b, head, :S].astype(np.float64)
-    g = cache.group
-    q = np.empty((S, cache.head_dim), np.float64)
-    q[:, 0::2] = codes & 0x0F
-    q[:, 1::2] = codes >> 4
-    mn = np.repeat(params[..., 0], g, axis=1)
-    sc = np.repeat(params[..., 1], g, axis=1)
-    return mn + q * sc
-
-
-def _softmax_rows(s: np.ndarray) -> np.ndarray:
-    m = s.max(axis=-1, keepdims=True)
-    e = np.exp(s - m)
-    return e / e.sum(axis=-1, keepdims=True)
+    """Exact values mn + code*s of one (sequence, head), positions 0..S-1, float64 [S, hd]:
+    what attention consumes (no second rounding to fp16)."""
+    codes = np.ascontiguousarray((cache.k_codes if which == "k" else cache.v_codes)[b, head, :S])
+    params = np.ascontiguousarray((cache.k_params if which == "k" else cache.v_params)[b, head, :S])
+    out = np.empty((S, cache.head_dim), np.float64)
+    lib().orc_code_values(p(codes), p(params), S, cache.head_dim, cache.group, p(out))
+    return out
 
 
 def prefill_attention(qkv16: np.ndarray, n_heads: int, head_dim: int) -> np.ndarray:
     """Causal multi-head attention over [B, L, 3h] fp16 projections -> fp16 [B, L, h]."""
-    qkv = _f64(qkv16)
+    qkv = f16(qkv16)
     B, L, h3 = qkv.shape
-    h = h3 // 3
-    out = np.empty((B, L, h), np.float64)
-    scale = 1.0 / np.sqrt(head_dim)
-    mask = np.triu(np.ones((L, L), bool), k=1)          # key j > query i is masked
-    for j in range(n_heads):
-        c = slice(j * head_dim, (j + 1) * head_dim)
-        q = qkv[:, :, 0 * h:1 * h][:, :, c]
-        k = qkv[:, :, 1 * h:2 * h][:, :, c]
-        v = qkv[:, :, 2 * h:3 * h][:, :, c]
-        s = np.einsum("bid,bjd->bij", q, k) * scale
-        s[:, mask] = -np.inf
-        out[:, :, c] = np.einsum("bij,bjd->bid", _softmax_rows(s), v)
-    return out.astype(np.float16)
+    out = np.empty((B, L, h3 // 3), np.float16)
+    lib().orc_prefill_attention(p(qkv), B, L, n_heads, head_dim, p(out))
+    return out
 
 
 def decode_attention(q16: np.ndarray, cache: KVCache, S: int) -> np.ndarray:
-    """One query per sequence over cached positions 0..S-1 (dequantized) -> fp16 [B, h]."""
-    q = _f64(q16)
+    """One query per sequence over cached positions 0..S-1 (exact code values) -> fp16 [B, h]."""
+    q = f16(q16)
     B = q.shape[0]
-    nh, hd = cache.n_heads, cache.head_dim
-    out = np.empty((B, nh * hd), np.float64)
-    scale = 1.0 / np.sqrt(hd)
-    for b in range(B):
-        for j in range(nh):
-            c = slice(j * hd, (j + 1) * hd)
-            K = cache_values(cache, "k", b, j, S)
-            V = cache_values(cache, "v", b, j, S)
-            p = _softmax_rows((K @ q[b, c]) * scale)
-            out[b, c] = p @ V
-    return out.astype(np.float16)
+    out = np.empty((B, cache.n_heads * cache.head_dim), np.float16)
+    c = cache.c()
+    lib().orc_decode_attention(p(q), q.shape[1], ctypes.byref(c), S, p(out))
+    return out
+
+
+def _linear_c(lin) -> _lib.LinearW:
+    return _lib.LinearW(p(lin.weight16()), p(None if lin.bias is None else f16(lin.bias)), lin.K, lin.N)
+
+
+class _LayerC:
+    """C view of a QLayer, holding references to every buffer it points at."""
+
+    def __init__(self, layer: QLayer):
+        self.keep = [f16(layer.ln1_g), f16(layer.ln1_b), f16(layer.ln2_g), f16(layer.ln2_b)]
+        for lin in (layer.qkv, layer.out, layer.fc1, layer.fc2):
+            self.keep += [lin.weight16(), None if lin.bias is None else f16(lin.bias)]
+        lins = []
+        for i in range(4):
+            w, b = self.keep[4 + 2 * i], self.keep[5 + 2 * i]
+            lin = (layer.qkv, layer.out, layer.fc1, layer.fc2)[i]
+            lins.append(_lib.LinearW(p(w), p(b), lin.K, lin.N))
+        self.c = _lib.Layer(*[p(a) for a in self.keep[:4]], *lins)
 
 
 def prefill_layer(layer: QLayer, cache: KVCache, x16: np.ndarray) -> np.ndarray:
     """One decoder block over a whole prompt [B, L, h]; writes cache positions 0..L-1."""
-    B, L, h = x16.shape
-    xf = np.asarray(x16, np.float16).reshape(B * L, h)
-    h1 = layernorm(xf, layer.ln1_g, layer.ln1_b)
-    qkv = qlinear(h1, layer.qkv)
-    kv_append(cache, qkv[:, h:2 * h].reshape(B, L, h), qkv[:, 2 * h:].reshape(B, L, h), 0)
-    cache.length = L
-    att = prefill_attention(qkv.reshape(B, L, 3 * h), cache.n_heads, cache.head_dim)
-    x = qlinear(att.reshape(B * L, h), layer.out, residual16=xf)
-    f = qlinear(layernorm(x, layer.ln2_g, layer.ln2_b), layer.fc1, relu=True)
-    x = qlinear(f, layer.fc2, residual16=x)
-    return x.reshape(B, L, h)
+    x = np.array(x16, dtype=np.float16, copy=True, order="C")
+    B, L, h = x.shape
+    lc = _LayerC(layer)
+    cc = cache.c()
+    cc.len = 0
+    assert lib().orc_prefill_layer(ctypes.byref(lc.c), ctypes.byref(cc), p(x), B, L) == 0
+    cache.length = cc.len
+    return x
 
 
 def decode_layer(layer: QLayer, cache: KVCache, x16: np.ndarray) -> np.ndarray:
     """One decoder block for one new token per sequence [B, h]; appends at cache.length."""
-    x16 = np.asarray(x16, np.float16)
-    h = x16.shape[1]
-    h1 = layernorm(x16, layer.ln1_g, layer.ln1_b)
-    qkv = qlinear(h1, layer.qkv)
-    pos = cache.length
-    kv_append(cache, qkv[:, h:2 * h], qkv[:, 2 * h:], pos)
-    cache.length = pos + 1
-    att = decode_attention(qkv[:, :h], cache, pos + 1)
-    x = qlinear(att, layer.out, residual16=x16)
-    f = qlinear(layernorm(x, layer.ln2_g, layer.ln2_b), layer.fc1, relu=True)
-    return qlinear(f, layer.fc2, residual16=x)
+    x = f16(x16)
+    B, h = x.shape
+    y = np.empty_like(x)
+    lc = _LayerC(layer)
+    cc = cache.c()
+    assert lib().orc_decode_layer(ctypes.byref(lc.c), ctypes.byref(cc), p(x), p(y), B) == 0
+    cache.length = cc.len
+    return y
 
 
 @dataclass
@@ -290,18 +295,35 @@ class Model:
     layers: List[QLayer]
 
 
+class _ModelC:
+    def __init__(self, m: Model):
+        self.keep = [f16(m.embed), f16(m.pos_embed), f16(m.lnf_g), f16(m.lnf_b)]
+        self.layers = [_LayerC(l) for l in m.layers]
+        arr = (_lib.Layer * max(1, len(self.layers)))(*[l.c for l in self.layers])
+        self.arr = arr
+        self.c = _lib.Model(m.n_layers, m.hidden, m.n_heads, m.head_dim, m.ffn, m.vocab, m.max_pos, m.group,
+                            *[p(a) for a in self.keep], ctypes.cast(arr, ctypes.POINTER(_lib.Layer)))
+
+
 def embed(model: Model, ids: np.ndarray, pos0: int) -> np.ndarray:
     """fp16(E[id] + P[pos]) with one rounding; ids [B, T] -> [B, T, h]."""
-    ids = np.asarray(ids)
-    T = ids.shape[1]
-    pos = np.arange(pos0, pos0 + T)
-    return (_f64(model.embed[ids]) + _f64(model.pos_embed[pos])[None]).astype(np.float16)
+    ids = np.ascontiguousarray(ids, np.int32)
+    B, T = ids.shape
+    mc = _ModelC(model)
+    out = np.empty((B, T, model.hidden), np.float16)
+    lib().orc_embed(ctypes.byref(mc.c), p(ids), B, T, pos0, p(out))
+    return out
 
 
 def lm_head_argmax(model: Model, x16: np.ndarray):
     """Final LayerNorm, tied LM head, greedy argmax (lowest id on ties).  x16 [B, h]."""
-    logits = linear_fp16(layernorm(x16, model.lnf_g, model.lnf_b), model.embed)
-    return np.argmax(logits, axis=-1).astype(np.int32), logits   # argmax returns the first max
+    x = f16(x16)
+    B = x.shape[0]
+    mc = _ModelC(model)
+    logits = np.empty((B, model.vocab), np.float64)
+    tok = np.empty(B, np.int32)
+    lib().orc_lm_head_argmax(ctypes.byref(mc.c), p(x), B, p(logits), p(tok))
+    return tok, logits
 
 
 def generate(model: Model, ids: np.ndarray, gen_len: int, return_logits: bool = False):
@@ -309,23 +331,14 @@ def generate(model: Model, ids: np.ndarray, gen_len: int, return_logits: bool = 
 
     Returns tokens [B, gen_len] (and the float64 logits [gen_len, B, vocab] if asked).
     """
-    ids = np.asarray(ids, np.int32)
+    ids = np.ascontiguousarray(ids, np.int32)
     B, L = ids.shape
-    caches = [KVCache(B, model.n_heads, model.head_dim, model.group, L + gen_len)
-              for _ in range(model.n_layers)]
-    x = embed(model, ids, 0)
-    for layer, cache in zip(model.layers, caches):
-        x = prefill_layer(layer, cache, x)
-    tok, logits = lm_head_argmax(model, x[:, -1, :])
-    toks, all_logits = [tok], [logits]
-    for step in range(1, gen_len):
-        x = embed(model, tok[:, None], L + step - 1)[:, 0, :]
-        for layer, cache in zip(model.layers, caches):
-            x = decode_layer(layer, cache, x)
-        tok, logits = lm_head_argmax(model, x)
-        toks.append(tok)
-        all_logits.append(logits)
-    out = np.stack(toks, axis=1)
+    caches = [KVCache(B, model.n_heads, model.head_dim, model.group, L + gen_len) for _ in range(model.n_layers)]
+    cc = (_lib.Cache * max(1, len(caches)))(*[c.c() for c in caches])
+    mc = _ModelC(model)
+    out = np.empty((B, gen_len), np.int32)
+    logits = np.empty((gen_len, B, model.vocab), np.float64) if return_logits else None
+    assert lib().orc_generate(ctypes.byref(mc.c), p(ids), B, L, gen_len, p(out), cc, p(logits)) == 0
     if return_logits:
-        return out, np.stack(all_logits, axis=0)
+        return out, logits
     return out

@@ -29,10 +29,21 @@ def test_product_never_reaches_the_oracle():
 
 
 def test_oracle_never_reaches_the_cuda_path():
-    for path in _files("oracle", (".py", ".c", ".h")):
+    """The oracle (C++ and its Python marshalling) names neither the CUDA library nor torch,
+    includes nothing of csrc/ or include/, and loads no shared library but its own."""
+    for path in _files("oracle", (".py", ".c", ".cpp", ".h")):
         src = _text(path)
-        for name in ("bit_group_quantized_fg_b200", "libfg", "ctypes", "torch"):
+        for name in ("bit_group_quantized_fg_b200", "libfg", "torch", "fg.h", "csrc", "cuda"):
             assert name not in src, (path, name)
+        if path.endswith(".py"):
+            for m in re.finditer(r"CDLL\(([^)]*)\)", src):
+                assert m.group(1).strip() == "path", (path, m.group(0))
+            if "ctypes" in src:
+                assert os.path.basename(path) in ("_lib.py", "decoder.py"), path
+    lib_src = _text(os.path.join(ROOT, "oracle", "_lib.py"))
+    assert 'LIB = os.path.join(HERE, "liboracle.so")' in lib_src
+    for inc in re.findall(r'#include\s*[<"]([^>"]+)[>"]', _text(os.path.join(ROOT, "oracle", "fg_oracle.cpp"))):
+        assert inc in ("cmath", "cstdint", "cstring", "vector", "omp.h"), inc
 
 
 def test_input_generator_depends_on_neither():
@@ -60,7 +71,7 @@ def _oracle_import_sites(path):
 
 
 def test_oracle_imported_only_by_tests_smoke_and_cpu_baseline():
-    allowed = {"__graft_entry__.py": {"smoke"}, "bench.py": {"oracle_sample"}}
+    allowed = {"__graft_entry__.py": {"smoke"}, "bench.py": {"oracle_sample", "cpu_baseline_line"}}
     for path in _files(".", (".py",)):
         rel = os.path.relpath(path, ROOT)
         top = rel.split(os.sep)[0]
@@ -71,3 +82,19 @@ def test_oracle_imported_only_by_tests_smoke_and_cpu_baseline():
             continue
         assert rel in allowed, f"{rel} imports the oracle"
         assert set(sites) <= allowed[rel], (rel, sites)
+
+
+def test_oracle_build_flags_agree():
+    """build() in __graft_entry__ compiles the oracle with the loader's flags (IEEE arithmetic,
+    no contraction, no fast-math)."""
+    import ast as _ast
+    flags = []
+    for path, name in ((os.path.join(ROOT, "__graft_entry__.py"), "ORACLE_FLAGS"),
+                       (os.path.join(ROOT, "oracle", "_lib.py"), "FLAGS")):
+        tree = _ast.parse(_text(path))
+        vals = [_ast.literal_eval(n.value) for n in tree.body if isinstance(n, _ast.Assign)
+                and any(isinstance(t, _ast.Name) and t.id == name for t in n.targets)]
+        assert len(vals) == 1, (path, name)
+        flags.append(vals[0])
+    assert flags[0] == flags[1]
+    assert "-ffp-contract=off" in flags[0] and "-fno-fast-math" in flags[0]

@@ -70,20 +70,19 @@ def test_qgemm_decode_batches(fg, M, N, K, g, relu, resid):
     assert_close_rms(got, exp, what="decode qgemm")
 
 
-def oracle_weight_columns(seed, stream, K, N, g, cols, scale=0.02):
-    """W_hat[:, cols] (float64 [K, len(cols)]) of a seeded N(0, scale) weight [K][N], quantized
-    by the oracle group by group: only the groups holding ``cols`` are generated on the CPU."""
+def oracle_weight_groups(seed, stream, K, N, g, cols):
+    """The oracle's QLinear over just the column groups that hold ``cols`` of a seeded
+    N(0, 0.02) weight [K][N] (groups run along N, so each is quantized exactly as inside the
+    full weight), with the N(0, 0.5) bias of those columns drawn from stream + 1; and the
+    positions of ``cols`` in it."""
     cols = np.asarray(cols)
-    out = np.empty((K, len(cols)), np.float64)
-    for gi in np.unique(cols // g):
-        c0 = int(gi) * g
-        idx = (np.arange(K)[:, None] * N + c0 + np.arange(g)[None, :]).ravel()
-        wg = fg_synth.values(seed, stream, idx, "normal", scale).reshape(K, g)
-        codes, params = oracle.quantize_pack(wg, g, axis=1)
-        wh = oracle.dequantize(codes, params, K, g, g, 1).astype(np.float64)
-        sel = np.nonzero(cols // g == gi)[0]
-        out[:, sel] = wh[:, cols[sel] - c0]
-    return out
+    groups = np.unique(cols // g)
+    idx = (np.arange(K)[:, None] * N + (groups[:, None] * g + np.arange(g)[None, :]).reshape(1, -1)).ravel()
+    w = fg_synth.values(seed, stream, idx, "normal", 0.02).reshape(K, len(groups) * g)
+    bcols = (groups[:, None] * g + np.arange(g)[None, :]).ravel()
+    b = fg_synth.values(seed, stream + 1, bcols, "normal", 0.5)
+    pos = np.searchsorted(groups, cols // g) * g + cols % g
+    return oracle.QLinear.from_fp16(w, b, g), pos
 
 
 def _sampled_qgemm(fg, M, N, K, g, seed, rows, cols):
@@ -102,10 +101,9 @@ def _sampled_qgemm(fg, M, N, K, g, seed, rows, cols):
     y = fg.fg_qgemm(x, lin)
     torch.cuda.synchronize()
     assert bool(torch.isfinite(y.float()).all())
-    wcols = oracle_weight_columns(seed, 2, K, N, g, cols)
-    bh = fg_synth.values(seed, 3, np.arange(N), "normal", 0.5)
+    sub, pos = oracle_weight_groups(seed, 2, K, N, g, cols)
     xr = fg_synth.values(seed, 1, (rows[:, None] * K + np.arange(K)[None, :]).ravel(), "normal", 1.0).reshape(-1, K)
-    exp = (xr.astype(np.float64) @ wcols + bh[cols].astype(np.float64)).astype(np.float16)
+    exp = oracle.qlinear(xr, sub)[:, pos]
     return to_np(y)[rows][:, cols], exp
 
 
@@ -134,7 +132,8 @@ def test_qgemm_prefill_size_sampled(fg):
 
 @pytest.mark.parametrize("M,N,K", [(4, 256, 64), (300, 768, 320), (64, 4096, 2048)])
 def test_gemm_f16_matches_oracle(fg, M, N, K):
-    """The uncompressed fp16-weight GEMM against the float64 product of the same fp16 values."""
+    """The uncompressed fp16-weight GEMM against the oracle's linear layer over the same fp16
+    weight (the uncompressed side of the README mirror's with/without compression table)."""
     import torch
     x = fg_synth.tensor(M, 1, (M, K), "normal", 1.0)
     w = fg_synth.tensor(M, 2, (K, N), "normal", 0.02)
@@ -142,8 +141,8 @@ def test_gemm_f16_matches_oracle(fg, M, N, K):
     r = fg_synth.tensor(M, 4, (M, N), "normal", 1.0)
     y = fg.fg_gemm_f16(to_dev(x), to_dev(w), bias=to_dev(b), R=to_dev(r), relu=True)
     torch.cuda.synchronize()
-    exp = np.maximum(x.astype(np.float64) @ w.astype(np.float64) + b.astype(np.float64), 0) + r.astype(np.float64)
-    assert_close_rms(to_np(y), exp.astype(np.float16), what="fp16 GEMM")
+    exp = oracle.qlinear(x, oracle.Linear16(w, b), relu=True, residual16=r)
+    assert_close_rms(to_np(y), exp, what="fp16 GEMM")
 
 
 def test_lm_head_argmax(fg):

@@ -67,6 +67,10 @@ def test_qlinear_picks_rows_and_applies_bias_relu_residual():
     res = np.full((K, N), 0.5, np.float16)
     yres = oracle.qlinear(eye, lin, residual16=res).astype(np.float64)
     assert np.array_equal(yres, W + b + 0.5)
+    # ReLU applies to X W + b, before the residual is added
+    yrr = oracle.qlinear(eye, lin, relu=True, residual16=res).astype(np.float64)
+    assert np.array_equal(yrr, np.maximum(W + b, 0) + 0.5)
+    assert np.any((W + b < 0) & (W + b > -0.5))       # where the other order would differ
     cols = np.array([0, 1, 63, 64, 127])
     assert np.array_equal(lin.columns(cols), W[:, cols])
 
@@ -307,3 +311,80 @@ def test_kv_append_places_heads_and_positions():
                 assert np.array_equal(vv[pos + t], v[b, t, j * hd:(j + 1) * hd].astype(np.float64))
             untouched = [p for p in range(cap) if not pos <= p < pos + T]
             assert not cache.k_codes[b, j, untouched].any() and not cache.v_params[b, j, untouched].any()
+
+
+# ---------------------------------------------------------------- LayerNorm epsilon and LN2's input
+def test_layernorm_epsilon_inside_the_square_root():
+    """A near-constant row 1 +- 2^-8 has variance 2^-16 (the same order as eps = 1e-5), so
+    where eps sits shows: y = +-1/sqrt(1 + eps/2^-16) with eps inside the square root,
+    +-1/(1 + eps/2^-8) with eps added to the standard deviation, +-1 without it."""
+    import math
+    d = 2.0 ** -8
+    x = np.array([[1.0 + d, 1.0 - d] * 32], np.float16)
+    y = oracle.layernorm(x, np.ones(64, np.float16), np.zeros(64, np.float16)).astype(np.float64)
+    inside = 1.0 / math.sqrt(1.0 + 1e-5 / d ** 2)
+    assert np.all(np.abs(y[0, 0::2] - inside) <= 2.0 ** -11)
+    assert np.all(np.abs(y[0, 1::2] + inside) <= 2.0 ** -11)
+    for wrong in (1.0, 1.0 / (1.0 + 1e-5 / d)):
+        assert np.all(np.abs(y[0, 0::2] - wrong) > 1e-2)
+
+
+def test_second_layernorm_reads_the_attention_residual():
+    """A block with V = 0 (attention output 0), an out-projection bias bo that varies by
+    feature, and identity FFN weights: x1 = fp16(x + bo), and the output must be
+    fp16(x1 + relu(LN2(x1))).  Feeding LN2 the block input x instead (LayerNorm is not
+    shift-invariant for a non-constant bo) gives a different result, which is asserted too."""
+    h, F, B, nh = 64, 256, 3, 1
+    zeros_h, ones_h = np.zeros(h, np.float16), np.ones(h, np.float16)
+    bo = f16(np.linspace(-2.0, 2.0, h))
+    w1 = np.zeros((h, F), np.float16)
+    w1[np.arange(h), np.arange(h)] = 1.0
+    w2 = np.zeros((F, h), np.float16)
+    w2[np.arange(h), np.arange(h)] = 1.0
+    layer = QLayer(ones_h, zeros_h, ones_h, zeros_h,
+                   oracle.Linear16(np.zeros((h, 3 * h), np.float16), np.zeros(3 * h, np.float16)),
+                   oracle.Linear16(np.zeros((h, h), np.float16), bo),
+                   oracle.Linear16(w1, np.zeros(F, np.float16)),
+                   oracle.Linear16(w2, np.zeros(h, np.float16)))
+    x = fg_synth.tensor(12, 1, (B, h), "normal", 1.0)
+    x1 = (x.astype(np.float64) + bo.astype(np.float64)).astype(np.float16)
+
+    def block_out(ln_in):
+        ln = oracle.layernorm(ln_in, ones_h, zeros_h).astype(np.float64)
+        return (x1.astype(np.float64) + np.maximum(ln, 0.0)).astype(np.float16)
+    expect, wrong = block_out(x1), block_out(x)
+    assert not np.array_equal(expect, wrong)
+    y = oracle.decode_layer(layer, KVCache(B, nh, h, 64, 2), x)
+    assert np.array_equal(y, expect)
+    xp = fg_synth.tensor(12, 2, (B, 4, h), "normal", 1.0)
+    x1p = (xp.astype(np.float64) + bo.astype(np.float64)).astype(np.float16)
+    lnp = oracle.layernorm(x1p, ones_h, zeros_h).astype(np.float64)
+    yp = oracle.prefill_layer(layer, KVCache(B, nh, h, 64, 4), xp)
+    assert np.array_equal(yp, (x1p.astype(np.float64) + np.maximum(lnp, 0.0)).astype(np.float16))
+
+
+def test_decode_step_attends_over_the_new_token():
+    """All keys zero (uniform attention), V = LN1(x), identity out-projection, zero FFN: a
+    decode step after a 3-token prompt outputs fp16(x + fp16(mean of the 4 cached V)), the
+    new token's V included; the mean over the 3 prompt positions alone is far from it."""
+    h, B, L = 64, 2, 3
+    z = np.zeros
+    wqkv = z((h, 3 * h), np.float16)
+    wqkv[np.arange(h), 2 * h + np.arange(h)] = 1.0          # v = LN1(x); q = k = 0
+    ones_h, zeros_h = np.ones(h, np.float16), z(h, np.float16)
+    layer = QLayer(ones_h, zeros_h, ones_h, zeros_h,
+                   oracle.Linear16(wqkv, z(3 * h, np.float16)),
+                   oracle.Linear16(np.eye(h, dtype=np.float16), zeros_h),
+                   oracle.Linear16(z((h, 128), np.float16), z(128, np.float16)),
+                   oracle.Linear16(z((128, h), np.float16), zeros_h))
+    cache = KVCache(B, 1, h, 64, L + 1)
+    oracle.prefill_layer(layer, cache, fg_synth.tensor(13, 1, (B, L, h), "normal", 1.0))
+    x = fg_synth.tensor(13, 2, (B, h), "normal", 1.0)
+    y = oracle.decode_layer(layer, cache, x).astype(np.float64)
+    assert cache.length == L + 1
+    for b in range(B):
+        V = oracle.cache_values(cache, "v", b, 0, L + 1)
+        with_new = (x[b].astype(np.float64) + V.mean(axis=0).astype(np.float16)).astype(np.float16)
+        without = (x[b].astype(np.float64) + V[:L].mean(axis=0).astype(np.float16)).astype(np.float16)
+        assert np.max(np.abs(y[b] - with_new.astype(np.float64))) <= 2.0 ** -9
+        assert np.max(np.abs(y[b] - without.astype(np.float64))) > 0.05

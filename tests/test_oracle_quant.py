@@ -226,3 +226,30 @@ def test_storage_matches_readme_about_70_percent(g, expect_pct):
     saving = 100.0 * (1 - nbytes / (2 * rows * cols))
     assert saving == pytest.approx(expect_pct)
     assert abs(saving - 70.0) < 4.0          # "around 70 %"
+
+
+# ----------------------------------------------------------------------------------------
+def test_oracle_fp16_rounding_is_exact_rne():
+    """The oracle's own double -> fp16 rounding against exact rational rounding: halfway
+    points between neighbours (ties to even), values just off them, subnormals, the
+    smallest normal, and the overflow boundary (65520 = halfway between 65504 and 2^16)."""
+    from oracle import _lib
+    L = _lib.lib()
+    rng = np.random.default_rng(3)
+    vals = []
+    for bits in rng.integers(0, 0x7BFF, 300):        # finite fp16 values and their midpoints
+        a = float(np.uint16(bits).view(np.float16))
+        b = float(np.uint16(bits + 1).view(np.float16))
+        mid = (a + b) / 2
+        vals += [a, mid, np.nextafter(mid, 0.0), np.nextafter(mid, np.inf)]
+    vals += [2.0 ** -25, 3 * 2.0 ** -26, 2.0 ** -14, 2.0 ** -14 - 2.0 ** -25, 65504.0, 65519.99, 65520.0, 1e-30]
+    vals += list(rng.standard_normal(200) * 10.0 ** rng.integers(-6, 4, 200))
+    for v in vals:
+        for sv in (v, -v):
+            got = int(L.orc_d2h(sv))
+            if abs(sv) >= 65520.0:
+                assert got & 0x7FFF == 0x7C00
+                continue
+            exp = rn16(F(sv))
+            assert F(np.uint16(got).view(np.float16)) == exp, (sv, hex(got))
+            assert (got >> 15) == (1 if np.signbit(sv) else 0)
