@@ -369,7 +369,7 @@ struct GraphCache {
   bool seen = false, valid = false;
   cudaGraphExec_t prefill = nullptr, decode = nullptr;
   int64_t n_prefill = 0, n_decode = 0;
-  cudaStream_t cap = nullptr;
+  cudaStream_t cap[64] = {nullptr};  // capture stream of each device (created on first use there)
   // timing events the graphs record (captured while profiling was on)
   std::vector<ProfRec> prof_prefill, prof_decode;
 };
@@ -403,8 +403,7 @@ void collect_graph(const std::vector<ProfRec>& recs) {
 }
 
 template <class F>
-int capture_one(F&& seq, cudaGraphExec_t* exec, int64_t* n_launches, std::vector<ProfRec>* recs) {
-  cudaStream_t cs = g_graph.cap;
+int capture_one(F&& seq, cudaStream_t cs, cudaGraphExec_t* exec, int64_t* n_launches, std::vector<ProfRec>* recs) {
   const int64_t before = g_launches.load();
   size_t rec0 = 0;
   {
@@ -438,9 +437,13 @@ int capture_one(F&& seq, cudaGraphExec_t* exec, int64_t* n_launches, std::vector
 
 template <class P, class D>
 int capture_graphs(P&& prefill_seq, D&& decode_seq) {
-  if (!g_graph.cap) FG_CHECK_CUDA(cudaStreamCreateWithFlags(&g_graph.cap, cudaStreamNonBlocking));
-  FG_TRY(capture_one(prefill_seq, &g_graph.prefill, &g_graph.n_prefill, &g_graph.prof_prefill));
-  FG_TRY(capture_one(decode_seq, &g_graph.decode, &g_graph.n_decode, &g_graph.prof_decode));
+  int dev = 0;
+  FG_CHECK_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(FG_ERR_UNSUPPORTED, "device ordinal %d above 63", dev);
+  if (!g_graph.cap[dev]) FG_CHECK_CUDA(cudaStreamCreateWithFlags(&g_graph.cap[dev], cudaStreamNonBlocking));
+  const cudaStream_t cs = g_graph.cap[dev];
+  FG_TRY(capture_one(prefill_seq, cs, &g_graph.prefill, &g_graph.n_prefill, &g_graph.prof_prefill));
+  FG_TRY(capture_one(decode_seq, cs, &g_graph.decode, &g_graph.n_decode, &g_graph.prof_decode));
   g_graph.valid = true;
   return FG_OK;
 }

@@ -306,21 +306,13 @@ int prefill_attention_impl(const void* qkv, int B, int L, int nh, int hd, void* 
   if (!err) return fail(FG_ERR_CUDA, "device error flag unavailable");
   const dim3 grid((L + kTQ - 1) / kTQ, nh, B);
   if (hd == 128) {
-    static bool set = false;
-    if (!set) {
-      FG_CHECK_CUDA(cudaFuncSetAttribute(prefill_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         TcAttnCfg<128>::kSmem));
-      set = true;
-    }
+    static std::atomic<uint64_t> attr_done{0};
+    FG_TRY(ensure_smem_attr(prefill_attn_tc_kernel<128>, TcAttnCfg<128>::kSmem, attr_done));
     FG_LAUNCH("prefill attention kernel", prefill_attn_tc_kernel<128>, grid, dim3(TcAttnCfg<128>::kThreads), size_t(TcAttnCfg<128>::kSmem),
               s, tm, L, nh, reinterpret_cast<__half*>(out), err);
   } else {
-    static bool set = false;
-    if (!set) {
-      FG_CHECK_CUDA(cudaFuncSetAttribute(prefill_attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         TcAttnCfg<64>::kSmem));
-      set = true;
-    }
+    static std::atomic<uint64_t> attr_done{0};
+    FG_TRY(ensure_smem_attr(prefill_attn_tc_kernel<64>, TcAttnCfg<64>::kSmem, attr_done));
     FG_LAUNCH("prefill attention kernel", prefill_attn_tc_kernel<64>, grid, dim3(TcAttnCfg<64>::kThreads), size_t(TcAttnCfg<64>::kSmem),
               s, tm, L, nh, reinterpret_cast<__half*>(out), err);
   }

@@ -7,6 +7,8 @@
 #include <stdint.h>
 #include <stdio.h>
 
+#include <atomic>
+
 #include "../../include/fg.h"
 
 namespace fg {
@@ -73,6 +75,21 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
 int num_sms();
+
+// Raises a kernel's dynamic shared-memory limit once per device: the attribute belongs to
+// the device's context, so a process that drives several GPUs sets it on each of them.
+// `done` holds one bit per device ordinal (0..63).
+template <typename Kernel>
+int ensure_smem_attr(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  FG_CHECK_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(FG_ERR_UNSUPPORTED, "device ordinal %d above 63", dev);
+  const uint64_t bit = uint64_t(1) << dev;
+  if (done.load(std::memory_order_acquire) & bit) return FG_OK;
+  FG_CHECK_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  done.fetch_or(bit, std::memory_order_acq_rel);
+  return FG_OK;
+}
 
 // Row count from which a 4-bit GEMM expands its weight to fp16 once and runs the plain
 // fp16 tensor-core GEMM (measured break-even ~700 rows on B200).

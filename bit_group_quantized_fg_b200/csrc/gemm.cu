@@ -516,11 +516,8 @@ namespace {
 template <int MODE, bool F32>
 int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& p, const GemmArgs& args, cudaStream_t s) {
   using C = Cfg<MODE>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    FG_CHECK_CUDA(cudaFuncSetAttribute(gemm_tc_kernel<MODE, F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem));
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  FG_TRY(ensure_smem_attr(gemm_tc_kernel<MODE, F32>, C::kSmem, attr_done));
   const int grid = std::min(args.total, num_sms());
   FG_LAUNCH("tcgen05 gemm kernel", gemm_tc_kernel<MODE, F32>, dim3(grid), dim3(C::kThreads), size_t(C::kSmem), s, a, b, p, args);
   return FG_OK;

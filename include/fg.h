@@ -193,17 +193,29 @@ int fg_decode_attention_noalloc(const void* q, int64_t q_stride, const fg_kv_cac
 int fg_prefill_attention(const void* qkv, int B, int L, int n_heads, int head_dim, void* out,
                          void* stream);
 
-/* LayerNorm over rows: y = (x - mean)/sqrt(var + 1e-5) * g + b, fp32 statistics, fp16 in/out. */
+/* LayerNorm over rows: y = (x - mean)/sqrt(var + 1e-5) * g + b, fp32 statistics (population
+ * variance), fp16 in/out.  The pages benchmark OPT-6.7B/30B/175B ("FlexGen" README mirror,
+ * benchmark table); the OPT block is pre-LayerNorm, which this call implements (eps 1e-5 is a
+ * reading: the pages give none).  x, y fp16 [rows][cols], g, b fp16 [cols]; cols % 8 == 0 and
+ * 16-byte aligned pointers (FG_ERR_SHAPE / FG_ERR_ALIGN). */
 int fg_layernorm(const void* x, int64_t rows, int cols, const void* g, const void* b, void* y,
                  void* stream);
 
-/* x[b*T + t] = fp16(E[ids[b*T+t]] + P[pos0 + t]) (one rounding). ids int32 [B][T]. */
+/* Token + learned position embedding of the OPT decoders the pages benchmark ("FlexGen" README
+ * mirror, benchmark table): x[b*T + t] = fp16(E[ids[b*T+t]] + P[pos0 + t]) with one rounding of
+ * the exact sum.  Positions start at 0 for the prompt with no offset (a reading).  ids device
+ * int32 [B][T] (each in [0, vocab): not checked, the caller's contract); E fp16 [vocab][hidden],
+ * P fp16 [max_pos][hidden] with pos0 + T <= max_pos; out fp16 [B*T][hidden]; hidden % 8 == 0. */
 int fg_embed(const int32_t* ids, int B, int T, int pos0, const void* E, const void* P,
              int hidden, void* out, void* stream);
 
 /* Tied LM head + greedy argmax: tokens[b] = argmax_v (x[b] . E[v]) over v < vocab, ties to
- * the lowest id; x fp16 [B][hidden] (already final-LayerNormed); logits fp32 [B][vocab]
- * are written when `logits` is not NULL.  Needs fg_lm_head_workspace_bytes. */
+ * the lowest id.  Greedy decoding of the generated tokens the "FlexGen" README mirror's
+ * benchmark counts (output length 32); the head is the fp16 embedding itself, not
+ * compressed, and ties go to the lowest id (readings).  x fp16 [B][hidden] (already
+ * final-LayerNormed); E fp16 [vocab][hidden]; logits fp32 [B][vocab] are written when
+ * `logits` is not NULL, otherwise the workspace (fg_lm_head_workspace_bytes) holds them;
+ * tokens device int32 [B].  hidden % 64 == 0 (FG_ERR_SHAPE). */
 size_t fg_lm_head_workspace_bytes(int B, int vocab);
 int fg_lm_head_argmax(const void* x, int B, int hidden, const void* E, int vocab, float* logits,
                       int32_t* tokens, void* workspace, size_t ws_bytes, void* stream);
@@ -212,8 +224,14 @@ int fg_lm_head_argmax(const void* x, int B, int hidden, const void* E, int vocab
  * Layers and generation.
  * ---------------------------------------------------------------------------------- */
 
-/* One decoder block for one new token per sequence: x_out = block(x_in), both fp16 [B][h].
- * Appends the token's K/V at cache->len (then attends over 0..len) and advances len.
+/* One decoder block for one new token per sequence, the step the decode phase repeats
+ * ("FlexGen" README mirror: generation time is part of the throughput metric; key features:
+ * weights and attention cache in 4 bits): x_out = block(x_in), both fp16 [B][h]:
+ *   h1 = LN1(x_in); qkv = h1 W_qkv + b; append k, v (4-bit) at cache->len; attention of q over
+ *   positions 0..len (the new one included); x1 = x_in + att W_o + b_o;
+ *   x_out = x1 + relu(LN2(x1) W_1 + b_1) W_2 + b_2.
+ * Advances cache->len.  x_out may alias x_in.  FG_ERR_CAPACITY when the cache is full,
+ * FG_ERR_SHAPE when B != cache->B or a weight's shape does not match h and ffn.
  * workspace >= fg_decode_layer_workspace_bytes(h, ffn, n_heads, B, cache->capacity). */
 size_t fg_decode_layer_workspace_bytes(int hidden, int ffn, int n_heads, int B, int capacity);
 int fg_decode_layer(const fg_layer* layer, fg_kv_cache* cache, const void* x_in, void* x_out,

@@ -167,3 +167,24 @@ def test_lm_head_argmax(fg):
     tok2 = fg.fg_lm_head_argmax(to_dev(x[:1]), to_dev(E2))
     torch.cuda.synchronize()
     assert int(to_np(tok2)[0]) == 123
+
+
+def test_two_devices_in_one_process(fg):
+    """Launch state kept per device (shared-memory attributes, capture streams): a GEMM on
+    device 0 and then on device 1 of the same process both match the oracle.  Skipped with a
+    single visible GPU."""
+    import torch
+    if torch.cuda.device_count() < 2:
+        pytest.skip("needs two visible GPUs")
+    M, N, K, g = 64, 1024, 512, 64
+    x = fg_synth.tensor(31, 1, (M, K), "normal", 1.0)
+    w = fg_synth.tensor(31, 2, (K, N), "normal", 0.02)
+    b = fg_synth.tensor(31, 3, (N,), "normal", 0.5)
+    exp = oracle.qlinear(x, oracle.QLinear.from_fp16(w, b, g))
+    for d in (0, 1):
+        with torch.cuda.device(d):
+            dev = torch.device("cuda", d)
+            lin = fg.DeviceQLinear.from_fp16(torch.from_numpy(w).to(dev), torch.from_numpy(b).to(dev), g)
+            y = fg.fg_qgemm(torch.from_numpy(x).to(dev), lin)
+            torch.cuda.synchronize(d)
+            assert_close_rms(to_np(y), exp, what=f"GEMM on device {d}")
