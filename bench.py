@@ -608,12 +608,35 @@ def run_generate(args, fg, torch, dev, stream, world, rank, barrier):
     from fg_synth import gpu as sg
     import fg_synth
     c = CFG
-    model, caches = build_model(fg, torch, dev, args.weights)
+    offload = args.weights == "offload"
+    model, caches = build_model(fg, torch, dev, "4bit" if offload else args.weights)
     B, L, T = c["batch"], c["prompt_len"], c["gen_len"]
     ids = torch.empty((B, L), dtype=torch.int32, device=dev)
     sg.fill_ids(ids, replica_seed(rank), fg_synth.S_IDS, c["vocab"])
     out = torch.empty((B, T), dtype=torch.int32, device=dev)
-    ws = torch.empty((fg.fg_workspace_bytes(model, B, L, T),), dtype=torch.uint8, device=dev)
+    h2d_weights = [0.0]
+    if offload:
+        # every layer's 4-bit weights to pinned host memory; the device copies are freed
+        mc = model.c
+        host_layers = []
+        for i in range(len(model.layers)):
+            host_layers.append(fg.pinned_layer(model.layers[i]))
+            model.layers[i] = None
+        E, P, g1, b1 = model.tensors
+        model = fg.DeviceModel(mc.n_layers, mc.hidden, mc.n_heads, mc.head_dim, mc.ffn, mc.vocab, mc.max_pos,
+                               mc.group, E, P, g1, b1, host_layers)
+        torch.cuda.empty_cache()
+        ws = torch.empty((fg.fg_offload_workspace_bytes(model, B, L, T),), dtype=torch.uint8, device=dev)
+
+        def generate():
+            o, tm, hb = fg.fg_generate_offload(model, ids, T, caches, out_ids=out, workspace=ws)
+            h2d_weights[0] = hb
+            return o, tm
+    else:
+        ws = torch.empty((fg.fg_workspace_bytes(model, B, L, T),), dtype=torch.uint8, device=dev)
+
+        def generate():
+            return fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
     torch.cuda.synchronize()
 
     # The roofline kernel (the prompt-pass GEMM) is timed by CUDA events from the warm-up on:
@@ -624,7 +647,7 @@ def run_generate(args, fg, torch, dev, stream, world, rank, barrier):
     fg.fg_profile_select([0])
     fg.fg_profile_enable(True)
     for _ in range(args.warmup):
-        fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
+        generate()
     # ---- timed region: device-resident inputs
     fg.fg_profile_reset()
     launches0 = fg.fg_launch_count()
@@ -634,7 +657,7 @@ def run_generate(args, fg, torch, dev, stream, world, rank, barrier):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.steps):
-            _, tm = fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
+            _, tm = generate()
             timings.append((tm.prefill_ms, tm.decode_ms))
         e1.record(stream)
         barrier()
@@ -653,7 +676,7 @@ def run_generate(args, fg, torch, dev, stream, world, rank, barrier):
     e2.record(stream)
     for _ in range(e2e_steps):
         ids.copy_(ids_host, non_blocking=True)
-        fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
+        generate()
         out_host.copy_(out, non_blocking=True)
     e3.record(stream)
     barrier()
@@ -662,16 +685,16 @@ def run_generate(args, fg, torch, dev, stream, world, rank, barrier):
     # ---- per-kernel breakdown: every kernel class timed, one replayed step (not timed above)
     fg.fg_profile_select(None)
     for _ in range(2):   # eager, then captured with the new timing nodes
-        fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
+        generate()
     fg.fg_profile_reset()
-    fg.fg_generate(model, ids, T, caches, out_ids=out, workspace=ws)
+    generate()
     breakdown = {fg.PROF_NAMES[k]: fg.fg_profile_read(k) for k in range(7)}
     fg.fg_profile_enable(False)
     del model, caches, ws
     torch.cuda.empty_cache()
     return dict(ms_total=ms_total, ms_e2e=ms_e2e, e2e_steps=e2e_steps, timings=timings, prof=prof,
                 breakdown=breakdown, clocks=clocks, launches=launches,
-                h2d=B * L * 4, d2h=B * T * 4)
+                h2d=B * L * 4, d2h=B * T * 4, h2d_weights=h2d_weights[0])
 
 
 def run_slice(args, fg, torch, dev, stream, world, rank, barrier):
@@ -775,8 +798,9 @@ def main():
                     default="generate",
                     help="kernel-only cases sized for ncu captures (inputs larger than L2, a few GB at most)")
     ap.add_argument("--mnk", default="", help="M,N,K of the qgemm_decode case")
-    ap.add_argument("--weights", choices=["4bit", "fp16"], default="4bit",
-                    help="fp16: the same generation over uncompressed weights (compression contrast)")
+    ap.add_argument("--weights", choices=["4bit", "fp16", "offload"], default="4bit",
+                    help="fp16: the same generation over uncompressed weights (compression contrast); "
+                         "offload: 4-bit weights in pinned host memory, streamed layer by layer")
     args = ap.parse_args()
     if args.case == "sweep":
         return sweep_case(args)
@@ -784,7 +808,8 @@ def main():
         return kernel_case(args)
     c = use_config(args.config)
     world, rank, local = replica_env()
-    wdesc = "4-bit weights" if args.weights == "4bit" else "fp16 (uncompressed) weights"
+    wdesc = {"4bit": "4-bit weights", "fp16": "fp16 (uncompressed) weights",
+             "offload": "4-bit weights in pinned host memory (streamed per layer)"}[args.weights]
     config = {"workload": describe(c, wdesc), "name": args.config, "layers": c["n_layers"], "hidden": c["hidden"],
               "heads": f"{c['n_heads']}x{c['head_dim']}", "ffn": c["ffn"], "vocab": c["vocab"] or None,
               "global_batch": c["batch"] * max(world, args.gpus if world == 1 else world),
@@ -826,6 +851,8 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
 
+    if c["kind"] == "slice" and args.weights == "offload":
+        raise SystemExit("--weights offload runs a full decoder (c2 or c3)")
     runner = run_slice if c["kind"] == "slice" else run_generate
     r = runner(args, fg, torch, dev, stream, world, rank, barrier)
     B, L, T = c["batch"], c["prompt_len"], c["gen_len"]
@@ -913,7 +940,7 @@ def main():
         "prefill_ms": statistics.median(t[0] for t in r["timings"]),
         "decode_ms": statistics.median(t[1] for t in r["timings"]),
         "roofline": {"kernel": f"tcgen05 GEMM of the prompt pass (M = {M_pf}; " +
-                               ("4-bit weights expanded to fp16 once per layer)" if args.weights == "4bit"
+                               ("4-bit weights expanded to fp16 once per layer)" if args.weights != "fp16"
                                 else "uncompressed fp16 weights)"), "bound": "tensor",
                      "achieved": achieved_tf, "peak": pk["tf_sust"], "unit": "TFLOP/s",
                      "frac": achieved_tf / pk["tf_sust"], "traffic": traffic,
@@ -931,6 +958,11 @@ def main():
                 "d2h_bytes_per_step": r["d2h"], "steps": r["e2e_steps"]},
         "gpu_launches": r["launches"],
     }
+    if r.get("h2d_weights"):
+        per_step_s = ms_step * 1e-3
+        line["offload"] = {"weight_bytes_h2d_per_step": r["h2d_weights"],
+                           "host_link_GB/s": r["h2d_weights"] / per_step_s / 1e9,
+                           "note": "weights cross the host link once per pass (prompt pass + each decode step)"}
     if c["kind"] == "slice":
         line["slice"] = {"tokens_per_s_12_layers": slice_value, "per_layer_tokens_per_s": slice_value * c["n_layers"],
                          "extrapolation": f"value = slice tokens/s x {c['n_layers']}/{c['full_layers']} "

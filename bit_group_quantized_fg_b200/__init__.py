@@ -89,6 +89,9 @@ _SIGS = {
     "fg_workspace_bytes": (c_size_t, [POINTER(Model), c_int, c_int, c_int]),
     "fg_generate": (c_int, [POINTER(Model), c_void_p, c_int, c_int, c_int, c_void_p, POINTER(KVCache),
                             c_void_p, c_size_t, POINTER(Timing), c_void_p]),
+    "fg_offload_workspace_bytes": (c_size_t, [POINTER(Model), c_int, c_int, c_int]),
+    "fg_generate_offload": (c_int, [POINTER(Model), c_void_p, c_int, c_int, c_int, c_void_p, POINTER(KVCache),
+                                    c_void_p, c_size_t, POINTER(Timing), POINTER(c_double), c_void_p]),
     "fg_profile_enable": (c_int, [c_int]),
     "fg_profile_select": (c_int, [ctypes.c_uint]),
     "fg_profile_read": (c_int, [c_int, POINTER(c_double), POINTER(c_int64), POINTER(c_double),
@@ -367,6 +370,42 @@ def fg_generate(model: DeviceModel, prompt_ids, gen_len: int, caches, out_ids=No
         c.c.len = arr[i].len
     _check(st)
     return out_ids, timing
+
+
+def pinned_layer(layer: DeviceLayer) -> DeviceLayer:
+    """A copy of a layer whose tensors live in pinned host memory (for fg_generate_offload)."""
+    def pin(t):
+        return None if t is None else t.detach().cpu().pin_memory()
+
+    def lin(q: DeviceQLinear) -> DeviceQLinear:
+        return DeviceQLinear(pin(q.codes), pin(q.params), pin(q.bias), q.K, q.N, q.group, pin(q.w16))
+    return DeviceLayer(*[pin(t) for t in layer.t], lin(layer.qkv), lin(layer.out), lin(layer.fc1), lin(layer.fc2))
+
+
+def fg_offload_workspace_bytes(model: DeviceModel, B: int, L: int, gen_len: int) -> int:
+    return lib().fg_offload_workspace_bytes(ctypes.byref(model.c), B, L, gen_len)
+
+
+def fg_generate_offload(model: DeviceModel, prompt_ids, gen_len: int, caches, out_ids=None, workspace=None,
+                        stream=None):
+    """Greedy generation with the layers' weights in pinned host memory, streamed to the GPU
+    layer by layer; returns (out_ids int32 [B, gen_len] on the device, Timing, h2d bytes)."""
+    import torch
+    B, L = prompt_ids.shape
+    if out_ids is None:
+        out_ids = _empty((B, gen_len), torch.int32, prompt_ids.device)
+    if workspace is None:
+        workspace = _empty((fg_offload_workspace_bytes(model, B, L, gen_len),), torch.uint8, prompt_ids.device)
+    arr = (KVCache * len(caches))(*[c.c for c in caches])
+    timing = Timing()
+    h2d = c_double()
+    st = lib().fg_generate_offload(ctypes.byref(model.c), _ptr(prompt_ids), B, L, gen_len, _ptr(out_ids), arr,
+                                   _ptr(workspace), workspace.numel(), ctypes.byref(timing), ctypes.byref(h2d),
+                                   _stream(stream))
+    for i, c in enumerate(caches):
+        c.c.len = arr[i].len
+    _check(st)
+    return out_ids, timing, h2d.value
 
 
 def fg_profile_enable(on: bool = True):

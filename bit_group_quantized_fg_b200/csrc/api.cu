@@ -564,6 +564,285 @@ int generate_impl(const fg_model* m, const int32_t* ids, int B, int L, int T, in
   return st;
 }
 
+// ---------------------------------------------------------------- host-offloaded weights
+// Generation with every layer's 4-bit weights resident in pinned HOST memory ("FlexGen"
+// README mirror: offloading weights to CPU memory with the --percent policy and pinned weights,
+// and the block schedule that overlaps the loading of the next layer's weights with the
+// computation of the current one).  The block here is the whole batch: each layer's weights
+// cross the host link once per pass (the prompt pass, then each decode step) and serve every
+// sequence before the next layer runs.  Two weight slots in the workspace alternate: while the
+// compute stream runs layer c out of one slot, a copy stream fills the other slot with layer
+// c + 1, and the slot of layer c is refilled with layer c + 2 once layer c's kernels are done.
+namespace {
+
+struct LayerSpan {
+  size_t off[4][3];   // per linear: codes (or fp16 weight), params, bias
+  size_t bytes[4][3];
+  size_t ln_off[4];
+  size_t total;    // slot bytes (each tensor 256-byte aligned)
+  size_t payload;  // bytes copied per layer
+};
+
+size_t lin_bytes_codes(const fg_qlinear& w) {
+  return w.w16 ? size_t(w.K) * size_t(w.N) * 2 : size_t(w.K) * size_t(w.N) / 2;
+}
+size_t lin_bytes_params(const fg_qlinear& w) {
+  return w.w16 ? 0 : size_t(w.K) * size_t(w.N / w.group) * 4;
+}
+
+LayerSpan layer_span(const fg_layer& L, int h) {
+  LayerSpan sp{};
+  size_t t = 0;
+  const fg_qlinear* lins[4] = {&L.qkv, &L.out, &L.fc1, &L.fc2};
+  for (int i = 0; i < 4; ++i) {
+    const size_t b[3] = {lin_bytes_codes(*lins[i]), lin_bytes_params(*lins[i]),
+                         lins[i]->bias ? size_t(lins[i]->N) * 2 : 0};
+    for (int j = 0; j < 3; ++j) {
+      sp.off[i][j] = t;
+      sp.bytes[i][j] = b[j];
+      t += align256(b[j]);
+      sp.payload += b[j];
+    }
+  }
+  for (int j = 0; j < 4; ++j) {
+    sp.ln_off[j] = t;
+    t += align256(size_t(h) * 2);
+    sp.payload += size_t(h) * 2;
+  }
+  sp.total = t;
+  return sp;
+}
+
+bool is_host_memory(const void* p) {
+  if (!p) return true;
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeHost;
+}
+
+// The device-side layer whose pointers lie in a weight slot.
+fg_layer slot_layer(const fg_layer& H, const LayerSpan& sp, uint8_t* slot) {
+  fg_layer D = H;
+  fg_qlinear* lins[4] = {&D.qkv, &D.out, &D.fc1, &D.fc2};
+  for (int i = 0; i < 4; ++i) {
+    if (lins[i]->w16) {
+      lins[i]->w16 = slot + sp.off[i][0];
+    } else {
+      lins[i]->codes = slot + sp.off[i][0];
+      lins[i]->params = slot + sp.off[i][1];
+    }
+    if (lins[i]->bias) lins[i]->bias = slot + sp.off[i][2];
+  }
+  D.ln1_g = slot + sp.ln_off[0];
+  D.ln1_b = slot + sp.ln_off[1];
+  D.ln2_g = slot + sp.ln_off[2];
+  D.ln2_b = slot + sp.ln_off[3];
+  return D;
+}
+
+// One cudaMemcpyAsync per tensor of layer H into `slot` on stream cs.
+int copy_layer(const fg_layer& H, const LayerSpan& sp, uint8_t* slot, int h, cudaStream_t cs) {
+  const fg_qlinear* lins[4] = {&H.qkv, &H.out, &H.fc1, &H.fc2};
+  for (int i = 0; i < 4; ++i) {
+    const void* src[3] = {lins[i]->w16 ? lins[i]->w16 : static_cast<const void*>(lins[i]->codes), lins[i]->params,
+                          lins[i]->bias};
+    for (int j = 0; j < 3; ++j)
+      if (sp.bytes[i][j] && src[j])
+        FG_CHECK_CUDA(cudaMemcpyAsync(slot + sp.off[i][j], src[j], sp.bytes[i][j], cudaMemcpyHostToDevice, cs));
+  }
+  const void* ln[4] = {H.ln1_g, H.ln1_b, H.ln2_g, H.ln2_b};
+  for (int j = 0; j < 4; ++j)
+    FG_CHECK_CUDA(cudaMemcpyAsync(slot + sp.ln_off[j], ln[j], size_t(h) * 2, cudaMemcpyHostToDevice, cs));
+  return FG_OK;
+}
+
+cudaStream_t g_copy_stream[64] = {nullptr};
+std::mutex g_copy_mu;
+
+size_t offload_ws(const fg_model* m, int B, int L, int T) {
+  const LayerSpan sp = layer_span(m->layers[0], m->hidden);
+  return generate_ws(m, B, L, T) + 2 * align256(sp.total) + 256;
+}
+
+// The weight slots and the events of the double buffer for one generation.
+struct Offload {
+  const fg_model* m;
+  LayerSpan sp;
+  uint8_t* slot[2];
+  fg_layer dev[2];
+  cudaEvent_t loaded[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
+  cudaStream_t cs = nullptr;
+  int64_t visits = 0, issued = 0;  // layer visits of the whole generation, copies issued so far
+  double bytes = 0;
+
+  ~Offload() {
+    for (int i = 0; i < 2; ++i) {
+      if (loaded[i]) cudaEventDestroy(loaded[i]);
+      if (freed[i]) cudaEventDestroy(freed[i]);
+    }
+  }
+  // enqueue the copy of visit number `c` (layer c % n_layers) into slot c % 2
+  int issue(int64_t c) {
+    const int l = int(c % m->n_layers), k = int(c % 2);
+    if (c >= 2) FG_CHECK_CUDA(cudaStreamWaitEvent(cs, freed[k], 0));
+    FG_TRY(copy_layer(m->layers[l], sp, slot[k], m->hidden, cs));
+    FG_CHECK_CUDA(cudaEventRecord(loaded[k], cs));
+    bytes += double(sp.payload);
+    ++issued;
+    return FG_OK;
+  }
+  // the device layer of visit c, ready for the compute stream s
+  int acquire(int64_t c, cudaStream_t s, const fg_layer** out) {
+    const int k = int(c % 2);
+    FG_CHECK_CUDA(cudaStreamWaitEvent(s, loaded[k], 0));
+    *out = &dev[k];
+    return FG_OK;
+  }
+  // layer visit c is enqueued on s: its slot is refilled with visit c + 2 after it
+  int release(int64_t c, cudaStream_t s) {
+    FG_CHECK_CUDA(cudaEventRecord(freed[c % 2], s));
+    if (c + 2 < visits) FG_TRY(issue(c + 2));
+    return FG_OK;
+  }
+};
+
+}  // namespace
+
+int generate_offload_impl(const fg_model* m, const int32_t* ids, int B, int L, int T, int32_t* out,
+                          fg_kv_cache* caches, void* ws, size_t wsb, fg_timing* timing, double* h2d_bytes,
+                          cudaStream_t s) {
+  if (!m || !ids || !out || !caches) return fail(FG_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || L <= 0 || T <= 0) return fail(FG_ERR_SHAPE, "B, L and gen_len must be positive");
+  if (!m->embed || !m->pos_embed || !m->lnf_g || !m->lnf_b || !m->layers || m->n_layers <= 0)
+    return fail(FG_ERR_INVALID_ARG, "model tensors not set");
+  if (m->hidden != m->n_heads * m->head_dim) return fail(FG_ERR_SHAPE, "hidden != n_heads * head_dim");
+  if (L + T - 1 > m->max_pos) return fail(FG_ERR_SHAPE, "L + gen_len - 1 exceeds max_pos");
+  const int h = m->hidden;
+  const LayerSpan sp0 = layer_span(m->layers[0], h);
+  for (int l = 0; l < m->n_layers; ++l) {
+    int F = 0;
+    FG_TRY(check_layer(&m->layers[l], h, &F));
+    if (F != m->ffn) return fail(FG_ERR_SHAPE, "layer %d ffn %d != model ffn %d", l, F, m->ffn);
+    const fg_layer& H = m->layers[l];
+    const void* ptrs[] = {H.ln1_g, H.ln1_b, H.ln2_g, H.ln2_b, H.qkv.codes, H.qkv.params, H.qkv.bias, H.qkv.w16,
+                          H.out.codes, H.out.params, H.out.bias, H.out.w16, H.fc1.codes, H.fc1.params,
+                          H.fc1.bias, H.fc1.w16, H.fc2.codes, H.fc2.params, H.fc2.bias, H.fc2.w16};
+    for (const void* p : ptrs)
+      if (!is_host_memory(p))
+        return fail(FG_ERR_INVALID_ARG, "layer %d: offloaded weights must be pinned host memory", l);
+    const LayerSpan sp = layer_span(H, h);
+    if (sp.total != sp0.total || memcmp(sp.bytes, sp0.bytes, sizeof(sp.bytes)) != 0)
+      return fail(FG_ERR_SHAPE, "layer %d: every layer must have the same tensor sizes", l);
+    fg_kv_cache& c = caches[l];
+    if (c.B != B || c.n_heads != m->n_heads || c.head_dim != m->head_dim)
+      return fail(FG_ERR_SHAPE, "cache %d shape does not match the model", l);
+    if (c.capacity < L + T) return fail(FG_ERR_CAPACITY, "cache %d capacity %d < L + gen_len", l, c.capacity);
+  }
+  const size_t need = offload_ws(m, B, L, T);
+  if (!ws || wsb < need) return fail(FG_ERR_WORKSPACE, "offloaded generate needs %zu workspace bytes", need);
+
+  int dev = 0;
+  FG_CHECK_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(FG_ERR_UNSUPPORTED, "device ordinal %d above 63", dev);
+  {
+    std::lock_guard<std::mutex> lk(g_copy_mu);
+    if (!g_copy_stream[dev]) FG_CHECK_CUDA(cudaStreamCreateWithFlags(&g_copy_stream[dev], cudaStreamNonBlocking));
+  }
+  Carver c(ws, wsb);
+  void* x = c.take(size_t(B) * L * h * 2);
+  void* xd = c.take(size_t(B) * h * 2);
+  void* xn = c.take(size_t(B) * h * 2);
+  const size_t layer_b = std::max(prefill_ws(h, m->ffn, B, L), decode_ws(h, m->ffn, m->n_heads, B, L + T));
+  void* lws = c.take(layer_b);
+  void* lgw = c.take(lm_ws(B, m->vocab));
+  Offload off;
+  off.m = m;
+  off.sp = sp0;
+  off.cs = g_copy_stream[dev];
+  off.visits = int64_t(m->n_layers) * T;  // the prompt pass and T-1 decode steps
+  for (int k = 0; k < 2; ++k) {
+    off.slot[k] = reinterpret_cast<uint8_t*>(c.take(sp0.total));
+    off.dev[k] = slot_layer(m->layers[0], sp0, off.slot[k]);
+    FG_CHECK_CUDA(cudaEventCreateWithFlags(&off.loaded[k], cudaEventDisableTiming));
+    FG_CHECK_CUDA(cudaEventCreateWithFlags(&off.freed[k], cudaEventDisableTiming));
+  }
+  for (int l = 0; l < m->n_layers; ++l) caches[l].len = 0;
+
+  cudaEvent_t e0, e1, e2;
+  FG_CHECK_CUDA(cudaEventCreate(&e0));
+  FG_CHECK_CUDA(cudaEventCreate(&e1));
+  FG_CHECK_CUDA(cudaEventCreate(&e2));
+  int st = FG_OK;
+  int64_t visit = 0;
+  do {
+    cudaError_t ce = cudaEventRecord(e0, s);
+    if (ce != cudaSuccess) { st = cuda_fail(ce, "event"); break; }
+    // the copy stream starts after everything already queued on s (the caller's inputs)
+    if ((ce = cudaEventRecord(e1, s)) != cudaSuccess || (ce = cudaStreamWaitEvent(off.cs, e1, 0)) != cudaSuccess) {
+      st = cuda_fail(ce, "copy stream ordering");
+      break;
+    }
+    if ((st = off.issue(0)) != FG_OK) break;
+    if (off.visits > 1 && (st = off.issue(1)) != FG_OK) break;
+    // prompt pass, layer-major over the whole batch
+    if ((st = embed_impl(ids, B, L, L, 0, m->embed, m->pos_embed, h, x, s)) != FG_OK) break;
+    for (int l = 0; l < m->n_layers && st == FG_OK; ++l, ++visit) {
+      const fg_layer* ly = nullptr;
+      if ((st = off.acquire(visit, s, &ly)) != FG_OK) break;
+      if ((st = prefill_layer_impl(ly, &caches[l], x, B, L, lws, layer_b, s)) != FG_OK) break;
+      st = off.release(visit, s);
+    }
+    if (st != FG_OK) break;
+    ce = cudaMemcpy2DAsync(xd, size_t(h) * 2, reinterpret_cast<uint8_t*>(x) + size_t(L - 1) * h * 2,
+                           size_t(L) * h * 2, size_t(h) * 2, B, cudaMemcpyDeviceToDevice, s);
+    if (ce != cudaSuccess) { st = cuda_fail(ce, "last prompt rows"); break; }
+    if ((st = layernorm_impl(xd, B, h, m->lnf_g, m->lnf_b, xn, s)) != FG_OK) break;
+    if ((st = lm_head_impl(xn, B, h, m->embed, m->vocab, nullptr, out, T, lgw, lm_ws(B, m->vocab), s)) != FG_OK)
+      break;
+    cudaEventRecord(e1, s);
+    for (int j = 1; j < T && st == FG_OK; ++j) {
+      if ((st = embed_impl(out + (j - 1), B, 1, T, L + j - 1, m->embed, m->pos_embed, h, xd, s)) != FG_OK) break;
+      for (int l = 0; l < m->n_layers && st == FG_OK; ++l, ++visit) {
+        const fg_layer* ly = nullptr;
+        if ((st = off.acquire(visit, s, &ly)) != FG_OK) break;
+        if ((st = decode_layer_impl(ly, &caches[l], xd, xd, B, lws, layer_b, s)) != FG_OK) break;
+        st = off.release(visit, s);
+      }
+      if (st != FG_OK) break;
+      if ((st = layernorm_impl(xd, B, h, m->lnf_g, m->lnf_b, xn, s)) != FG_OK) break;
+      st = lm_head_impl(xn, B, h, m->embed, m->vocab, nullptr, out + j, T, lgw, lm_ws(B, m->vocab), s);
+    }
+    if (st != FG_OK) break;
+    cudaEventRecord(e2, s);
+    ce = cudaEventSynchronize(e2);
+    if (ce != cudaSuccess) { st = cuda_fail(ce, "offloaded generate"); break; }
+    int derr = 0;
+    if (read_device_error(&derr) == FG_OK && derr != 0) {
+      st = fail(FG_ERR_CUDA, "a device-side wait timed out (code %d)", derr);
+      break;
+    }
+    float pm = 0.f, dm = 0.f;
+    cudaEventElapsedTime(&pm, e0, e1);
+    cudaEventElapsedTime(&dm, e1, e2);
+    if (timing) {
+      timing->prefill_ms = pm;
+      timing->decode_ms = dm;
+      timing->tokens = int64_t(B) * T;
+      timing->tok_per_s = double(B) * T / ((double(pm) + double(dm)) * 1e-3);
+    }
+    if (h2d_bytes) *h2d_bytes = off.bytes;
+  } while (false);
+  // nothing of this call may still be copying when it returns (the slots are the caller's)
+  cudaStreamSynchronize(off.cs);
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  cudaEventDestroy(e2);
+  return st;
+}
+
 }  // namespace fg
 
 // ==================================================================== extern "C"
@@ -676,6 +955,18 @@ int fg_generate(const fg_model* model, const int32_t* prompt_ids, int B, int L, 
                 fg_kv_cache* caches, void* workspace, size_t ws_bytes, fg_timing* timing, void* stream) {
   return generate_impl(model, prompt_ids, B, L, gen_len, out_ids, caches, workspace, ws_bytes, timing,
                        as_stream(stream));
+}
+
+size_t fg_offload_workspace_bytes(const fg_model* model, int B, int L, int gen_len) {
+  if (!model || !model->layers || model->n_layers <= 0 || B <= 0 || L <= 0 || gen_len <= 0) return 0;
+  return offload_ws(model, B, L, gen_len);
+}
+
+int fg_generate_offload(const fg_model* model, const int32_t* prompt_ids, int B, int L, int gen_len,
+                        int32_t* out_ids, fg_kv_cache* caches, void* workspace, size_t ws_bytes, fg_timing* timing,
+                        double* h2d_bytes, void* stream) {
+  return generate_offload_impl(model, prompt_ids, B, L, gen_len, out_ids, caches, workspace, ws_bytes, timing,
+                               h2d_bytes, as_stream(stream));
 }
 
 int fg_profile_enable(int on) {

@@ -257,6 +257,27 @@ int fg_generate(const fg_model* model, const int32_t* prompt_ids, int B, int L, 
                 int32_t* out_ids, fg_kv_cache* caches, void* workspace, size_t ws_bytes,
                 fg_timing* timing, void* stream);
 
+/* Greedy generation with the layers' weights in pinned HOST memory ("FlexGen" README mirror:
+ * weights offloaded to CPU memory under the --percent placement policy with --pin-weight,
+ * and the block schedule that overlaps loading the next layer's weights with computing the
+ * current one).  Same arguments and results as fg_generate, except:
+ *  - model->layers[l]: every weight, bias and LayerNorm pointer is pinned host memory
+ *    (cudaHostAlloc / cudaHostRegister; FG_ERR_INVALID_ARG otherwise), all layers with the same
+ *    tensor sizes; embedding, positions and the final LayerNorm stay in device memory.
+ *  - Schedule: layer-major over the whole batch; two weight slots in the workspace alternate.
+ *    A copy stream owned by the library (one per device) fills the slot of layer visit c + 2
+ *    (one cudaMemcpyAsync per tensor) as soon as the kernels of visit c are done, so each
+ *    layer's weights cross the host link once per pass (prompt pass, then each decode step)
+ *    while the previous layer computes.
+ *  - Runs eagerly (no CUDA graphs); returns after the copy stream has drained.
+ *  - h2d_bytes (may be NULL) receives the weight bytes copied host -> device.
+ * workspace >= fg_offload_workspace_bytes(model, B, L, gen_len) (fg_workspace_bytes plus two
+ * weight slots). */
+size_t fg_offload_workspace_bytes(const fg_model* model, int B, int L, int gen_len);
+int fg_generate_offload(const fg_model* model, const int32_t* prompt_ids, int B, int L, int gen_len,
+                        int32_t* out_ids, fg_kv_cache* caches, void* workspace, size_t ws_bytes,
+                        fg_timing* timing, double* h2d_bytes, void* stream);
+
 /* Per-kernel device timing of the library's own launches (CUDA events on the launching
  * stream).  kind: 0 = dequant GEMM of a prompt pass (M > 256), 1 = decode attention,
  * 2 = prefill attention, 3 = quantize/append, 4 = other (LayerNorm, embedding, argmax),
