@@ -145,6 +145,27 @@ def test_gemm_f16_matches_oracle(fg, M, N, K):
     assert_close_rms(to_np(y), exp, what="fp16 GEMM")
 
 
+@pytest.mark.parametrize("M,N,K,relu,resid", [
+    (1024, 256, 64, False, False),     # one k-block, one column tile, four pair tiles
+    (1300, 768, 320, True, True),      # ragged rows: the last pair tile is mostly past M
+    (2176, 512, 2048, False, True),    # the last tile's second CTA holds no rows at all
+    (4096, 1024, 1024, True, False),   # two rasterization bands of 8 pair tiles
+])
+def test_gemm_f16_cta_pairs(fg, M, N, K, relu, resid):
+    """fp16 GEMMs with M >= 1024 run 256 x 256 tiles on CTA pairs (cta_group::2): against
+    the oracle's linear layer over the same fp16 weight."""
+    import torch
+    x = fg_synth.tensor(M + 1, 1, (M, K), "normal", 1.0)
+    w = fg_synth.tensor(M + 1, 2, (K, N), "normal", 0.02)
+    b = fg_synth.tensor(M + 1, 3, (N,), "normal", 0.5)
+    r = fg_synth.tensor(M + 1, 4, (M, N), "normal", 1.0) if resid else None
+    y = fg.fg_gemm_f16(to_dev(x), to_dev(w), bias=to_dev(b), R=None if r is None else to_dev(r), relu=relu)
+    torch.cuda.synchronize()
+    exp = oracle.qlinear(x, oracle.Linear16(w, b), relu=relu, residual16=r)
+    err, rms = assert_close_rms(to_np(y), exp, what="pair GEMM")
+    print(f"pair GEMM {M}x{N}x{K}: max|err| / RMS = {err / rms:.2e}")
+
+
 def test_lm_head_argmax(fg):
     import torch
     B, h, V = 5, 256, 1000      # V not a multiple of the 256-wide tile
