@@ -31,7 +31,7 @@ class FGError(RuntimeError):
 
 class QLinear(ctypes.Structure):
     _fields_ = [("codes", c_void_p), ("params", c_void_p), ("bias", c_void_p),
-                ("K", c_int), ("N", c_int), ("group", c_int), ("w16", c_void_p)]
+                ("K", c_int), ("N", c_int), ("group", c_int), ("w16", c_void_p), ("group_along_k", c_int)]
 
 
 class Layer(ctypes.Structure):
@@ -165,16 +165,18 @@ def fg_dequantize(codes, params, rows: int, cols: int, group: int = 64, axis: in
 class DeviceQLinear:
     """A 4-bit linear layer resident in HBM (keeps the tensors alive for the C struct)."""
 
-    def __init__(self, codes, params, bias, K: int, N: int, group: int = 64, w16=None):
+    def __init__(self, codes, params, bias, K: int, N: int, group: int = 64, w16=None, along_k: bool = False):
         self.codes, self.params, self.bias, self.w16 = codes, params, bias, w16
-        self.K, self.N, self.group = K, N, group
-        self.c = QLinear(_ptr(codes), _ptr(params), _ptr(bias), K, N, group, _ptr(w16))
+        self.K, self.N, self.group, self.along_k = K, N, group, along_k
+        self.c = QLinear(_ptr(codes), _ptr(params), _ptr(bias), K, N, group, _ptr(w16), int(along_k))
 
     @staticmethod
-    def from_fp16(w, bias, group: int = 64, stream=None) -> "DeviceQLinear":
+    def from_fp16(w, bias, group: int = 64, stream=None, along_k: bool = False) -> "DeviceQLinear":
+        """Quantize an fp16 weight [K][N] on the GPU: groups along N (output channel) by
+        default, along K (input dimension) with along_k."""
         K, N = w.shape
-        codes, params = fg_quantize_pack(w, group, 1, stream=stream)
-        return DeviceQLinear(codes, params, bias, K, N, group)
+        codes, params = fg_quantize_pack(w, group, 0 if along_k else 1, stream=stream)
+        return DeviceQLinear(codes, params, bias, K, N, group, along_k=along_k)
 
     @staticmethod
     def uncompressed(w, bias) -> "DeviceQLinear":
@@ -378,7 +380,7 @@ def pinned_layer(layer: DeviceLayer) -> DeviceLayer:
         return None if t is None else t.detach().cpu().pin_memory()
 
     def lin(q: DeviceQLinear) -> DeviceQLinear:
-        return DeviceQLinear(pin(q.codes), pin(q.params), pin(q.bias), q.K, q.N, q.group, pin(q.w16))
+        return DeviceQLinear(pin(q.codes), pin(q.params), pin(q.bias), q.K, q.N, q.group, pin(q.w16), q.along_k)
     return DeviceLayer(*[pin(t) for t in layer.t], lin(layer.qkv), lin(layer.out), lin(layer.fc1), lin(layer.fc2))
 
 

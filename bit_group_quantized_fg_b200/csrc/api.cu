@@ -191,12 +191,14 @@ int qlinear_run(const void* X, int64_t M, const fg_qlinear& w, const void* R, in
   if (w.w16)  // uncompressed weight: the fp16 GEMM over it directly
     return gemm_impl(1, X, M, w.N, w.K, w.w16, nullptr, 0, w.bias, R, relu, Y, false, ws, wsb, s, w_ready);
   const size_t wbytes = (size_t(w.K) * size_t(w.N) * 2 + 255) & ~size_t(255);
+  const int axis = w.group_along_k ? 0 : 1;
   if (M >= kExpandRows && ws != nullptr && wsb >= wbytes && aligned16(ws)) {
-    FG_TRY(dequantize_impl(w.codes, w.params, w.K, w.N, w.group, 1, ws, s));
+    FG_TRY(dequantize_impl(w.codes, w.params, w.K, w.N, w.group, axis, ws, s));
     return gemm_impl(1, X, M, w.N, w.K, ws, nullptr, 0, w.bias, R, relu, Y, false,
                      reinterpret_cast<uint8_t*>(ws) + wbytes, wsb - wbytes, s, false);  // weight just written
   }
-  return gemm_impl(0, X, M, w.N, w.K, w.codes, w.params, w.group, w.bias, R, relu, Y, false, ws, wsb, s, w_ready);
+  return gemm_impl(w.group_along_k ? 3 : 0, X, M, w.N, w.K, w.codes, w.params, w.group, w.bias, R, relu, Y, false, ws,
+                   wsb, s, w_ready);
 }
 
 size_t gemm_ws_for_layer(int64_t M, int h, int F) {

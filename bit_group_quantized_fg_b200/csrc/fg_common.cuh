@@ -155,4 +155,18 @@ __device__ __forceinline__ void dequant8_interleaved(uint32_t w, __half2 s2, __h
   }
 }
 
+// dequant8_interleaved with a {min, scale} of its own for each output pair: pair j holds
+// columns j and j + 4 of the word (weights grouped along K have one pair per column).
+__device__ __forceinline__ void dequant8_interleaved_pairs(uint32_t w, const __half2 (&s2)[4], const __half2 (&mn2)[4],
+                                                           uint32_t out[4]) {
+  const uint32_t MAGIC = 0x64006400u;
+  const __half2 K1024 = u32_as_h2(MAGIC);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t pair = ((w >> (4 * j)) & 0x000F000Fu) | MAGIC;
+    const __half2 q = __hsub2(u32_as_h2(pair), K1024);
+    out[j] = h2_as_u32(__hfma2(q, s2[j], mn2[j]));
+  }
+}
+
 }  // namespace fg

@@ -45,7 +45,9 @@ constexpr int kBBytes = BN * BK * 2;   // 32 KB
 constexpr int kCodeBytes = BK * BN / 2; // 8 KB
 constexpr int kParamBytesMax = BK * 8 * 4;  // up to 8 half2 per k row (G = 32)
 
-enum BMode { B_Q4 = 0, B_F16_MN = 1, B_F16_K = 2 };
+// B_Q4: 4-bit weight, groups along N (params [K][N/G]); B_Q4K: 4-bit weight, groups along K
+// (params [K/G][N]); B_F16_MN: fp16 [K][N]; B_F16_K: fp16 [N][K].
+enum BMode { B_Q4 = 0, B_F16_MN = 1, B_F16_K = 2, B_Q4K = 3 };
 
 // Shared memory: a ring of TMA stages, then (4-bit mode) a ring of expanded fp16 B tiles.
 // 4-bit mode: TMA stage = X tile + code tile + param tile (26 KB), 6 deep, so that the loads
@@ -53,7 +55,7 @@ enum BMode { B_Q4 = 0, B_F16_MN = 1, B_F16_K = 2 };
 // separate 2-deep ring of 32 KB fp16 B tiles.  fp16 modes: TMA stage = X tile + B tile, 4 deep.
 template <int MODE>
 struct Cfg {
-  static constexpr bool kQ4 = MODE == B_Q4;
+  static constexpr bool kQ4 = MODE == B_Q4 || MODE == B_Q4K;
   static constexpr int kStages = kQ4 ? 6 : 4;
   static constexpr int kCodeOff = kABytes;
   static constexpr int kParamOff = kABytes + kCodeBytes;
@@ -73,7 +75,8 @@ struct GemmArgs {
   int band;         // row tiles per rasterization band
   int prefetch_w;   // weight tiles may be requested before the previous kernel completes
   int total;        // m_tiles * n_tiles * splits
-  int G, PB;        // group size, params per k row in a stage
+  int G, PB;        // group size, params per k row in a stage (B_Q4)
+  int param_bytes;  // bytes of a stage's param tile
   const __half* bias;
   const __half* R;
   int relu;
@@ -147,7 +150,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
-    if (MODE == B_Q4) prefetch_tmap(&tm_p);
+    if (C::kQ4) prefetch_tmap(&tm_p);
   }
   if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
@@ -160,7 +163,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t tx = kABytes + (MODE == B_Q4 ? (kCodeBytes + BK * args.PB * 4) : kBBytes);
+      uint32_t tx = kABytes + (C::kQ4 ? (kCodeBytes + args.param_bytes) : kBBytes);
       bool ok = true;
       bool pend[S];
       uint32_t pend_phase[S];
@@ -172,6 +175,9 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
           tma_load_2d(st + C::kCodeOff, &tm_b, c.n0 / 2, kb * BK, bar);
           const int px = (c.n0 / args.G) & ~3;
           tma_load_2d(st + C::kParamOff, &tm_p, px, kb * BK, bar);
+        } else if (MODE == B_Q4K) {
+          tma_load_2d(st + C::kCodeOff, &tm_b, c.n0 / 2, kb * BK, bar);
+          tma_load_2d(st + C::kParamOff, &tm_p, c.n0, (kb * BK) / args.G, bar);
         } else if (MODE == B_F16_MN) {
 #pragma unroll
           for (int j = 0; j < BN / 64; ++j) tma_load_2d(st + kABytes + j * 8192, &tm_b, c.n0 + 64 * j, kb * BK, bar);
@@ -240,10 +246,10 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
         const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
         for (int kb = c.kb0; kb < c.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, &g_device_error, 4)) { ok = false; break; }
-          if (MODE == B_Q4 && !mbar_wait(&bfull[bs], bphase, abort_flag, &g_device_error, 8)) { ok = false; break; }
+          if (C::kQ4 && !mbar_wait(&bfull[bs], bphase, abort_flag, &g_device_error, 8)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + stage * C::kStageBytes);
-          const uint32_t b_addr = MODE == B_Q4 ? smem_u32(bring + bs * kBBytes) : a_addr + kABytes;
+          const uint32_t b_addr = C::kQ4 ? smem_u32(bring + bs * kBBytes) : a_addr + kABytes;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t ad = smem_desc_sw128(a_addr + k * 32, 16, 1024);
@@ -254,7 +260,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
           }
           mma_commit(&empty[stage]);
           if (++stage == S) { stage = 0; phase ^= 1; }
-          if (MODE == B_Q4) {
+          if (C::kQ4) {
             mma_commit(&bempty[bs]);
             if (++bs == SB) { bs = 0; bphase ^= 1; }
           }
@@ -284,7 +290,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
         uint32_t r[32];
         tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * BN + cc), r);
         tmem_ld_wait();
-        if (MODE == B_Q4) {
+        if (C::kQ4) {
           // the dequant warps stored each 8 columns in the order [0,4,1,5,2,6,3,7]:
           // natural column j of a group sits at position (j < 4 ? 2j : 2(j-4)+1)
           uint32_t t[32];
@@ -370,7 +376,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
-  } else if (MODE == B_Q4 && warp >= 8) {
+  } else if (C::kQ4 && warp >= 8) {
     // ------------------------------------------------------------ dequant warps
     constexpr int DW = C::kDequantWarps > 0 ? C::kDequantWarps : 1;
     constexpr int RPW = BK / DW;   // k rows per warp: dw, dw + DW, ...
@@ -389,18 +395,44 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
         const uint8_t* st = smem + stage * C::kStageBytes;
         const uint32_t* codes = reinterpret_cast<const uint32_t*>(st + C::kCodeOff);
         const uint32_t* prm = reinterpret_cast<const uint32_t*>(st + C::kParamOff);
-        uint32_t w[RPW], p[RPW];
-#pragma unroll
-        for (int i = 0; i < RPW; ++i) {
-          const int row = dw + DW * i;
-          w[i] = codes[row * (BN / 8) + lane];
-          p[i] = prm[row * args.PB + pcol];
-        }
+        uint32_t w[RPW];
         uint32_t o[RPW][4];
 #pragma unroll
-        for (int i = 0; i < RPW; ++i) {
-          const __half2 pr = u32_as_h2(p[i]);
-          dequant8_interleaved(w[i], __high2half2(pr), __low2half2(pr), o[i]);
+        for (int i = 0; i < RPW; ++i) w[i] = codes[(dw + DW * i) * (BN / 8) + lane];
+        if (MODE == B_Q4) {
+          uint32_t p[RPW];
+#pragma unroll
+          for (int i = 0; i < RPW; ++i) p[i] = prm[(dw + DW * i) * args.PB + pcol];
+#pragma unroll
+          for (int i = 0; i < RPW; ++i) {
+            const __half2 pr = u32_as_h2(p[i]);
+            dequant8_interleaved(w[i], __high2half2(pr), __low2half2(pr), o[i]);
+          }
+        } else {
+          // groups along K: one {min, scale} per column for each group of G rows; the rows of
+          // this k-block lie in one group (G >= 64) or two (G = 32: rows 0-31, 32-63)
+          // rows dw + 8i: i < 4 lie in rows 0-31, i >= 4 in rows 32-63 of the k-block
+          const bool two = args.G == 32;
+          const uint4* pp0 = reinterpret_cast<const uint4*>(prm + lane * 8);
+          const uint4* pp1 = reinterpret_cast<const uint4*>(prm + (two ? BN : 0) + lane * 8);
+          const uint4 a0 = pp0[0], b0 = pp0[1], a1 = pp1[0], b1 = pp1[1];  // columns +0..3, +4..7
+          __half2 s_lo[4], m_lo[4], s_hi[4], m_hi[4];
+          {
+            const uint32_t la[4] = {a0.x, a0.y, a0.z, a0.w}, ha[4] = {b0.x, b0.y, b0.z, b0.w};
+            const uint32_t lb[4] = {a1.x, a1.y, a1.z, a1.w}, hb[4] = {b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {   // pair j holds columns j and j + 4 (interleaved order)
+              m_lo[j] = u32_as_h2(__byte_perm(la[j], ha[j], 0x5410));
+              s_lo[j] = u32_as_h2(__byte_perm(la[j], ha[j], 0x7632));
+              m_hi[j] = u32_as_h2(__byte_perm(lb[j], hb[j], 0x5410));
+              s_hi[j] = u32_as_h2(__byte_perm(lb[j], hb[j], 0x7632));
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < RPW; ++i) {
+            if (i < RPW / 2) dequant8_interleaved_pairs(w[i], s_lo, m_lo, o[i]);
+            else dequant8_interleaved_pairs(w[i], s_hi, m_hi, o[i]);
+          }
         }
         // the B tile this k-block fills must have been consumed by the MMA two blocks ago
         if (!mbar_wait(&bempty[bs], bphase ^ 1, abort_flag, &g_device_error, 64)) { ok = false; break; }
@@ -581,7 +613,8 @@ size_t qgemm_ws_bytes(int64_t M, int N, int K) {
 int gemm_pair_launch(const void* X, int64_t M, int N, int K, const void* W, const void* bias, const void* R,
                      int relu, void* Y, cudaStream_t s);
 
-// mode: 0 = 4-bit weight W (codes/params), 1 = fp16 [K][N] weight, 2 = fp16 [N][K] weight.
+// mode: 0 = 4-bit weight W grouped along N, 1 = fp16 [K][N] weight, 2 = fp16 [N][K] weight,
+// 3 = 4-bit weight grouped along K.
 // An fp16 [K][N] weight with many rows (the prompt pass) runs on CTA pairs (gemm_pair.cu).
 int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, const void* wparams, int G,
               const void* bias, const void* R, int relu, void* Y, bool out_f32, void* ws, size_t ws_bytes,
@@ -590,11 +623,12 @@ int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, c
   if (M < 0 || N <= 0 || K <= 0) return fail(FG_ERR_SHAPE, "bad GEMM shape");
   if (K % BK) return fail(FG_ERR_SHAPE, "K must be a multiple of 64");
   if (M > 0x7fffff00LL) return fail(FG_ERR_SHAPE, "M too large");
-  if (mode == B_Q4) {
+  if (mode == B_Q4 || mode == B_Q4K) {
     if (!wparams) return fail(FG_ERR_INVALID_ARG, "null params");
     if (G != 32 && G != 64 && G != 128) return fail(FG_ERR_SHAPE, "group must be 32, 64 or 128");
     if (N % BN) return fail(FG_ERR_SHAPE, "N must be a multiple of 256");
-    if (N % (4 * G)) return fail(FG_ERR_SHAPE, "N must be a multiple of 4*group");
+    if (mode == B_Q4 && N % (4 * G)) return fail(FG_ERR_SHAPE, "N must be a multiple of 4*group");
+    if (mode == B_Q4K && K % G) return fail(FG_ERR_SHAPE, "K must be a multiple of the group (groups along K)");
   } else if (mode == B_F16_MN) {
     if (N % BN) return fail(FG_ERR_SHAPE, "N must be a multiple of 256");
   } else if (N % 8) {
@@ -621,6 +655,7 @@ int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, c
   a.total = a.m_tiles * a.n_tiles * a.splits;
   a.G = G;
   a.PB = G == 32 ? 8 : 4;
+  a.param_bytes = mode == B_Q4 ? BK * a.PB * 4 : (mode == B_Q4K ? std::max(1, BK / G) * BN * 4 : 0);
   a.bias = reinterpret_cast<const __half*>(bias);
   a.R = reinterpret_cast<const __half*>(R);
   a.relu = relu;
@@ -643,6 +678,11 @@ int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, c
                        BN / 2, BK, CU_TENSOR_MAP_SWIZZLE_NONE));
     FG_TRY(make_map_2d(&tp, wparams, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, uint64_t(N / G), uint64_t(K),
                        uint64_t(N / G) * 4, uint32_t(a.PB), BK, CU_TENSOR_MAP_SWIZZLE_NONE));
+  } else if (mode == B_Q4K) {
+    FG_TRY(make_map_2d(&tb, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(N / 2), uint64_t(K), uint64_t(N / 2),
+                       BN / 2, BK, CU_TENSOR_MAP_SWIZZLE_NONE));
+    FG_TRY(make_map_2d(&tp, wparams, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, uint64_t(N), uint64_t(K / G), uint64_t(N) * 4,
+                       BN, uint32_t(std::max(1, BK / G)), CU_TENSOR_MAP_SWIZZLE_NONE));
   } else if (mode == B_F16_MN) {
     FG_TRY(make_map_2d(&tb, w, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, uint64_t(N), uint64_t(K), uint64_t(N) * 2, 64, BK,
                        CU_TENSOR_MAP_SWIZZLE_128B));
@@ -650,10 +690,10 @@ int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, c
     FG_TRY(make_map_2d(&tb, w, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, uint64_t(K), uint64_t(N), uint64_t(K) * 2, BK, BN,
                        CU_TENSOR_MAP_SWIZZLE_128B));
   }
-  if (mode != B_Q4) tp = tb;
+  if (mode != B_Q4 && mode != B_Q4K) tp = tb;
 
   const double flops = 2.0 * double(M) * N * K;
-  const double bytes = (mode == B_Q4 ? double(N) * K * (0.5 + 4.0 / G) : double(N) * K * 2.0) +
+  const double bytes = (mode == B_Q4 || mode == B_Q4K ? double(N) * K * (0.5 + 4.0 / G) : double(N) * K * 2.0) +
                        double(M) * K * 2.0 + double(M) * N * (out_f32 ? 4.0 : 2.0) + (R ? double(M) * N * 2.0 : 0.0);
   {
     ProfScope ps(out_f32 ? PROF_LM_HEAD : (M > 256 ? PROF_GEMM : PROF_GEMM_DECODE), s, flops, bytes);
@@ -661,6 +701,7 @@ int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, c
     if (mode == B_F16_MN && !out_f32 && a.splits == 1 && M >= kPairRows)
       st = gemm_pair_launch(X, M, N, K, w, bias, R, relu, Y, s);   // 256 x 256 tiles on CTA pairs
     else if (mode == B_Q4) st = launch<B_Q4, false>(ta, tb, tp, a, s);
+    else if (mode == B_Q4K) st = launch<B_Q4K, false>(ta, tb, tp, a, s);
     else if (mode == B_F16_MN) st = launch<B_F16_MN, false>(ta, tb, tp, a, s);
     else st = out_f32 ? launch<B_F16_K, true>(ta, tb, tp, a, s) : launch<B_F16_K, false>(ta, tb, tp, a, s);
     if (st != FG_OK) return st;

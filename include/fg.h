@@ -77,9 +77,14 @@ int fg_dequantize(const uint8_t* codes, const void* params, int64_t rows, int64_
  * ---------------------------------------------------------------------------------- */
 
 /* A linear layer Y = X W + b whose weight W [K][N] (math convention, N contiguous) is
- * stored 4-bit with groups of `group` along N (the output channel):
- *   codes  uint8 [K][N/2], params half2 [K][N/group], bias fp16 [N] (may be NULL).
- * This is exactly fg_quantize_pack(W, K, N, group, axis=1).
+ * stored 4-bit in groups of `group` consecutive elements:
+ *   group_along_k == 0: groups along N (the output channel), the default:
+ *     codes uint8 [K][N/2], params half2 [K][N/group]  = fg_quantize_pack(W, K, N, group, 1)
+ *   group_along_k != 0: groups along K (the input dimension, one group per column):
+ *     codes uint8 [K][N/2], params half2 [K/group][N]  = fg_quantize_pack(W, K, N, group, 0)
+ *     (K % group == 0).  The pages fix neither axis; the README mirror's out-of-memory tips
+ *     fix only the storage, about 70 % below fp16, which both axes give.
+ * bias fp16 [N] (may be NULL).
  * w16: when not NULL the layer uses this uncompressed fp16 weight [K][N] instead (codes
  * and params are then ignored and may be NULL; N % 256 == 0).  The "FlexGen" README
  * mirror's benchmark table contrasts FlexGen with and without compression; this is the
@@ -90,6 +95,7 @@ typedef struct {
   const void* bias;
   int K, N, group;
   const void* w16;
+  int group_along_k;
 } fg_qlinear;
 
 /* One OPT decoder block (pre-LayerNorm, MHA, ReLU FFN).  qkv: [h][3h] with output

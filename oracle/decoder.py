@@ -63,18 +63,19 @@ class QLinear:
     K: int
     N: int
     group: int = 64
+    axis: int = 1               # 1: groups along N (output channel), 0: along K (input dim)
     _w16: Optional[np.ndarray] = field(default=None, repr=False)
 
     @staticmethod
-    def from_fp16(w16: np.ndarray, b16: np.ndarray, group: int = 64) -> "QLinear":
+    def from_fp16(w16: np.ndarray, b16: np.ndarray, group: int = 64, axis: int = 1) -> "QLinear":
         K, N = w16.shape
-        codes, params = quantize_pack(w16, group, axis=1)
-        return QLinear(codes, params, f16(b16), K, N, group)
+        codes, params = quantize_pack(w16, group, axis=axis)
+        return QLinear(codes, params, f16(b16), K, N, group, axis)
 
     def weight16(self) -> np.ndarray:
         """W_hat as fp16 [K, N] (the oracle's dequantization of the stored weight)."""
         if self._w16 is None:
-            self._w16 = dequantize(self.codes, self.params, self.K, self.N, self.group, 1)
+            self._w16 = dequantize(self.codes, self.params, self.K, self.N, self.group, self.axis)
         return self._w16
 
     def weight(self) -> np.ndarray:
@@ -84,6 +85,7 @@ class QLinear:
     def columns(self, cols) -> np.ndarray:
         """Dequantized columns ``cols`` only, float64 [K, len(cols)]; only the groups holding
         them are dequantized (for sampled checks of large weights)."""
+        assert self.axis == 1, "column sampling reads groups along N"
         cols = np.asarray(cols)
         g = self.group
         out = np.empty((self.K, len(cols)), np.float64)

@@ -166,6 +166,31 @@ def test_gemm_f16_cta_pairs(fg, M, N, K, relu, resid):
     print(f"pair GEMM {M}x{N}x{K}: max|err| / RMS = {err / rms:.2e}")
 
 
+@pytest.mark.parametrize("M,N,K,g,relu,resid", [
+    (64, 4096, 4096, 64, False, True),    # decode batch with the K loop split
+    (144, 768, 512, 32, True, False),     # G 32: two parameter rows per 64-deep k-block
+    (256, 512, 1024, 128, False, True),   # G 128: one parameter row serves two k-blocks
+    (1024, 512, 640, 64, True, True),     # prompt rows: expanded along K, then the pair GEMM
+])
+def test_qgemm_groups_along_k(fg, M, N, K, g, relu, resid):
+    """Weights grouped along K (the input dimension, one group per column): quantized
+    bit-exactly like the oracle's axis-0 quantizer, then the fused GEMM (decode rows) or the
+    expanded fp16 weight (prompt rows) against the oracle's linear layer."""
+    import torch
+    x = fg_synth.tensor(K + g, 1, (M, K), "normal", 1.0)
+    w = fg_synth.tensor(K + g, 2, (K, N), "outlier", 0.02)
+    b = fg_synth.tensor(K + g, 3, (N,), "normal", 0.5)
+    r = fg_synth.tensor(K + g, 4, (M, N), "normal", 1.0) if resid else None
+    lin = fg.DeviceQLinear.from_fp16(to_dev(w), to_dev(b), g, along_k=True)
+    ref = oracle.QLinear.from_fp16(w, b, g, axis=0)
+    assert np.array_equal(to_np(lin.codes), ref.codes)
+    assert np.array_equal(to_np(lin.params).view(np.uint16).reshape(-1), ref.params.view(np.uint16).reshape(-1))
+    y = fg.fg_qgemm(to_dev(x), lin, R=None if r is None else to_dev(r), relu=relu)
+    torch.cuda.synchronize()
+    err, rms = assert_close_rms(to_np(y), oracle.qlinear(x, ref, relu=relu, residual16=r), what="groups along K")
+    print(f"groups along K {M}x{N}x{K} g {g}: max|err| / RMS = {err / rms:.2e}")
+
+
 def test_lm_head_argmax(fg):
     import torch
     B, h, V = 5, 256, 1000      # V not a multiple of the 256-wide tile

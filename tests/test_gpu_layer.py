@@ -27,9 +27,10 @@ def fg():
     return m
 
 
-def make_layer(seed, l, h, F, g=64, wscale=0.02, ln_random=False, uncompressed=False):
+def make_layer(seed, l, h, F, g=64, wscale=0.02, ln_random=False, uncompressed=False, along_k=False):
     """Oracle and device copies of one decoder layer from seeded fp16 tensors (with
-    ``uncompressed`` the fp16 weights are used as they are, on both sides)."""
+    ``uncompressed`` the fp16 weights are used as they are, on both sides; with ``along_k``
+    the weights are grouped along their input dimension)."""
     def t(kind, shape, dist="normal", scale=wscale):
         return fg_synth.tensor(seed, ls(l, kind), shape, dist, scale)
     if ln_random:
@@ -43,17 +44,18 @@ def make_layer(seed, l, h, F, g=64, wscale=0.02, ln_random=False, uncompressed=F
     for wk, bk, K, N in ws:
         w = t(wk, (K, N))
         b = t(bk, (N,), scale=0.02)
-        o_lins.append(oracle.Linear16(w, b) if uncompressed else oracle.QLinear.from_fp16(w, b, g))
+        o_lins.append(oracle.Linear16(w, b) if uncompressed else
+                      oracle.QLinear.from_fp16(w, b, g, axis=0 if along_k else 1))
         d_lins.append((w, b, K, N))
     ol = oracle.QLayer(*ln, *o_lins)
     return ol, ln, d_lins
 
 
-def to_device_layer(fg, ln, d_lins, g=64, uncompressed=False):
+def to_device_layer(fg, ln, d_lins, g=64, uncompressed=False, along_k=False):
     if uncompressed:
         lins = [fg.DeviceQLinear.uncompressed(to_dev(w), to_dev(b)) for (w, b, K, N) in d_lins]
     else:
-        lins = [fg.DeviceQLinear.from_fp16(to_dev(w), to_dev(b), g) for (w, b, K, N) in d_lins]
+        lins = [fg.DeviceQLinear.from_fp16(to_dev(w), to_dev(b), g, along_k=along_k) for (w, b, K, N) in d_lins]
     return fg.DeviceLayer(*[to_dev(x) for x in ln], *lins)
 
 
@@ -86,14 +88,15 @@ def test_embed_exact(fg):
     assert np.array_equal(to_np(out).view(np.uint16), exp.view(np.uint16))
 
 
-@pytest.mark.parametrize("ln_random", [False, True])
-def test_config1_layer_prefill_then_decode(fg, ln_random):
+@pytest.mark.parametrize("ln_random,along_k", [(False, False), (True, False), (True, True)])
+def test_config1_layer_prefill_then_decode(fg, ln_random, along_k):
     """Config 1: OPT-125M-shaped layer (h 768, 12 x 64, F 3072), batch 4, prompt 32 hidden
-    states ~ N(0,1), then 4 decode steps with a 4-bit cache (group 64)."""
+    states ~ N(0,1), then 4 decode steps with a 4-bit cache (group 64); weights grouped along
+    the output channel, or along the input dimension."""
     import torch
     h, nh, hd, F, B, L, steps = 768, 12, 64, 3072, 4, 32, 4
-    ol, ln, d_lins = make_layer(1234, 0, h, F, ln_random=ln_random)
-    dl = to_device_layer(fg, ln, d_lins)
+    ol, ln, d_lins = make_layer(1234, 0, h, F, ln_random=ln_random, along_k=along_k)
+    dl = to_device_layer(fg, ln, d_lins, along_k=along_k)
     x = fg_synth.tensor(1234, fg_synth.S_HIDDEN, (B, L, h), "normal", 1.0)
     xd = to_dev(x.reshape(B * L, h))
     dcache = fg.DeviceKVCache(B, nh, hd, L + steps, 64)
