@@ -3,6 +3,7 @@ conversions and the float tolerance (max |err| <= 1e-2 * RMS(oracle output))."""
 import numpy as np
 
 import fg_synth
+import oracle
 
 TOL_RMS = 1e-2
 
@@ -63,34 +64,57 @@ def compare_free_running(got, exp_tokens, exp_logits):
     return agree, compared
 
 
-def gpu_teacher_forced(fg, md, ids, forced, group=64):
-    """GPU logits [T, B, V] at every position of a generation whose history is ``forced``
-    (the oracle's tokens [B, T]), through the layer calls: prompt pass, then decode step j
-    embeds forced[:, j-1] at position L + j - 1.  Every position is then scored on the same
-    history on both sides."""
+def stepwise_forced(fg, md, mo, ids, T, group=64):
+    """Every position scored from the same state on both sides.  The oracle generates greedily
+    step by step (its layer calls); the GPU runs the prompt pass itself, and before each decode
+    step j its caches are loaded with the oracle's 4-bit caches after step j-1 and it embeds
+    the oracle's token j-1.  Within a step both sides run their own layers, so the comparison
+    covers the embedding, every decode layer (KV append, attention over the cache, projections,
+    FFN), the final LayerNorm and the LM head, while a 4-bit code that one side rounds
+    differently (its K/V differ by an fp16 ulp) cannot carry over into later steps.
+    Returns (GPU logits [T, B, V], oracle tokens [B, T], oracle logits [T, B, V])."""
     import torch
     E, P, lnf_g, lnf_b = md.tensors
     B, L = ids.shape
-    T = forced.shape[1]
     V, h = E.shape
     nh, hd = md.c.n_heads, md.c.head_dim
-    caches = [fg.DeviceKVCache(B, nh, hd, L + T, group) for _ in md.layers]
+    n_layers = len(md.layers)
+    dc = [fg.DeviceKVCache(B, nh, hd, L + T, group) for _ in range(n_layers)]
+    oc = [oracle.KVCache(B, nh, hd, group, L + T) for _ in range(n_layers)]
+    g_logits = torch.empty((T, B, V), dtype=torch.float32, device=E.device)
+    o_tok = np.empty((B, T), np.int32)
+    o_logits = np.empty((T, B, V), np.float64)
+    # prompt pass
     x = fg.fg_embed(to_dev(np.ascontiguousarray(ids, np.int32)), 0, E, P)
-    for layer, c in zip(md.layers, caches):
+    for layer, c in zip(md.layers, dc):
         fg.fg_prefill_layer(layer, c, x, B, L)
-    logits = torch.empty((T, B, V), dtype=torch.float32, device=E.device)
     last = x.view(B, L, h)[:, L - 1, :].contiguous()
-    fg.fg_lm_head_argmax(fg.fg_layernorm(last, lnf_g, lnf_b), E, logits=logits[0])
+    fg.fg_lm_head_argmax(fg.fg_layernorm(last, lnf_g, lnf_b), E, logits=g_logits[0])
+    xo = oracle.embed(mo, ids, 0)
+    for layer, c in zip(mo.layers, oc):
+        xo = oracle.prefill_layer(layer, c, xo)
+    o_tok[:, 0], o_logits[0] = oracle.lm_head_argmax(mo, xo[:, -1, :])
     for j in range(1, T):
-        xd = fg.fg_embed(to_dev(np.ascontiguousarray(forced[:, j - 1:j], np.int32)), L + j - 1, E, P)
-        for layer, c in zip(md.layers, caches):
+        for d, o in zip(dc, oc):   # the oracle's cache state after step j-1
+            d.k_codes.copy_(torch.from_numpy(o.k_codes))
+            d.v_codes.copy_(torch.from_numpy(o.v_codes))
+            d.k_params.copy_(torch.from_numpy(o.k_params))
+            d.v_params.copy_(torch.from_numpy(o.v_params))
+            d.length = o.length
+        tok = np.ascontiguousarray(o_tok[:, j - 1:j])
+        xd = fg.fg_embed(to_dev(tok), L + j - 1, E, P)
+        for layer, c in zip(md.layers, dc):
             xd = fg.fg_decode_layer(layer, c, xd)
-        fg.fg_lm_head_argmax(fg.fg_layernorm(xd, lnf_g, lnf_b), E, logits=logits[j])
+        fg.fg_lm_head_argmax(fg.fg_layernorm(xd, lnf_g, lnf_b), E, logits=g_logits[j])
+        xo = oracle.embed(mo, tok, L + j - 1)[:, 0, :]
+        for layer, c in zip(mo.layers, oc):
+            xo = oracle.decode_layer(layer, c, xo)
+        o_tok[:, j], o_logits[j] = oracle.lm_head_argmax(mo, xo)
     torch.cuda.synchronize()
-    return to_np(logits).astype(np.float64)
+    return to_np(g_logits).astype(np.float64), o_tok, o_logits
 
 
-def check_teacher_forced(gpu_logits, exp_tokens, exp_logits, min_agree=0.99):
+def check_logits_and_tokens(gpu_logits, exp_tokens, exp_logits, min_agree=0.99):
     """Logits within the float tolerance at every position, and the GPU's argmax equal to the
     oracle's token at >= 99 % of all positions, every disagreement a near tie."""
     T, B, _ = gpu_logits.shape

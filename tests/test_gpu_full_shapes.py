@@ -13,7 +13,7 @@ import pytest
 import fg_synth
 import oracle
 from fg_synth import layer_stream as ls
-from gpu_util import assert_close_rms, check_teacher_forced, compare_free_running, gpu_teacher_forced, to_np
+from gpu_util import assert_close_rms, check_logits_and_tokens, compare_free_running, stepwise_forced, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -123,5 +123,7 @@ def test_generate_two_layer_opt6p7b_shape_graph_replay(fg):
     exp, logits = oracle.generate(mo, ids, T, return_logits=True)
     agree, compared = compare_free_running(calls[2], exp, logits)
     print(f"free-running replay: {agree}/{compared} compared positions agree")
-    frac = check_teacher_forced(gpu_teacher_forced(fg, md, ids, exp, g), exp, logits)
-    print(f"teacher-forced agreement {frac:.3f}")
+    g_lg, f_tok, f_lg = stepwise_forced(fg, md, mo, ids, T, g)
+    assert np.array_equal(f_tok, exp)
+    frac = check_logits_and_tokens(g_lg, f_tok, f_lg)
+    print(f"stepwise token agreement {frac:.3f}")

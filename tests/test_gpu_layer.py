@@ -1,18 +1,19 @@
 """GPU parity of LayerNorm, embedding, the decoder layer (prefill and decode) and greedy
 generation against the oracle.  Float outputs: max|err| <= 1e-2 * RMS(oracle).  Tokens:
-(1) teacher forcing through the layer calls (the GPU scores every position on the oracle's
-token history): logits within tolerance everywhere and the GPU's argmax equal to the
-oracle's token at >= 99 % of all positions, every disagreement a near tie (the oracle's
-top-2 margin within the float tolerance); (2) free-running fg_generate against the oracle's
-own generation: identical tokens up to the first near tie, after which the two
-continuations legitimately differ and are not compared."""
+(1) every position scored from the same state (gpu_util.stepwise_forced: before each decode
+step the GPU gets the oracle's token history and the oracle's 4-bit cache): logits within
+tolerance everywhere and the GPU's argmax equal to the oracle's token at >= 99 % of all
+positions, every disagreement a near tie (the oracle's top-2 margin within the float
+tolerance); (2) free-running fg_generate against the oracle's own generation: identical
+tokens up to the first near tie, after which the two continuations legitimately differ and
+are not compared."""
 import numpy as np
 import pytest
 
 import fg_synth
 import oracle
 from fg_synth import layer_stream as ls
-from gpu_util import (assert_close_rms, check_teacher_forced, compare_free_running, gpu_teacher_forced,
+from gpu_util import (assert_close_rms, check_logits_and_tokens, compare_free_running, stepwise_forced,
                       to_dev, to_np)
 
 pytestmark = pytest.mark.gpu
@@ -145,7 +146,9 @@ def test_generate_small_model(fg):
     assert compared >= B
     assert timing.tokens == B * T and timing.tok_per_s > 0
     assert all(c.length == L + T - 1 for c in caches)
-    check_teacher_forced(gpu_teacher_forced(fg, md, ids, exp), exp, logits)
+    g_lg, f_tok, f_lg = stepwise_forced(fg, md, mo, ids, T)
+    assert np.array_equal(f_tok, exp)          # the oracle's stepwise generation is its generate()
+    check_logits_and_tokens(g_lg, f_tok, f_lg)
     # rows are independent: a sub-batch generates the same tokens
     caches2 = [fg.DeviceKVCache(2, mo.n_heads, mo.head_dim, L + T, 64) for _ in range(mo.n_layers)]
     out2, _ = fg.fg_generate(md, to_dev(ids[[3, 1]]), T, caches2)
@@ -227,9 +230,12 @@ def test_uncompressed_weights_layer_and_generate(fg):
     assert_close_rms(to_np(yd), oracle.decode_layer(ol, oc, xd), what="uncompressed decode layer")
     mo, md = small_model(fg, seed=6, uncompressed=True)
     ids = fg_synth.token_ids(6, fg_synth.S_IDS, (4, 16), mo.vocab)
+    T = 8
     caches = [fg.DeviceKVCache(4, mo.n_heads, mo.head_dim, 24, 64) for _ in range(mo.n_layers)]
-    out, _ = fg.fg_generate(md, to_dev(ids), 8, caches)
+    out, _ = fg.fg_generate(md, to_dev(ids), T, caches)
     torch.cuda.synchronize()
-    exp, logits = oracle.generate(mo, ids, 8, return_logits=True)
+    exp, logits = oracle.generate(mo, ids, T, return_logits=True)
     compare_free_running(to_np(out), exp, logits)
-    check_teacher_forced(gpu_teacher_forced(fg, md, ids, exp), exp, logits)
+    g_lg, f_tok, f_lg = stepwise_forced(fg, md, mo, ids, T)
+    assert np.array_equal(f_tok, exp)          # the oracle's stepwise generation is its generate()
+    check_logits_and_tokens(g_lg, f_tok, f_lg)
