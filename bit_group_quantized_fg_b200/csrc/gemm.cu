@@ -610,12 +610,8 @@ size_t qgemm_ws_bytes(int64_t M, int N, int K) {
   return w + splitk_ws_bytes(M, N, K);
 }
 
-int gemm_pair_launch(const void* X, int64_t M, int N, int K, const void* W, const void* bias, const void* R,
-                     int relu, void* Y, cudaStream_t s);
-
 // mode: 0 = 4-bit weight W grouped along N, 1 = fp16 [K][N] weight, 2 = fp16 [N][K] weight,
 // 3 = 4-bit weight grouped along K.
-// An fp16 [K][N] weight with many rows (the prompt pass) runs on CTA pairs (gemm_pair.cu).
 int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, const void* wparams, int G,
               const void* bias, const void* R, int relu, void* Y, bool out_f32, void* ws, size_t ws_bytes,
               cudaStream_t s, bool w_ready) {
@@ -698,9 +694,7 @@ int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, c
   {
     ProfScope ps(out_f32 ? PROF_LM_HEAD : (M > 256 ? PROF_GEMM : PROF_GEMM_DECODE), s, flops, bytes);
     int st;
-    if (mode == B_F16_MN && !out_f32 && a.splits == 1 && M >= kPairRows)
-      st = gemm_pair_launch(X, M, N, K, w, bias, R, relu, Y, s);   // 256 x 256 tiles on CTA pairs
-    else if (mode == B_Q4) st = launch<B_Q4, false>(ta, tb, tp, a, s);
+    if (mode == B_Q4) st = launch<B_Q4, false>(ta, tb, tp, a, s);
     else if (mode == B_Q4K) st = launch<B_Q4K, false>(ta, tb, tp, a, s);
     else if (mode == B_F16_MN) st = launch<B_F16_MN, false>(ta, tb, tp, a, s);
     else st = out_f32 ? launch<B_F16_K, true>(ta, tb, tp, a, s) : launch<B_F16_K, false>(ta, tb, tp, a, s);

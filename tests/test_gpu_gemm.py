@@ -146,13 +146,13 @@ def test_gemm_f16_matches_oracle(fg, M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K,relu,resid", [
-    (1024, 256, 64, False, False),     # one k-block, one column tile, four pair tiles
-    (1300, 768, 320, True, True),      # ragged rows: the last pair tile is mostly past M
-    (2176, 512, 2048, False, True),    # the last tile's second CTA holds no rows at all
-    (4096, 1024, 1024, True, False),   # two rasterization bands of 8 pair tiles
+    (1024, 256, 64, False, False),     # one k-block, one column tile, eight row tiles
+    (1300, 768, 320, True, True),      # ragged rows: the last row tile is mostly past M
+    (2176, 512, 2048, False, True),    # a second band with one row tile
+    (4096, 1024, 1024, True, False),   # two rasterization bands of 16 row tiles
 ])
-def test_gemm_f16_cta_pairs(fg, M, N, K, relu, resid):
-    """fp16 GEMMs with M >= 1024 run 256 x 256 tiles on CTA pairs (cta_group::2): against
+def test_gemm_f16_prompt_rows(fg, M, N, K, relu, resid):
+    """fp16 GEMMs at prompt-pass row counts (ragged rows, several rasterization bands) against
     the oracle's linear layer over the same fp16 weight."""
     import torch
     x = fg_synth.tensor(M + 1, 1, (M, K), "normal", 1.0)
@@ -162,8 +162,8 @@ def test_gemm_f16_cta_pairs(fg, M, N, K, relu, resid):
     y = fg.fg_gemm_f16(to_dev(x), to_dev(w), bias=to_dev(b), R=None if r is None else to_dev(r), relu=relu)
     torch.cuda.synchronize()
     exp = oracle.qlinear(x, oracle.Linear16(w, b), relu=relu, residual16=r)
-    err, rms = assert_close_rms(to_np(y), exp, what="pair GEMM")
-    print(f"pair GEMM {M}x{N}x{K}: max|err| / RMS = {err / rms:.2e}")
+    err, rms = assert_close_rms(to_np(y), exp, what="prompt-row GEMM")
+    print(f"fp16 GEMM {M}x{N}x{K}: max|err| / RMS = {err / rms:.2e}")
 
 
 @pytest.mark.parametrize("M,N,K,g,relu,resid", [

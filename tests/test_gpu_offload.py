@@ -10,7 +10,7 @@ import pytest
 
 import fg_synth
 import oracle
-from gpu_util import check_teacher_forced, compare_free_running, gpu_teacher_forced, to_dev, to_np
+from gpu_util import compare_free_running, to_dev, to_np
 from test_gpu_layer import small_model
 
 pytestmark = pytest.mark.gpu
