@@ -27,7 +27,7 @@ int argmax_impl(const float*, int, int, int32_t*, int64_t, cudaStream_t);
 size_t qgemm_ws_bytes(int64_t, int, int);
 size_t splitk_ws_bytes(int64_t, int, int);
 int gemm_impl(int, const void*, int64_t, int, int, const void*, const void*, int, const void*, const void*, int,
-              void*, bool, void*, size_t, cudaStream_t, bool);
+              void*, bool, void*, size_t, cudaStream_t, bool, LnFuse* = nullptr);
 int read_device_error(int*);
 
 // ---------------------------------------------------------------- errors
@@ -186,10 +186,13 @@ int check_layer(const fg_layer* L, int h, int* ffn) {
 // w_ready: the weight was not written by the kernel just before this one in the stream
 // (true inside the layer calls, whose first kernel is a LayerNorm), so its tiles may be
 // requested before the previous kernel finishes.
+// ln: a LayerNorm of Y's rows to fuse into the GEMM's split-K reduction (decode batches);
+// ln->done tells the caller whether it still has to run it.
 int qlinear_run(const void* X, int64_t M, const fg_qlinear& w, const void* R, int relu, void* Y, void* ws,
-                size_t wsb, cudaStream_t s, bool w_ready = false) {
+                size_t wsb, cudaStream_t s, bool w_ready = false, LnFuse* ln = nullptr) {
+  if (ln) ln->done = false;
   if (w.w16)  // uncompressed weight: the fp16 GEMM over it directly
-    return gemm_impl(1, X, M, w.N, w.K, w.w16, nullptr, 0, w.bias, R, relu, Y, false, ws, wsb, s, w_ready);
+    return gemm_impl(1, X, M, w.N, w.K, w.w16, nullptr, 0, w.bias, R, relu, Y, false, ws, wsb, s, w_ready, ln);
   const size_t wbytes = (size_t(w.K) * size_t(w.N) * 2 + 255) & ~size_t(255);
   const int axis = w.group_along_k ? 0 : 1;
   if (M >= kExpandRows && ws != nullptr && wsb >= wbytes && aligned16(ws)) {
@@ -198,7 +201,7 @@ int qlinear_run(const void* X, int64_t M, const fg_qlinear& w, const void* R, in
                      reinterpret_cast<uint8_t*>(ws) + wbytes, wsb - wbytes, s, false);  // weight just written
   }
   return gemm_impl(w.group_along_k ? 3 : 0, X, M, w.N, w.K, w.codes, w.params, w.group, w.bias, R, relu, Y, false, ws,
-                   wsb, s, w_ready);
+                   wsb, s, w_ready, ln);
 }
 
 size_t gemm_ws_for_layer(int64_t M, int h, int F) {
@@ -230,8 +233,11 @@ size_t prefill_ws(int h, int F, int B, int L) {
 }
 }  // namespace
 
+// h1_in: LN1(x_in) already computed (fused into the previous block's fc2 reduction), or NULL.
+// next: the LayerNorm that follows this block (the next block's LN1, or the final LN) to fuse
+// into fc2's split-K reduction; next->done reports whether it was.
 int decode_layer_impl(const fg_layer* layer, fg_kv_cache* cache, const void* x_in, void* x_out, int B, void* ws,
-                      size_t ws_bytes, cudaStream_t s) {
+                      size_t ws_bytes, cudaStream_t s, const void* h1_in = nullptr, LnFuse* next = nullptr) {
   if (!cache || !x_in || !x_out) return fail(FG_ERR_INVALID_ARG, "null pointer");
   if (B <= 0 || B != cache->B) return fail(FG_ERR_SHAPE, "B must equal the cache batch");
   const int h = cache->n_heads * cache->head_dim;
@@ -253,14 +259,16 @@ int decode_layer_impl(const fg_layer* layer, fg_kv_cache* cache, const void* x_i
   void* aws = c.take(aws_b);
   auto* qkvh = reinterpret_cast<__half*>(qkv);
 
-  FG_TRY(layernorm_impl(x_in, B, h, layer->ln1_g, layer->ln1_b, h1, s));
+  if (h1_in) h1 = const_cast<void*>(h1_in);
+  else FG_TRY(layernorm_impl(x_in, B, h, layer->ln1_g, layer->ln1_b, h1, s));
   FG_TRY(qlinear_run(h1, B, layer->qkv, nullptr, 0, qkv, gws, gws_b, s, true));
   FG_TRY(kv_append_impl(cache, qkvh + h, qkvh + 2 * h, 3 * int64_t(h), 1, s));
   FG_TRY(decode_attention_impl(qkv, 3 * int64_t(h), cache, att, aws, aws_b, s));
-  FG_TRY(qlinear_run(att, B, layer->out, x_in, 0, x1, gws, gws_b, s, true));
-  FG_TRY(layernorm_impl(x1, B, h, layer->ln2_g, layer->ln2_b, h2, s));
+  LnFuse ln2{layer->ln2_g, layer->ln2_b, h2, false};   // LN2 in the out-projection's reduction
+  FG_TRY(qlinear_run(att, B, layer->out, x_in, 0, x1, gws, gws_b, s, true, &ln2));
+  if (!ln2.done) FG_TRY(layernorm_impl(x1, B, h, layer->ln2_g, layer->ln2_b, h2, s));
   FG_TRY(qlinear_run(h2, B, layer->fc1, nullptr, 1, f, gws, gws_b, s, true));
-  FG_TRY(qlinear_run(f, B, layer->fc2, x1, 0, x_out, gws, gws_b, s, true));
+  FG_TRY(qlinear_run(f, B, layer->fc2, x1, 0, x_out, gws, gws_b, s, true, next));
   return FG_OK;
 }
 
@@ -318,7 +326,7 @@ size_t generate_ws(const fg_model* m, int B, int L, int T) {
   const int h = m->hidden, F = m->ffn;
   size_t t = 0;
   t += align256(size_t(B) * L * h * 2);                 // x (prompt hidden states)
-  t += align256(size_t(B) * h * 2) * 2;                 // decode x, final LN out
+  t += align256(size_t(B) * h * 2) * 3;                 // decode x, final LN out, next block's LN1
   size_t layer = std::max(prefill_ws(h, F, B, L), decode_ws(h, F, m->n_heads, B, L + T));
   t += align256(layer);
   t += lm_ws(B, m->vocab);
@@ -472,12 +480,15 @@ int generate_impl(const fg_model* m, const int32_t* ids, int B, int L, int T, in
   void* x = c.take(size_t(B) * L * h * 2);
   void* xd = c.take(size_t(B) * h * 2);
   void* xn = c.take(size_t(B) * h * 2);
+  void* hn = c.take(size_t(B) * h * 2);   // LN1 of the next block, from the previous block's fc2
   const size_t layer_b = std::max(prefill_ws(h, m->ffn, B, L), decode_ws(h, m->ffn, m->n_heads, B, L + T));
   void* lws = c.take(layer_b);
   void* lgw = c.take(lm_ws(B, m->vocab));
 
   // The two launch sequences of a generation (prompt pass; decode steps).  They run directly
-  // on `s`, or on the capture stream while a CUDA graph is recorded.
+  // on `s`, or on the capture stream while a CUDA graph is recorded.  In a decode step each
+  // block's fc2 reduction also applies the LayerNorm that follows it (the next block's LN1,
+  // or the final LayerNorm before the LM head) whenever that GEMM splits K.
   auto prefill_seq = [&](cudaStream_t st_) -> int {
     for (int l = 0; l < m->n_layers; ++l) caches[l].len = 0;
     FG_TRY(embed_impl(ids, B, L, L, 0, m->embed, m->pos_embed, h, x, st_));
@@ -492,8 +503,15 @@ int generate_impl(const fg_model* m, const int32_t* ids, int B, int L, int T, in
     for (int j = 1; j < T; ++j) {
       // token j-1 sits at position L + j - 1
       FG_TRY(embed_impl(out + (j - 1), B, 1, T, L + j - 1, m->embed, m->pos_embed, h, xd, st_));
-      for (int l = 0; l < m->n_layers; ++l) FG_TRY(decode_layer_impl(&m->layers[l], &caches[l], xd, xd, B, lws, layer_b, st_));
-      FG_TRY(layernorm_impl(xd, B, h, m->lnf_g, m->lnf_b, xn, st_));
+      const void* h1 = nullptr;
+      for (int l = 0; l < m->n_layers; ++l) {
+        const bool last = l + 1 == m->n_layers;
+        LnFuse nx{last ? m->lnf_g : m->layers[l + 1].ln1_g, last ? m->lnf_b : m->layers[l + 1].ln1_b,
+                  last ? xn : hn, false};
+        FG_TRY(decode_layer_impl(&m->layers[l], &caches[l], xd, xd, B, lws, layer_b, st_, h1, &nx));
+        if (!nx.done) FG_TRY(layernorm_impl(xd, B, h, nx.g, nx.b, nx.H, st_));
+        h1 = last ? nullptr : hn;
+      }
       FG_TRY(lm_head_impl(xn, B, h, m->embed, m->vocab, nullptr, out + j, T, lgw, lm_ws(B, m->vocab), st_, true));
     }
     return FG_OK;
@@ -757,6 +775,8 @@ int generate_offload_impl(const fg_model* m, const int32_t* ids, int B, int L, i
   void* x = c.take(size_t(B) * L * h * 2);
   void* xd = c.take(size_t(B) * h * 2);
   void* xn = c.take(size_t(B) * h * 2);
+  c.take(size_t(B) * h * 2);  // (the resident path's next-LN1 buffer; unused here: the next
+                              // layer's LayerNorm parameters may still be on their way)
   const size_t layer_b = std::max(prefill_ws(h, m->ffn, B, L), decode_ws(h, m->ffn, m->n_heads, B, L + T));
   void* lws = c.take(layer_b);
   void* lgw = c.take(lm_ws(B, m->vocab));

@@ -98,6 +98,15 @@ constexpr int64_t kExpandRows = 1024;
 // Device address of the flag that bounded device-side waits set when they give up.
 int* device_error_ptr();
 
+// A LayerNorm of a GEMM's output rows to fuse into its split-K reduction when there is one
+// (H = LN(Y) with gamma g, beta b); `done` reports whether it was fused.
+struct LnFuse {
+  const void* g;
+  const void* b;
+  void* H;
+  bool done;
+};
+
 int splitk_reduce_launch(const float* P, int splits, int64_t M, int N, const void* bias, const void* R, int relu,
                          void* Y, cudaStream_t s);
 

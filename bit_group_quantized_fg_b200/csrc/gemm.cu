@@ -512,6 +512,119 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ P, int splits, in
   }
 }
 
+// Split-K reduction + epilogue + LayerNorm of the row, for a GEMM whose output row feeds a
+// LayerNorm (the out-projection's residual sum x1 -> LN2, fc2's -> the next block's LN1):
+// one CTA per row reduces the partials, adds bias and residual, stores the fp16 row Y, and
+// normalizes the stored fp16 values: H = fp16((y - mean) / sqrt(var + 1e-5) * g + b), fp32
+// two-pass statistics, population variance (the same definition as the LayerNorm kernel).
+// CPT = 8-column chunks per thread (N <= 256 * 8 * CPT).
+template <int CPT>
+__global__ void __launch_bounds__(256) splitk_reduce_ln_kernel(const float* __restrict__ P, int splits, int M, int N,
+                                                               const __half* __restrict__ bias,
+                                                               const __half* __restrict__ R, __half* __restrict__ Y,
+                                                               const __half* __restrict__ g,
+                                                               const __half* __restrict__ b, __half* __restrict__ H) {
+  pdl_wait();  // the previous kernel in the stream has finished (see fg_launch)
+  __shared__ float red[8];
+  const int row = blockIdx.x;
+  const int chunks = N / 8;
+  const int64_t MN = int64_t(M) * N;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto block_sum = [&](float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    __syncthreads();  // earlier readers of red[] are done
+    if (lane == 0) red[warp] = x;
+    __syncthreads();
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += red[w];
+    return t;
+  };
+  float v[CPT][8];
+  float sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    const int c = threadIdx.x + i * 256;
+    if (c >= chunks) continue;
+    const int64_t e = int64_t(row) * N + int64_t(c) * 8;
+    const float4* p0 = reinterpret_cast<const float4*>(P + e);
+    float4 a = p0[0], bb = p0[1];
+    float t[8] = {a.x, a.y, a.z, a.w, bb.x, bb.y, bb.z, bb.w};
+    for (int sp = 1; sp < splits; ++sp) {
+      const float4* ps = reinterpret_cast<const float4*>(P + sp * MN + e);
+      a = ps[0];
+      bb = ps[1];
+      t[0] += a.x; t[1] += a.y; t[2] += a.z; t[3] += a.w; t[4] += bb.x; t[5] += bb.y; t[6] += bb.z; t[7] += bb.w;
+    }
+    if (bias) {
+      const uint4 bw = __ldg(reinterpret_cast<const uint4*>(bias + int64_t(c) * 8));
+      const __half2* bh = reinterpret_cast<const __half2*>(&bw);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __half22float2(bh[k]);
+        t[2 * k] += f.x;
+        t[2 * k + 1] += f.y;
+      }
+    }
+    if (R) {
+      const uint4 rw = __ldg(reinterpret_cast<const uint4*>(R + e));
+      const __half2* rh = reinterpret_cast<const __half2*>(&rw);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __half22float2(rh[k]);
+        t[2 * k] += f.x;
+        t[2 * k + 1] += f.y;
+      }
+    }
+    uint4 o;
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const __half2 hv = __floats2half2_rn(t[2 * k], t[2 * k + 1]);
+      ow[k] = h2_as_u32(hv);
+      const float2 f = __half22float2(hv);  // the stored fp16 values are what LayerNorm reads
+      v[i][2 * k] = f.x;
+      v[i][2 * k + 1] = f.y;
+      sum += f.x + f.y;
+    }
+    *reinterpret_cast<uint4*>(Y + e) = o;
+  }
+  const float mean = block_sum(sum) / float(N);
+  float sq = 0.f;
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    const int c = threadIdx.x + i * 256;
+    if (c >= chunks) continue;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float d = v[i][k] - mean;
+      sq = fmaf(d, d, sq);
+    }
+  }
+  const float var = block_sum(sq) / float(N);
+  const float rstd = 1.0f / sqrtf(var + 1e-5f);
+#pragma unroll
+  for (int i = 0; i < CPT; ++i) {
+    const int c = threadIdx.x + i * 256;
+    if (c >= chunks) continue;
+    const uint4 gw = __ldg(reinterpret_cast<const uint4*>(g + int64_t(c) * 8));
+    const uint4 bw = __ldg(reinterpret_cast<const uint4*>(b + int64_t(c) * 8));
+    const __half2* gh = reinterpret_cast<const __half2*>(&gw);
+    const __half2* bh = reinterpret_cast<const __half2*>(&bw);
+    uint4 o;
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 gg = __half22float2(gh[k]), be = __half22float2(bh[k]);
+      const float y0 = fmaf((v[i][2 * k] - mean) * rstd, gg.x, be.x);
+      const float y1 = fmaf((v[i][2 * k + 1] - mean) * rstd, gg.y, be.y);
+      ow[k] = h2_as_u32(__floats2half2_rn(y0, y1));
+    }
+    *reinterpret_cast<uint4*>(H + int64_t(row) * N + int64_t(c) * 8) = o;
+  }
+}
+
 // ---------------------------------------------------------------- host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -574,6 +687,22 @@ int splitk_reduce_launch(const float* P, int splits, int64_t M, int N, const voi
   return FG_OK;
 }
 
+// One CTA per row: reduce + epilogue + LayerNorm (see splitk_reduce_ln_kernel).
+int splitk_reduce_ln_launch(const float* P, int splits, int64_t M, int N, const void* bias, const void* R, void* Y,
+                            const void* g, const void* b, void* H, cudaStream_t s) {
+  const int cpt = (N / 8 + 255) / 256;
+  using K = void (*)(const float*, int, int, int, const __half*, const __half*, __half*, const __half*,
+                     const __half*, __half*);
+  static const K table[6] = {splitk_reduce_ln_kernel<1>, splitk_reduce_ln_kernel<2>, splitk_reduce_ln_kernel<3>,
+                             splitk_reduce_ln_kernel<4>, splitk_reduce_ln_kernel<5>, splitk_reduce_ln_kernel<6>};
+  if (cpt < 1 || cpt > 6) return fail(FG_ERR_UNSUPPORTED, "fused LayerNorm supports rows of up to 12288");
+  FG_LAUNCH("split-K reduce + LayerNorm kernel", table[cpt - 1], dim3(unsigned(M)), dim3(256), size_t(0), s, P, splits,
+            int(M), N, reinterpret_cast<const __half*>(bias), reinterpret_cast<const __half*>(R),
+            reinterpret_cast<__half*>(Y), reinterpret_cast<const __half*>(g), reinterpret_cast<const __half*>(b),
+            reinterpret_cast<__half*>(H));
+  return FG_OK;
+}
+
 int read_device_error(int* out) {
   return cudaMemcpyFromSymbol(out, g_device_error, sizeof(int)) == cudaSuccess ? FG_OK : FG_ERR_CUDA;
 }
@@ -614,7 +743,8 @@ size_t qgemm_ws_bytes(int64_t M, int N, int K) {
 // 3 = 4-bit weight grouped along K.
 int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, const void* wparams, int G,
               const void* bias, const void* R, int relu, void* Y, bool out_f32, void* ws, size_t ws_bytes,
-              cudaStream_t s, bool w_ready) {
+              cudaStream_t s, bool w_ready, LnFuse* ln) {
+  if (ln) ln->done = false;
   if (!X || !w || !Y) return fail(FG_ERR_INVALID_ARG, "null pointer");
   if (M < 0 || N <= 0 || K <= 0) return fail(FG_ERR_SHAPE, "bad GEMM shape");
   if (K % BK) return fail(FG_ERR_SHAPE, "K must be a multiple of 64");
@@ -699,8 +829,17 @@ int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, c
     else if (mode == B_F16_MN) st = launch<B_F16_MN, false>(ta, tb, tp, a, s);
     else st = out_f32 ? launch<B_F16_K, true>(ta, tb, tp, a, s) : launch<B_F16_K, false>(ta, tb, tp, a, s);
     if (st != FG_OK) return st;
+    // the split-K reduction (and a fused LayerNorm) is timed with its GEMM
+    if (a.splits > 1) {
+      if (ln && ln->g && ln->b && ln->H && !relu && N % 8 == 0 && N <= 12288 && aligned16(ln->g) &&
+          aligned16(ln->b) && aligned16(ln->H)) {
+        FG_TRY(splitk_reduce_ln_launch(a.partial, a.splits, M, N, a.bias, a.R, Y, ln->g, ln->b, ln->H, s));
+        ln->done = true;
+      } else {
+        FG_TRY(splitk_reduce_launch(a.partial, a.splits, M, N, a.bias, a.R, relu, Y, s));
+      }
+    }
   }
-  if (a.splits > 1) FG_TRY(splitk_reduce_launch(a.partial, a.splits, M, N, a.bias, a.R, relu, Y, s));
   return FG_OK;
 }
 
