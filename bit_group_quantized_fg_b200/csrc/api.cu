@@ -19,7 +19,8 @@ int quantize_pack_impl(const void*, int64_t, int64_t, int, int, uint8_t*, void*,
 int dequantize_impl(const uint8_t*, const void*, int64_t, int64_t, int, int, void*, cudaStream_t);
 int kv_append_impl(fg_kv_cache*, const void*, const void*, int64_t, int, cudaStream_t);
 size_t decode_attention_ws_bytes(int, int, int, int);
-int decode_attention_impl(const void*, int64_t, const fg_kv_cache*, void*, void*, size_t, cudaStream_t);
+int decode_attention_impl(const void*, int64_t, const fg_kv_cache*, void*, void*, size_t, cudaStream_t,
+                          const void* = nullptr, const void* = nullptr, int64_t = 0, fg_kv_cache* = nullptr);
 int prefill_attention_impl(const void*, int, int, int, int, void*, cudaStream_t);
 int layernorm_impl(const void*, int64_t, int, const void*, const void*, void*, cudaStream_t);
 int embed_impl(const int32_t*, int64_t, int, int, int, const void*, const void*, int, void*, cudaStream_t);
@@ -262,8 +263,9 @@ int decode_layer_impl(const fg_layer* layer, fg_kv_cache* cache, const void* x_i
   if (h1_in) h1 = const_cast<void*>(h1_in);
   else FG_TRY(layernorm_impl(x_in, B, h, layer->ln1_g, layer->ln1_b, h1, s));
   FG_TRY(qlinear_run(h1, B, layer->qkv, nullptr, 0, qkv, gws, gws_b, s, true));
-  FG_TRY(kv_append_impl(cache, qkvh + h, qkvh + 2 * h, 3 * int64_t(h), 1, s));
-  FG_TRY(decode_attention_impl(qkv, 3 * int64_t(h), cache, att, aws, aws_b, s));
+  // the step's K/V append runs inside the attention kernel (the last-chunk CTA of each head)
+  FG_TRY(decode_attention_impl(qkv, 3 * int64_t(h), cache, att, aws, aws_b, s, qkvh + h, qkvh + 2 * h,
+                               3 * int64_t(h), cache));
   LnFuse ln2{layer->ln2_g, layer->ln2_b, h2, false};   // LN2 in the out-projection's reduction
   FG_TRY(qlinear_run(att, B, layer->out, x_in, 0, x1, gws, gws_b, s, true, &ln2));
   if (!ln2.done) FG_TRY(layernorm_impl(x1, B, h, layer->ln2_g, layer->ln2_b, h2, s));

@@ -18,11 +18,14 @@
 #include <mutex>
 
 #include "fg_common.cuh"
+#include "quant_common.cuh"
 
 namespace fg {
 namespace {
 
 constexpr int kWarps = 2;
+// Blocks of positions whose loads a warp keeps in flight ahead of the one it computes on.
+constexpr int kAhead = 2;
 constexpr int kThreads = kWarps * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -82,17 +85,25 @@ struct AttnMma {
   static constexpr int TB = 16;        // positions per block
 };
 
+// Fused append (the decode step's KV append): when `knew` is not NULL, position S - 1 is the
+// step's new token, whose K and V rows (knew/vnew + b * new_stride, fp16) are not yet in the
+// cache.  The CTA of each (sequence, head) that owns the last chunk quantizes them with the
+// same group quantizer as the append kernel (warp 0: K, warp 1: V), stores codes and params
+// at position S - 1, and attends over that position from shared memory (no other CTA reads it).
 template <int HD, int G>
 __global__ void __launch_bounds__(kThreads) decode_attn_mma_kernel(
     const __half* __restrict__ q, int64_t q_stride, const uint8_t* __restrict__ kc,
     const __half2* __restrict__ kp, const uint8_t* __restrict__ vc, const __half2* __restrict__ vp,
     int nh, int cap, int S, int chunk_len, __half* __restrict__ out, float* __restrict__ part_ml,
-    float* __restrict__ part_acc) {
+    float* __restrict__ part_acc, const __half* knew, const __half* vnew, int64_t new_stride, uint8_t* kc_w,
+    __half2* kp_w, uint8_t* vc_w, __half2* vp_w) {
   pdl_wait();  // the previous kernel in the stream has finished (see fg_launch)
   using C = AttnMma<HD, G>;
   constexpr int NG = C::NG, KW = C::KW, KS = C::KS, MT = C::MT, DPT = C::DPT, VW = C::VW, TB = C::TB;
   __shared__ float red_v[kWarps][HD];
   __shared__ float red_ml[kWarps][2];
+  __shared__ uint32_t new_codes[2][HD / 8];  // the new token's K / V code words
+  __shared__ uint32_t new_par[2][NG];        // and {min, scale} pairs
 
   const int b = blockIdx.z, head = blockIdx.y, chunk = blockIdx.x;
   const int t0 = chunk * chunk_len;
@@ -100,6 +111,32 @@ __global__ void __launch_bounds__(kThreads) decode_attn_mma_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, q4 = lane & 3;
   const __half* qh = q + int64_t(b) * q_stride + head * HD;
+  const bool app = knew != nullptr && chunk == int(gridDim.x) - 1;
+  const int tnew = S - 1;
+  if (app) {
+    static_assert(kWarps == 2, "one warp quantizes K, the other V");
+    constexpr int TPG = G / 16;  // lanes per group (16 values per lane)
+    const __half* src = (warp == 0 ? knew : vnew) + int64_t(b) * new_stride + head * HD;
+    uint4 xa = make_uint4(0, 0, 0, 0), xb = xa;
+    if (lane < HD / 16) {
+      xa = *reinterpret_cast<const uint4*>(src + lane * 16);
+      xb = *reinterpret_cast<const uint4*>(src + lane * 16 + 8);
+    }
+    const GroupQ r = quantize_chunk16<TPG>(xa, xb);  // every lane takes part in the shuffles
+    if (lane < HD / 16) {
+      const int64_t slot = (int64_t(b) * nh + head) * cap + tnew;
+      uint8_t* cw = warp == 0 ? kc_w : vc_w;
+      __half2* pw = warp == 0 ? kp_w : vp_w;
+      *reinterpret_cast<uint2*>(cw + slot * (HD / 2) + lane * 8) = r.words;
+      new_codes[warp][2 * lane] = r.words.x;
+      new_codes[warp][2 * lane + 1] = r.words.y;
+      if (lane % TPG == 0) {
+        pw[slot * NG + lane / TPG] = r.params;
+        new_par[warp][lane / TPG] = h2_as_u32(r.params);
+      }
+    }
+    __syncthreads();
+  }
 
   // ---- query: B fragments of the score MMA, and per-group O_n, Q_n
   uint32_t qb[KS][2];
@@ -158,7 +195,8 @@ __global__ void __launch_bounds__(kThreads) decode_attn_mma_kernel(
   };
   auto load = [&](Blk& o, int blk) {
     const int tA = blk + g, tB = blk + g + 8;
-    const bool okA = tA < t1, okB = tB < t1;
+    // the new token's position is taken from shared memory below, not loaded
+    const bool okA = tA < t1 && !(app && tA == tnew), okB = tB < t1 && !(app && tB == tnew);
     if (KW == 4) {
       const uint4 za = okA ? ldg_v4(reinterpret_cast<const uint4*>(kbase + int64_t(tA) * (HD / 2)) + q4)
                            : make_uint4(0, 0, 0, 0);
@@ -177,7 +215,7 @@ __global__ void __launch_bounds__(kThreads) decode_attn_mma_kernel(
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const int t = blk + 2 * q4 + (r & 1) + (r >> 1) * 8;
-      const bool ok = t < t1;
+      const bool ok = t < t1 && !(app && t == tnew);
       const uint32_t* src = reinterpret_cast<const uint32_t*>(vbase + int64_t(t) * (HD / 2)) + VW * g;
       if (VW == 2) {
         const uint2 z = ok ? __ldg(reinterpret_cast<const uint2*>(src)) : make_uint2(0, 0);
@@ -197,13 +235,43 @@ __global__ void __launch_bounds__(kThreads) decode_attn_mma_kernel(
     }
     o.vpA = (q4 < NG && okA) ? __ldg(vpu + int64_t(tA) * NG + q4) : 0u;
     o.vpB = (q4 < NG && okB) ? __ldg(vpu + int64_t(tB) * NG + q4) : 0u;
+    if (app && tnew >= blk && tnew < blk + TB) {
+      const bool pA = tA == tnew, pB = tB == tnew;
+      if (pA || pB) {
+#pragma unroll
+        for (int i = 0; i < KW; ++i) {
+          const uint32_t w = new_codes[0][KW * q4 + i];
+          if (pA) o.kA[i] = w;
+          if (pB) o.kB[i] = w;
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int n = 2 * q4 + j;
+          const uint32_t pk = n < NG ? new_par[0][n < NG ? n : 0] : 0u;
+          if (pA) o.kpA[j] = pk;
+          if (pB) o.kpB[j] = pk;
+        }
+        const uint32_t pv = q4 < NG ? new_par[1][q4 < NG ? q4 : 0] : 0u;
+        if (pA) o.vpA = pv;
+        if (pB) o.vpB = pv;
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        if (blk + 2 * q4 + (r & 1) + (r >> 1) * 8 == tnew) {
+#pragma unroll
+          for (int w = 0; w < VW; ++w) o.vw[r][w] = new_codes[1][VW * g + w];
+        }
+      }
+    }
   };
 
-  Blk cur;
+  Blk cur, nx1;
   load(cur, t0 + warp * TB);
+  if (kAhead > 1) load(nx1, t0 + warp * TB + kWarps * TB);
   for (int blk = t0 + warp * TB; blk < t1; blk += kWarps * TB) {
     Blk nxt;
-    load(nxt, blk + kWarps * TB);  // next block's loads in flight while this one computes
+    // the loads of the next kAhead blocks are in flight while this one computes
+    load(nxt, blk + kAhead * kWarps * TB);
     const int tA = blk + g, tB = blk + g + 8;
     const bool okA = tA < t1, okB = tB < t1;
     const uint32_t(&kA)[KW] = cur.kA;
@@ -296,7 +364,12 @@ __global__ void __launch_bounds__(kThreads) decode_attn_mma_kernel(
       const uint32_t a2 = ((r23 << 4) & 0x00F000F0u) | 0x54005400u, a3 = (r23 & 0x00F000F0u) | 0x54005400u;
       mma16816(acc[mt], a0, a1, a2, a3, b0, b1);
     }
-    cur = nxt;
+    if (kAhead > 1) {
+      cur = nx1;
+      nx1 = nxt;
+    } else {
+      cur = nxt;
+    }
   }
 
   // ---- finish the warp: sums over rows, then out_d for the dims this lane holds
@@ -418,10 +491,20 @@ size_t decode_attention_ws_bytes(int B, int nh, int hd, int ctx) {
   return size_t(B) * nh * nc * (2 + hd) * sizeof(float) + 256;
 }
 
+// With knew/vnew (rows of the step's new K and V, new_stride elements apart) the step's token
+// is appended at position len inside the attention kernel, attention covers 0..len, and len
+// advances (the cache must be non-const then).
 int decode_attention_impl(const void* q, int64_t q_stride, const fg_kv_cache* c, void* out,
-                          void* ws, size_t ws_bytes, cudaStream_t s) {
+                          void* ws, size_t ws_bytes, cudaStream_t s, const void* knew = nullptr,
+                          const void* vnew = nullptr, int64_t new_stride = 0, fg_kv_cache* cw = nullptr) {
   if (!q || !c || !out) return fail(FG_ERR_INVALID_ARG, "null pointer");
-  const int B = c->B, nh = c->n_heads, hd = c->head_dim, G = c->group, S = c->len;
+  const bool append = knew != nullptr;
+  if (append && (!vnew || cw != c)) return fail(FG_ERR_INVALID_ARG, "fused append needs K, V and the cache");
+  if (append && c->len + 1 > c->capacity) return fail(FG_ERR_CAPACITY, "KV cache full (capacity %d)", c->capacity);
+  if (append && (new_stride < int64_t(c->n_heads) * c->head_dim || new_stride % 8 || !aligned16(knew) ||
+                 !aligned16(vnew)))
+    return fail(FG_ERR_ALIGN, "new K/V rows must be 16-byte aligned with a stride >= h, multiple of 8");
+  const int B = c->B, nh = c->n_heads, hd = c->head_dim, G = c->group, S = c->len + (append ? 1 : 0);
   if (hd != 64 && hd != 128) return fail(FG_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
   if (G != 32 && G != 64 && G != 128) return fail(FG_ERR_SHAPE, "group must be 32, 64 or 128");
   if (hd % G) return fail(FG_ERR_SHAPE, "group must divide head_dim");
@@ -452,9 +535,15 @@ int decode_attention_impl(const void* q, int64_t q_stride, const fg_kv_cache* c,
   auto* o = reinterpret_cast<__half*>(out);
   auto* kc8 = reinterpret_cast<const uint8_t*>(c->k_codes);
   auto* vc8 = reinterpret_cast<const uint8_t*>(c->v_codes);
+  auto* kn = reinterpret_cast<const __half*>(knew);
+  auto* vn = reinterpret_cast<const __half*>(vnew);
+  auto* kcw = append ? cw->k_codes : nullptr;
+  auto* vcw = append ? cw->v_codes : nullptr;
+  auto* kpw = append ? reinterpret_cast<__half2*>(cw->k_params) : nullptr;
+  auto* vpw = append ? reinterpret_cast<__half2*>(cw->v_params) : nullptr;
 #define FG_ATTN_LAUNCH(HD_, G_)                                                                      \
   FG_LAUNCH("decode attention kernel", decode_attn_mma_kernel<HD_, G_>, dim3(grid), dim3(kThreads), size_t(smem), s, qh, q_stride, kc8, kp, vc8, vp, nh, \
-                                                                c->capacity, S, chunk_len, o, ml, acc)
+                                                                c->capacity, S, chunk_len, o, ml, acc, kn, vn, new_stride, kcw, kpw, vcw, vpw)
   if (hd == 128 && G == 128) FG_ATTN_LAUNCH(128, 128);
   else if (hd == 128 && G == 64) FG_ATTN_LAUNCH(128, 64);
   else if (hd == 128 && G == 32) FG_ATTN_LAUNCH(128, 32);
@@ -468,6 +557,7 @@ int decode_attention_impl(const void* q, int64_t q_stride, const fg_kv_cache* c,
     else
       FG_LAUNCH("decode combine kernel", decode_combine_kernel<64>, dim3((n_bh + 3) / 4), dim3(128), size_t(0), s, ml, acc, n_bh, nc, nh, o);
   }
+  if (append) cw->len += 1;
   return FG_OK;
 }
 

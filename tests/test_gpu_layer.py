@@ -239,3 +239,34 @@ def test_uncompressed_weights_layer_and_generate(fg):
     g_lg, f_tok, f_lg = stepwise_forced(fg, md, mo, ids, T)
     assert np.array_equal(f_tok, exp)          # the oracle's stepwise generation is its generate()
     check_logits_and_tokens(g_lg, f_tok, f_lg)
+
+
+@pytest.mark.parametrize("g,hd", [(64, 128), (32, 128), (64, 64)])
+def test_decode_step_appends_like_kv_append(fg, g, hd):
+    """A decode step appends the token's K/V inside its attention kernel: the cache after
+    fg_decode_layer equals, bit for bit, the cache after the same step's LayerNorm, QKV GEMM
+    and fg_kv_append (the same kernels on the same values), at every position."""
+    import torch
+    h, F, B, L = 256, 1024, 3, 40
+    nh = h // hd
+    ol, ln, d_lins = make_layer(61, 0, h, F, g, wscale=0.05, ln_random=True)
+    dl = to_device_layer(fg, ln, d_lins, g)
+    ca = fg.DeviceKVCache(B, nh, hd, L + 2, g)
+    x = fg_synth.tensor(61, 1, (B * L, h), "normal", 1.0)
+    fg.fg_prefill_layer(dl, ca, to_dev(x), B, L)
+    cb = fg.DeviceKVCache(B, nh, hd, L + 2, g)
+    for name in ("k_codes", "v_codes", "k_params", "v_params"):
+        getattr(cb, name).copy_(getattr(ca, name))
+    cb.length = ca.length
+    for step in range(2):
+        xin = to_dev(fg_synth.tensor(61, 2 + step, (B, h), "normal", 1.0))
+        fg.fg_decode_layer(dl, ca, xin)
+        h1 = fg.fg_layernorm(xin, dl.t[0], dl.t[1])
+        qkv = fg.fg_qgemm(h1, dl.qkv)
+        fg.fg_kv_append(cb, qkv[:, h:], qkv[:, 2 * h:], 3 * h, 1)
+        torch.cuda.synchronize()
+        assert ca.length == cb.length == L + 1 + step
+        for name in ("k_codes", "v_codes"):
+            assert torch.equal(getattr(ca, name), getattr(cb, name)), name
+        for name in ("k_params", "v_params"):
+            assert torch.equal(getattr(ca, name).view(torch.int16), getattr(cb, name).view(torch.int16)), name
