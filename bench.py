@@ -450,7 +450,7 @@ def kernel_case(args):
     qgemm            prompt-pass QKV slice: M 16384, N 12288, K 4096, group 64 (X 134 MB)
     qgemm_decode     a decode step's QKV projection: M 64, N 12288, K 4096 (or --mnk M,N,K)
     gemm_f16         the QKV slice over an fp16 weight; lm_head: [N][K] weight, fp32 logits
-    gemm_prefill     one layer's four prompt-pass GEMMs at M 32768 over fp16 weights
+    gemm_prefill     one layer's four prompt-pass GEMMs at M = B*L of --config over fp16 weights
     decode_attention config-2 decode step: B 64, 32 heads x 128, context 543 (160 MB of cache)
     prefill_attention the prompt pass's causal attention of one layer: B 64, L 512, 32 x 128
                      (805 MB of projections, 268 MB out)
@@ -511,10 +511,14 @@ def kernel_case(args):
             run = lambda: fg.fg_lm_head_argmax(x, w, logits=logits)
         work = {"flops": 2.0 * M * N * K}
     elif args.case == "gemm_prefill":
-        # the prompt pass's four GEMMs of one layer at B*L = 32768 rows, over the fp16 weights
-        # the 4-bit ones expand to: QKV (+bias), out (+bias +residual), fc1 (+bias, relu),
-        # fc2 (+bias +residual); one launch each per step (2.8 GB on the device)
-        M, h, F = 32768, 4096, 16384
+        # the prompt pass's four GEMMs of one layer at B*L rows of the --config workload, over
+        # the fp16 weights the 4-bit ones expand to: QKV (+bias), out (+bias +residual), fc1
+        # (+bias, relu), fc2 (+bias +residual); one launch each per step (c2: M 32768, 2.8 GB
+        # on the device; c3: M 131072, 14 GB)
+        c = use_config(args.config)
+        M, h, F = c["batch"] * c["prompt_len"], c["hidden"], c["ffn"]
+        if args.rows:   # fewer rows of the same shapes (a capture small enough for ncu)
+            M = args.rows
         x = torch.empty((M, h), dtype=torch.float16, device=dev)
         sg.fill(x, SEED, 1, "normal", 1.0)
         ws_ = {}
@@ -798,6 +802,7 @@ def main():
                     default="generate",
                     help="kernel-only cases sized for ncu captures (inputs larger than L2, a few GB at most)")
     ap.add_argument("--mnk", default="", help="M,N,K of the qgemm_decode case")
+    ap.add_argument("--rows", type=int, default=0, help="rows M of the gemm_prefill case (default B*L)")
     ap.add_argument("--weights", choices=["4bit", "fp16", "offload"], default="4bit",
                     help="fp16: the same generation over uncompressed weights (compression contrast); "
                          "offload: 4-bit weights in pinned host memory, streamed layer by layer")
