@@ -25,7 +25,7 @@ namespace {
 
 constexpr int kWarps = 2;
 // Blocks of positions whose loads a warp keeps in flight ahead of the one it computes on.
-constexpr int kAhead = 2;
+constexpr int kAhead = 1;
 constexpr int kThreads = kWarps * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 

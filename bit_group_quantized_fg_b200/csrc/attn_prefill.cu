@@ -65,8 +65,9 @@ __global__ void __launch_bounds__(160, 2)
   uint64_t* pfull = bars + 6;   // [2] P_j written (one arrival per softmax warp)
   uint64_t* ofull = bars + 8;   // O += P_j V_j complete (one phase per tile)
   uint64_t* bar_d = bars + 9;   // drain on abort
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 11);
+  uint64_t* ofin = bars + 10;   // every P V complete (one phase, for the epilogue)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 12);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = gridDim.x - 1 - blockIdx.x;  // heavy (late) tiles first
@@ -101,7 +102,7 @@ __global__ void __launch_bounds__(160, 2)
   if (issuer) {
     // barriers, then the first copies at once: their latency overlaps the TMEM allocation
     prefetch_tmap(&tm);
-    for (int i = 0; i < 10; ++i) mbar_init(&bars[i], (i == 6 || i == 7) ? 4 : 1);
+    for (int i = 0; i < 11; ++i) mbar_init(&bars[i], (i == 6 || i == 7) ? 4 : 1);
     *abort_flag = 0;
     fence_barrier_init();
     // Q rides on the first key tile's barrier (its bytes counted in that phase's expect_tx)
@@ -171,6 +172,10 @@ __global__ void __launch_bounds__(160, 2)
           if (!(ok = issue_qk(j + 2))) break;
         }
       }
+      // The epilogue cannot wait for the last tile on ofull: the issuer never waits for
+      // P_{n-2} V_{n-2}, so two phases of ofull may be pending then, which a parity wait cannot
+      // tell from none.  This commit arrives once every MMA issued so far has completed.
+      if (ok) mma_commit(ofin);
       if (!ok) {
         // drain: copies still in flight, then every MMA issued so far
         for (; k_wt < k_iss; ++k_wt) mbar_wait_drain(&kfull[k_wt & 1], (k_wt >> 1) & 1);
@@ -252,8 +257,8 @@ __global__ void __launch_bounds__(160, 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(&pfull[bb]);
     }
-    // epilogue: O / l to fp16
-    if (ok) ok = mbar_wait(ofull, (n_kt - 1) & 1, abort_flag, err_flag, 0x8000);
+    // epilogue: O / l to fp16, once the last P V has landed
+    if (ok) ok = mbar_wait(ofin, 0, abort_flag, err_flag, 0x8000);
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const float inv = 1.f / l_run;
