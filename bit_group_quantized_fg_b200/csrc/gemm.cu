@@ -82,10 +82,18 @@ struct GemmArgs {
   int relu;
   void* Y;          // fp16 or fp32 [M][N]
   float* partial;   // [splits][M][N] when splits > 1
+  // Wave tail (splits == 1): tiles [0, full_units) run whole, gridDim.x at a time; the
+  // k-blocks of the remaining tail_tiles are divided evenly over all CTAs (CTA b takes the
+  // flat range [I b / grid, I (b + 1) / grid) of I = tail_tiles * k_blocks), which cuts
+  // at most two tiles per CTA; those segments go to tail_part[b][segment][BM][BN] in fp32
+  // and tail_fixup_kernel sums them per tile.
+  int full_units, tail_tiles;
+  float* tail_part;
 };
 
 struct TileCoord {
   int m0, n0, kb0, kb1, ks;
+  int seg;          // tail segment of this CTA (0 or 1), -1 for a whole tile or split-K slice
 };
 
 __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t) {
@@ -102,6 +110,37 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& a, int t) {
   c.n0 = n * BN;
   c.kb0 = int((int64_t(c.ks) * a.k_blocks) / a.splits);
   c.kb1 = int((int64_t(c.ks + 1) * a.k_blocks) / a.splits);
+  c.seg = -1;
+  return c;
+}
+
+// First flat k-block of the wave tail that CTA b computes.
+__host__ __device__ __forceinline__ int64_t tail_start(int64_t I, int b, int grid) { return I * b / grid; }
+
+// Work units of this CTA, in the order every role walks them.
+__device__ __forceinline__ int unit_count(const GemmArgs& a) {
+  const int b = blockIdx.x, G = gridDim.x;
+  if (a.tail_tiles == 0) return b < a.total ? (a.total - 1 - b) / G + 1 : 0;
+  const int64_t I = int64_t(a.tail_tiles) * a.k_blocks;
+  const int64_t s0 = tail_start(I, b, G), s1 = tail_start(I, b + 1, G);
+  int n = a.full_units / G;
+  if (s1 > s0) n += (s0 / a.k_blocks == (s1 - 1) / a.k_blocks) ? 1 : 2;
+  return n;
+}
+
+__device__ __forceinline__ TileCoord unit_coord(const GemmArgs& a, int u) {
+  const int b = blockIdx.x, G = gridDim.x;
+  const int nf = a.tail_tiles == 0 ? 0x7fffffff : a.full_units / G;
+  if (u < nf) return tile_coord(a, b + u * G);
+  const int64_t I = int64_t(a.tail_tiles) * a.k_blocks;
+  const int64_t s0 = tail_start(I, b, G), s1 = tail_start(I, b + 1, G);
+  const int seg = u - nf;
+  const int tile0 = int(s0 / a.k_blocks);
+  const int tile = tile0 + seg;
+  TileCoord c = tile_coord(a, a.full_units + tile);
+  c.kb0 = seg == 0 ? int(s0 - int64_t(tile0) * a.k_blocks) : 0;
+  c.kb1 = int(min(int64_t(a.k_blocks), s1 - int64_t(tile) * a.k_blocks));
+  c.seg = seg;
   return c;
 }
 
@@ -189,8 +228,9 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
       // requested before waiting for the previous kernel, whose output X may still be in
       // the making (programmatic dependent launch).
       int pre = 0;
-      if (args.prefetch_w && int(blockIdx.x) < args.total) {
-        const TileCoord c0 = tile_coord(args, blockIdx.x);
+      const int n_units = unit_count(args);
+      if (args.prefetch_w && n_units > 0) {
+        const TileCoord c0 = unit_coord(args, 0);
         pre = min(S, c0.kb1 - c0.kb0);
         for (int i = 0; i < pre; ++i) {
           mbar_expect_tx(&full[i], tx);
@@ -199,8 +239,8 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
       }
       pdl_wait();
       int issued = 0;
-      for (int t = blockIdx.x; t < args.total && ok; t += gridDim.x) {
-        const TileCoord c = tile_coord(args, t);
+      for (int u = 0; u < n_units && ok; ++u) {
+        const TileCoord c = unit_coord(args, u);
         for (int kb = c.kb0; kb < c.kb1; ++kb, ++issued) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, &g_device_error, 1)) { ok = false; break; }
           uint8_t* st = smem + stage * C::kStageBytes;
@@ -219,7 +259,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
         // issued get it now, so that their barriers complete; then let every copy this
         // thread issued land before the CTA exits
         if (issued < pre) {
-          const TileCoord c0 = tile_coord(args, blockIdx.x);
+          const TileCoord c0 = unit_coord(args, 0);
           for (int i = issued; i < pre; ++i) {
             tma_load_2d(smem + i * C::kStageBytes, &tm_a, (c0.kb0 + i) * BK, c0.m0, &full[i]);
             pend[i] = true;
@@ -239,8 +279,9 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < args.total && ok; t += gridDim.x) {
-        const TileCoord c = tile_coord(args, t);
+      const int n_units = unit_count(args);
+      for (int u = 0; u < n_units && ok; ++u) {
+        const TileCoord c = unit_coord(args, u);
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag, &g_device_error, 2)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
@@ -280,8 +321,9 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
     const int q = warp - 4;  // TMEM lane quarter
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < args.total; t += gridDim.x) {
-      const TileCoord c = tile_coord(args, t);
+    const int n_units = unit_count(args);
+    for (int u = 0; u < n_units; ++u) {
+      const TileCoord c = unit_coord(args, u);
       if (!mbar_wait(&acc_full[acc], acc_phase, abort_flag, &g_device_error, 16)) break;
       tc_fence_after();
       const int m = c.m0 + q * 32 + lane;
@@ -304,6 +346,15 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
         }
         const int n = c.n0 + cc;
         if (!row_ok || n >= args.N) continue;
+        if (c.seg >= 0) {
+          float4* dst = reinterpret_cast<float4*>(
+              args.tail_part + ((int64_t(blockIdx.x) * 2 + c.seg) * BM + (m - c.m0)) * BN + cc);
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                 __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+          continue;
+        }
         if (args.partial != nullptr) {
           float4* dst = reinterpret_cast<float4*>(args.partial + (int64_t(c.ks) * args.M + m) * args.N + n);
 #pragma unroll
@@ -386,8 +437,9 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
     int stage = 0, bs = 0;
     uint32_t phase = 0, bphase = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < args.total && ok; t += gridDim.x) {
-      const TileCoord c = tile_coord(args, t);
+    const int n_units = unit_count(args);
+    for (int u = 0; u < n_units && ok; ++u) {
+      const TileCoord c = unit_coord(args, u);
       const int poff = (c.n0 / args.G) & 3;
       const int pcol = poff + (lane * 8) / args.G;
       for (int kb = c.kb0; kb < c.kb1; ++kb) {
@@ -510,6 +562,67 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ P, int splits, in
     o.w = h2_as_u32(__floats2half2_rn(v[6], v[7]));
     reinterpret_cast<uint4*>(Y)[i] = o;
   }
+}
+
+// Wave tail of a GEMM (see GemmArgs): each tail tile's segments summed in CTA order, then
+// Y = [relu](sum + b) [+ R].  A block covers 8 rows of one tile (32 threads x 8 columns
+// per row); grid = tail_tiles * BM / 8.
+__global__ void __launch_bounds__(256) tail_fixup_kernel(const GemmArgs a, int grid) {
+  pdl_wait();  // the GEMM's partial tiles are complete (see fg_launch)
+  const int tau = blockIdx.x / (BM / 8);
+  const int row = (blockIdx.x % (BM / 8)) * 8 + (threadIdx.x >> 5);
+  const int col = (threadIdx.x & 31) * 8;
+  const TileCoord c = tile_coord(a, a.full_units + tau);
+  const int m = c.m0 + row, n = c.n0 + col;
+  if (m >= a.M || n >= a.N) return;
+  const int64_t kb = a.k_blocks, I = int64_t(a.tail_tiles) * kb;
+  const int64_t x0 = int64_t(tau) * kb, x1 = x0 + kb;
+  // first CTA whose range reaches past x0
+  int g = int(x0 * grid / I);
+  while (g + 1 < grid && tail_start(I, g + 1, grid) <= x0) ++g;
+  while (g > 0 && tail_start(I, g, grid) > x0) --g;
+  float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (; g < grid; ++g) {
+    const int64_t s0 = tail_start(I, g, grid), s1 = tail_start(I, g + 1, grid);
+    if (s0 >= x1) break;
+    if (s1 <= s0 || s1 <= x0) continue;
+    const int seg = s0 >= x0 ? 0 : 1;  // tau is this CTA's first tile, or its second
+    const float4* p = reinterpret_cast<const float4*>(a.tail_part + ((int64_t(g) * 2 + seg) * BM + row) * BN + col);
+    const float4 p0 = p[0], p1 = p[1];
+    v[0] += p0.x; v[1] += p0.y; v[2] += p0.z; v[3] += p0.w;
+    v[4] += p1.x; v[5] += p1.y; v[6] += p1.z; v[7] += p1.w;
+  }
+  if (a.bias) {
+    const uint4 bw = __ldg(reinterpret_cast<const uint4*>(a.bias + n));
+    const __half2* bh = reinterpret_cast<const __half2*>(&bw);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(bh[e]);
+      v[2 * e] += f.x;
+      v[2 * e + 1] += f.y;
+    }
+  }
+  if (a.relu) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = fmaxf(v[j], 0.f);
+  }
+  const int64_t e0 = int64_t(m) * a.N + n;
+  if (a.R) {
+    const uint4 rw = __ldg(reinterpret_cast<const uint4*>(a.R + e0));
+    const __half2* rh = reinterpret_cast<const __half2*>(&rw);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(rh[e]);
+      v[2 * e] += f.x;
+      v[2 * e + 1] += f.y;
+    }
+  }
+  uint4 o;
+  o.x = h2_as_u32(__floats2half2_rn(v[0], v[1]));
+  o.y = h2_as_u32(__floats2half2_rn(v[2], v[3]));
+  o.z = h2_as_u32(__floats2half2_rn(v[4], v[5]));
+  o.w = h2_as_u32(__floats2half2_rn(v[6], v[7]));
+  *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(a.Y) + e0) = o;
 }
 
 // Split-K reduction + epilogue + LayerNorm of the row, for a GEMM whose output row feeds a
@@ -663,7 +776,8 @@ int launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& p, con
   using C = Cfg<MODE>;
   static std::atomic<uint64_t> attr_done{0};
   FG_TRY(ensure_smem_attr(gemm_tc_kernel<MODE, F32>, C::kSmem, attr_done));
-  const int grid = std::min(args.total, num_sms());
+  // a wave tail is spread over every SM (tail_fixup_kernel assumes that grid)
+  const int grid = args.tail_tiles > 0 ? num_sms() : std::min(args.total, num_sms());
   FG_LAUNCH("tcgen05 gemm kernel", gemm_tc_kernel<MODE, F32>, dim3(grid), dim3(C::kThreads), size_t(C::kSmem), s, a, b, p, args);
   return FG_OK;
 }
@@ -674,6 +788,20 @@ int pick_splits(int tiles, int k_blocks) {
   int sp = sms / tiles;
   sp = std::min(sp, k_blocks / 2);
   return std::max(sp, 1);
+}
+
+// Tiles of a GEMM with one K-split that fill the SMs unevenly (a last, partial wave) spread
+// that wave's k-blocks over every SM when the estimated time, in k-blocks per SM, drops by
+// more than the fix-up's cost (taken as 16 k-blocks: the segments' fp32 write and the second
+// kernel; at 8 the OPT-175B QKV shape, 1.95 waves, chose the tail and ran 2 % slower).
+// Returns the number of tail tiles (0: tiles run whole, in waves).
+int pick_tail(int tiles, int k_blocks, int N) {
+  const int sms = num_sms();
+  if (N % BN || tiles < sms / 2 || tiles % sms == 0 || tiles >= 4 * sms) return 0;
+  const int tail = tiles % sms;
+  const int64_t waves = int64_t((tiles + sms - 1) / sms) * k_blocks;
+  const int64_t spread = int64_t(tiles / sms) * k_blocks + (int64_t(tail) * k_blocks + sms - 1) / sms;
+  return spread + 16 < waves ? tail : 0;
 }
 
 }  // namespace
@@ -720,13 +848,17 @@ int* device_error_ptr() {
   return ptr[dev];
 }
 
-// Split-K partials of one GEMM (0 when the tiles alone fill the GPU).
+// Split-K partials of one GEMM, or the fp32 segments of its wave tail (0 when the tiles
+// alone fill the GPU evenly).
 size_t splitk_ws_bytes(int64_t M, int N, int K) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
   const int m_tiles = int((M + BM - 1) / BM);
   const int n_tiles = (N + BN - 1) / BN;
   const int sp = pick_splits(m_tiles * n_tiles, K / BK);
-  if (sp <= 1) return 0;
+  if (sp <= 1) {
+    if (pick_tail(m_tiles * n_tiles, K / BK, N) == 0) return 0;
+    return size_t(num_sms()) * 2 * BM * BN * sizeof(float);
+  }
   return size_t(sp) * size_t(M) * size_t(N) * sizeof(float);
 }
 
@@ -791,6 +923,16 @@ int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, c
   a.Y = Y;
   a.prefetch_w = w_ready ? 1 : 0;
   a.partial = nullptr;
+  a.full_units = 0;
+  a.tail_tiles = (a.splits == 1 && !out_f32) ? pick_tail(a.m_tiles * a.n_tiles, a.k_blocks, N) : 0;
+  a.tail_part = nullptr;
+  if (a.tail_tiles > 0) {
+    const size_t need = size_t(num_sms()) * 2 * BM * BN * sizeof(float);
+    if (!ws || ws_bytes < need) return fail(FG_ERR_WORKSPACE, "GEMM wave tail needs %zu workspace bytes", need);
+    if (!aligned16(ws)) return fail(FG_ERR_ALIGN, "workspace must be 16-byte aligned");
+    a.full_units = a.total - a.tail_tiles;
+    a.tail_part = reinterpret_cast<float*>(ws);
+  }
   if (a.splits > 1) {
     const size_t need = size_t(a.splits) * size_t(M) * size_t(N) * sizeof(float);
     if (!ws || ws_bytes < need) return fail(FG_ERR_WORKSPACE, "GEMM split-K needs %zu workspace bytes", need);
@@ -832,7 +974,12 @@ int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, c
     else if (mode == B_F16_MN) st = launch<B_F16_MN, false>(ta, tb, tp, a, s);
     else st = out_f32 ? launch<B_F16_K, true>(ta, tb, tp, a, s) : launch<B_F16_K, false>(ta, tb, tp, a, s);
     if (st != FG_OK) return st;
-    // the split-K reduction (and a fused LayerNorm) is timed with its GEMM
+    // the split-K reduction (and a fused LayerNorm), or the wave tail's fix-up, is timed
+    // with its GEMM
+    if (a.tail_tiles > 0) {
+      FG_LAUNCH("wave-tail fix-up kernel", tail_fixup_kernel, dim3(a.tail_tiles * (BM / 8)), dim3(256), size_t(0), s,
+                a, num_sms());
+    }
     if (a.splits > 1) {
       if (ln && ln->g && ln->b && ln->H && !relu && N % 8 == 0 && N <= 12288 && aligned16(ln->g) &&
           aligned16(ln->b) && aligned16(ln->H)) {
