@@ -24,17 +24,29 @@ namespace fg {
 namespace {
 
 constexpr int kWarps = 2;
-// Blocks of positions whose loads a warp keeps in flight ahead of the one it computes on.
-constexpr int kAhead = 1;
+// Blocks of positions a warp keeps in flight (cp.async into its shared-memory ring) ahead of
+// the one it computes on: the bytes in flight no longer cost registers.
+constexpr int kDepth = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 
-__device__ __forceinline__ uint4 ldg_v4(const uint4* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
+// 16-byte global -> shared copy of which the first `bytes` (0..16) are read and the rest is
+// zero-filled (L2 only: the cache is streamed once); both addresses 16-byte aligned.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src), "r"(bytes)
+               : "memory");
+}
+// 4-byte copy (`bytes` 0 or 4; 0 writes a zero word without reading).
+__device__ __forceinline__ void cp_async4(void* dst, const void* src, int bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // ------------------------------------------------------------------ K4, tensor-core form
@@ -83,6 +95,11 @@ struct AttnMma {
   static constexpr int DPT = HD / 8;   // dims per value row-thread
   static constexpr int VW = HD / 64;   // code words a thread reads of a V row
   static constexpr int TB = 16;        // positions per block
+  // a block in a warp's ring: K codes, V codes (TB rows of HD/2 bytes), K params, V params
+  // (TB rows of NG {min, scale} pairs), each a contiguous run of the cache
+  static constexpr int RC = HD / 2, RP = NG * 4;                // row bytes
+  static constexpr int SLOT = 2 * TB * RC + 2 * TB * RP;      // bytes of one block
+  static_assert(SLOT % 16 == 0 && RC % 16 == 0, "16-byte copies");
 };
 
 // Fused append (the decode step's KV append): when `knew` is not NULL, position S - 1 is the
@@ -187,55 +204,75 @@ __global__ void __launch_bounds__(kThreads) decode_attn_mma_kernel(
 #pragma unroll
   for (int i = 0; i < MT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
 
-  // raw loads of one block: K rows g, g+8 (KW words from word KW*q4), V rows 2q4, 2q4+1,
+  // One block's registers: K rows g, g+8 (KW words from word KW*q4), V rows 2q4, 2q4+1,
   // 2q4+8, 2q4+9 (VW words at dim DPT*g), K params of (row, groups 2q4, 2q4+1), V params of
-  // (row, group q4); positions past t1 read as zeros
+  // (row, group q4); positions past t1 hold zeros (the ring copies zero-fill them).
   struct Blk {
     uint32_t kA[KW], kB[KW], vw[4][VW], kpA[2], kpB[2], vpA, vpB;
   };
-  auto load = [&](Blk& o, int blk) {
-    const int tA = blk + g, tB = blk + g + 8;
-    // the new token's position is taken from shared memory below, not loaded
-    const bool okA = tA < t1 && !(app && tA == tnew), okB = tB < t1 && !(app && tB == tnew);
-    if (KW == 4) {
-      const uint4 za = okA ? ldg_v4(reinterpret_cast<const uint4*>(kbase + int64_t(tA) * (HD / 2)) + q4)
-                           : make_uint4(0, 0, 0, 0);
-      const uint4 zb = okB ? ldg_v4(reinterpret_cast<const uint4*>(kbase + int64_t(tB) * (HD / 2)) + q4)
-                           : make_uint4(0, 0, 0, 0);
-      o.kA[0] = za.x; o.kA[1 % KW] = za.y; o.kA[2 % KW] = za.z; o.kA[3 % KW] = za.w;
-      o.kB[0] = zb.x; o.kB[1 % KW] = zb.y; o.kB[2 % KW] = zb.z; o.kB[3 % KW] = zb.w;
-    } else {
-      const uint2 za = okA ? __ldg(reinterpret_cast<const uint2*>(kbase + int64_t(tA) * (HD / 2)) + q4)
-                           : make_uint2(0, 0);
-      const uint2 zb = okB ? __ldg(reinterpret_cast<const uint2*>(kbase + int64_t(tB) * (HD / 2)) + q4)
-                           : make_uint2(0, 0);
-      o.kA[0] = za.x; o.kA[1 % KW] = za.y;
-      o.kB[0] = zb.x; o.kB[1 % KW] = zb.y;
-    }
+  __shared__ __align__(16) uint8_t ring[kWarps][kDepth][C::SLOT];
+  // the copies of block `blk` into ring slot `sl` of this warp; rows at or past t1 are
+  // written as zeros without being read.  Codes go in 16-byte chunks (a row is HD/2 bytes,
+  // a multiple of 16); the {min, scale} rows of one (sequence, head) start only 4 * NG-byte
+  // aligned (at (b * nh + head) * cap * NG pairs), so they go word by word.
+  auto issue = [&](int sl, int blk) {
+    uint8_t* dst = ring[warp][sl];
+    const int nv = max(0, min(TB, t1 - blk));   // valid rows of the block
+    constexpr int kCodeChunks = 2 * TB * C::RC / 16;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int t = blk + 2 * q4 + (r & 1) + (r >> 1) * 8;
-      const bool ok = t < t1 && !(app && t == tnew);
-      const uint32_t* src = reinterpret_cast<const uint32_t*>(vbase + int64_t(t) * (HD / 2)) + VW * g;
-      if (VW == 2) {
-        const uint2 z = ok ? __ldg(reinterpret_cast<const uint2*>(src)) : make_uint2(0, 0);
-        o.vw[r][0] = z.x;
-        o.vw[r][VW - 1] = z.y;
-      } else {
-        o.vw[r][0] = ok ? __ldg(src) : 0u;
+    for (int j = 0; j < (kCodeChunks + 31) / 32; ++j) {
+      const int i = lane + 32 * j;
+      if (i < kCodeChunks) {
+        const int o = i * 16;
+        const bool v = o >= TB * C::RC;
+        const int off = v ? o - TB * C::RC : o;
+        const bool ok = off / C::RC < nv;
+        cp_async16(dst + o, ok ? (v ? vbase : kbase) + int64_t(blk) * C::RC + off : kbase, ok ? 16 : 0);
       }
     }
+    constexpr int kParWords = 2 * TB * NG;
     const uint32_t* kpu = reinterpret_cast<const uint32_t*>(kpb);
     const uint32_t* vpu = reinterpret_cast<const uint32_t*>(vpb);
 #pragma unroll
+    for (int j = 0; j < (kParWords + 31) / 32; ++j) {
+      const int i = lane + 32 * j;
+      if (i < kParWords) {
+        const bool v = i >= TB * NG;
+        const int wi = v ? i - TB * NG : i;   // word of the block's param run
+        const bool ok = wi / NG < nv;
+        cp_async4(dst + 2 * TB * C::RC + 4 * i, ok ? (v ? vpu : kpu) + int64_t(blk) * NG + wi : kpu, ok ? 4 : 0);
+      }
+    }
+  };
+  // the block in ring slot `sl` into registers; the new token's position comes from the
+  // quantizer's shared-memory copy
+  auto fetch = [&](Blk& o, int sl, int blk) {
+    const uint8_t* r = ring[warp][sl];
+    const uint8_t* kr = r;
+    const uint8_t* vr = r + TB * C::RC;
+    const uint32_t* kpr = reinterpret_cast<const uint32_t*>(r + 2 * TB * C::RC);
+    const uint32_t* vpr = reinterpret_cast<const uint32_t*>(r + 2 * TB * C::RC + TB * C::RP);
+#pragma unroll
+    for (int i = 0; i < KW; ++i) {
+      o.kA[i] = reinterpret_cast<const uint32_t*>(kr + g * C::RC)[KW * q4 + i];
+      o.kB[i] = reinterpret_cast<const uint32_t*>(kr + (g + 8) * C::RC)[KW * q4 + i];
+    }
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+      const int t = 2 * q4 + (rr & 1) + (rr >> 1) * 8;
+#pragma unroll
+      for (int w = 0; w < VW; ++w) o.vw[rr][w] = reinterpret_cast<const uint32_t*>(vr + t * C::RC)[VW * g + w];
+    }
+#pragma unroll
     for (int j = 0; j < 2; ++j) {
       const int n = 2 * q4 + j;
-      o.kpA[j] = (n < NG && okA) ? __ldg(kpu + int64_t(tA) * NG + n) : 0u;
-      o.kpB[j] = (n < NG && okB) ? __ldg(kpu + int64_t(tB) * NG + n) : 0u;
+      o.kpA[j] = n < NG ? kpr[g * NG + (n < NG ? n : 0)] : 0u;
+      o.kpB[j] = n < NG ? kpr[(g + 8) * NG + (n < NG ? n : 0)] : 0u;
     }
-    o.vpA = (q4 < NG && okA) ? __ldg(vpu + int64_t(tA) * NG + q4) : 0u;
-    o.vpB = (q4 < NG && okB) ? __ldg(vpu + int64_t(tB) * NG + q4) : 0u;
+    o.vpA = q4 < NG ? vpr[g * NG + (q4 < NG ? q4 : 0)] : 0u;
+    o.vpB = q4 < NG ? vpr[(g + 8) * NG + (q4 < NG ? q4 : 0)] : 0u;
     if (app && tnew >= blk && tnew < blk + TB) {
+      const int tA = blk + g, tB = blk + g + 8;
       const bool pA = tA == tnew, pB = tB == tnew;
       if (pA || pB) {
 #pragma unroll
@@ -256,22 +293,31 @@ __global__ void __launch_bounds__(kThreads) decode_attn_mma_kernel(
         if (pB) o.vpB = pv;
       }
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        if (blk + 2 * q4 + (r & 1) + (r >> 1) * 8 == tnew) {
+      for (int rr = 0; rr < 4; ++rr) {
+        if (blk + 2 * q4 + (rr & 1) + (rr >> 1) * 8 == tnew) {
 #pragma unroll
-          for (int w = 0; w < VW; ++w) o.vw[r][w] = new_codes[1][VW * g + w];
+          for (int w = 0; w < VW; ++w) o.vw[rr][w] = new_codes[1][VW * g + w];
         }
       }
     }
   };
 
-  Blk cur, nx1;
-  load(cur, t0 + warp * TB);
-  if (kAhead > 1) load(nx1, t0 + warp * TB + kWarps * TB);
+  // one commit group per block, empty ones past t1, so that the wait count stays uniform
+#pragma unroll
+  for (int i = 0; i < kDepth; ++i) {
+    issue(i, t0 + warp * TB + i * kWarps * TB);
+    cp_async_commit();
+  }
+  int sl = 0;
   for (int blk = t0 + warp * TB; blk < t1; blk += kWarps * TB) {
-    Blk nxt;
-    // the loads of the next kAhead blocks are in flight while this one computes
-    load(nxt, blk + kAhead * kWarps * TB);
+    Blk cur;
+    cp_async_wait<kDepth - 1>();
+    __syncwarp();   // every lane's copies of this block have landed
+    fetch(cur, sl, blk);
+    __syncwarp();   // every lane has read the slot before it is refilled
+    issue(sl, blk + kDepth * kWarps * TB);
+    cp_async_commit();
+    if (++sl == kDepth) sl = 0;
     const int tA = blk + g, tB = blk + g + 8;
     const bool okA = tA < t1, okB = tB < t1;
     const uint32_t(&kA)[KW] = cur.kA;
@@ -364,13 +410,8 @@ __global__ void __launch_bounds__(kThreads) decode_attn_mma_kernel(
       const uint32_t a2 = ((r23 << 4) & 0x00F000F0u) | 0x54005400u, a3 = (r23 & 0x00F000F0u) | 0x54005400u;
       mma16816(acc[mt], a0, a1, a2, a3, b0, b1);
     }
-    if (kAhead > 1) {
-      cur = nx1;
-      nx1 = nxt;
-    } else {
-      cur = nxt;
-    }
   }
+  cp_async_wait<0>();   // nothing in flight when the warp leaves its ring
 
   // ---- finish the warp: sums over rows, then out_d for the dims this lane holds
 #pragma unroll
@@ -478,7 +519,11 @@ int pick_chunks(int B, int nh, int S) {
   int nc = (target + bh - 1) / bh;
   const int max_by_len = (S + 127) / 128;  // at least 128 positions per chunk
   nc = std::min(nc, std::max(1, max_by_len));
-  const int min_by_len = (S + 4095) / 4096;  // at most 4096 positions per chunk
+  // At most 2048 positions per chunk: the offset codes' cancellation error (the value MMA
+  // sums w (64 + c) over the chunk in fp32, then 64 * sum(w) is subtracted) grows with the
+  // chunk while the output of a near-uniform softmax shrinks; chunks of 4096 measured
+  // 1.24e-2 * RMS at context 8192, chunks of 2048 stay near 4e-3.
+  const int min_by_len = (S + 2047) / 2048;
   return std::max(nc, std::max(1, min_by_len));
 }
 

@@ -66,10 +66,13 @@ def test_decode_attention_t3_and_outliers(fg):
     (256, 56, 543),   # OPT-30B shape, batch 256
     (144, 96, 543),   # OPT-175B shape, batch 144
     (64, 32, 2048),   # a long context with enough sequences x heads for one chunk each
+    (64, 32, 8192),   # the sweep's longest context at batch 64: the offset-code cancellation
+                      # (64 + c summed over the context, 64 * sum(w) subtracted) at its largest
 ])
 def test_decode_attention_sampled_full_size(fg, B, nh, S):
     """Decode attention at the configurations' full shapes (head dim 128, group 64, context
-    543): sampled sequences checked against the oracle, the rest for finiteness."""
+    543) and at long contexts: sampled sequences checked against the oracle, the rest for
+    finiteness."""
     import torch
     hd, g = 128, 64
     h = nh * hd
