@@ -204,10 +204,6 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
       uint32_t phase = 0;
       uint32_t tx = kABytes + (C::kQ4 ? (kCodeBytes + args.param_bytes) : kBBytes);
       bool ok = true;
-      bool pend[S];
-      uint32_t pend_phase[S];
-#pragma unroll
-      for (int i = 0; i < S; ++i) { pend[i] = false; pend_phase[i] = 0; }
       // the weight operand of k-block kb of tile c into stage buffer st
       auto load_w = [&](uint8_t* st, const TileCoord& c, int kb, uint64_t* bar) {
         if (MODE == B_Q4) {
@@ -249,8 +245,6 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
             load_w(st, c, kb, &full[stage]);
           }
           tma_load_2d(st, &tm_a, kb * BK, c.m0, &full[stage]);
-          pend[stage] = true;
-          pend_phase[stage] = phase;
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
       }
@@ -260,14 +254,13 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
         // thread issued land before the CTA exits
         if (issued < pre) {
           const TileCoord c0 = unit_coord(args, 0);
-          for (int i = issued; i < pre; ++i) {
+          for (int i = issued; i < pre; ++i)
             tma_load_2d(smem + i * C::kStageBytes, &tm_a, (c0.kb0 + i) * BK, c0.m0, &full[i]);
-            pend[i] = true;
-            pend_phase[i] = 0;
-          }
         }
-        for (int i = 0; i < S; ++i)
-          if (pend[i]) mbar_wait_drain(&full[i], pend_phase[i]);
+        // stage q (in issue order) went to slot q % S in phase (q / S) & 1; only the last S
+        // can still be in flight
+        const int armed = max(issued, pre);
+        for (int q = max(0, armed - S); q < armed; ++q) mbar_wait_drain(&full[q % S], uint32_t(q / S) & 1u);
       }
     }
   } else if (warp == 1) {
@@ -291,14 +284,14 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1)
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + stage * C::kStageBytes);
           const uint32_t b_addr = C::kQ4 ? smem_u32(bring + bs * kBBytes) : a_addr + kABytes;
+          // the k-th 16-deep slice: +32 bytes along K (K-major) or +2048 (MN-major: two 8-row
+          // groups of 1024 bytes); the descriptor's address field counts 16-byte units
+          const uint64_t ad0 = smem_desc_sw128(a_addr, 16, 1024);
+          const uint64_t bd0 = MODE == B_F16_K ? smem_desc_sw128(b_addr, 16, 1024) : smem_desc_sw128(b_addr, 8192, 1024);
+          constexpr uint64_t kBStep = MODE == B_F16_K ? 2 : 128;
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t ad = smem_desc_sw128(a_addr + k * 32, 16, 1024);
-            uint64_t bd;
-            if (MODE == B_F16_K) bd = smem_desc_sw128(b_addr + k * 32, 16, 1024);
-            else bd = smem_desc_sw128(b_addr + k * 2048, 8192, 1024);
-            mma_f16_ss(d_tmem, ad, bd, idesc, (kb > c.kb0 || k > 0) ? 1u : 0u);
-          }
+          for (int k = 0; k < BK / 16; ++k)
+            mma_f16_ss(d_tmem, ad0 + uint64_t(2 * k), bd0 + kBStep * k, idesc, (kb > c.kb0 || k > 0) ? 1u : 0u);
           mma_commit(&empty[stage]);
           if (++stage == S) { stage = 0; phase ^= 1; }
           if (C::kQ4) {
