@@ -18,8 +18,8 @@
 //               the MN-major 128-byte-swizzled operand layout the MMA reads.
 // Other operand modes reuse the skeleton: B as a ready fp16 [K][N] tensor (MN-major, by
 // TMA) or as an fp16 [N][K] tensor (K-major by TMA, the tied LM head).  Tiles are
-// rasterized in bands of row tiles (~16 MB of X) so a band of X stays in L2 while the
-// weight streams past it.
+// rasterized in bands of row tiles (at most 64 MiB of X) so a band of X stays in L2 while
+// the weight streams past it.
 // With few tiles (decode batches) the K loop is split and fp32 partials are reduced by a
 // second kernel that applies the epilogue.
 #include <algorithm>
@@ -900,12 +900,12 @@ int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, c
   a.k_blocks = K / BK;
   a.splits = out_f32 ? 1 : pick_splits(a.m_tiles * a.n_tiles, a.k_blocks);
   // Rasterization: bands of row tiles whose X rows stay in L2 while every column tile of the
-  // band runs; the weight is read once per band.  A band holds at most ~16 MB of X (16 row
-  // tiles at K 4096, 8 up to K 8192, 4 beyond): the L2 is split between the two dies.  On
-  // the OPT-30B prompt-pass shapes 4 row tiles at K 28672 ran 23 % faster than 16, 8 at
-  // K 7168 the same as 16 within 4 %; on the OPT-6.7B ones bands of ~48 MB moved 5-35 % more
-  // DRAM bytes than bands of 16 MB.
-  a.band = K <= 4096 ? 16 : (K <= 8192 ? 8 : 4);
+  // band runs; the weight is read once per band, so larger bands read it less often.  A band
+  // holds at most 64 MiB of X (half the L2): 16 row tiles up to K 16384, 8 at K 28672.  On the
+  // OPT-30B prompt-pass shapes (K 7168 and 28672) that ran 2.5 % faster than bands of ~16 MB,
+  // and 23 % faster than 16 row tiles at K 28672 (117 MB of X).
+  a.band = 16;
+  while (a.band > 2 && int64_t(BM) * a.band * K * 2 > (int64_t(64) << 20)) a.band /= 2;
   a.total = a.m_tiles * a.n_tiles * a.splits;
   a.G = G;
   a.PB = G == 32 ? 8 : 4;
