@@ -63,9 +63,12 @@ def test_qgemm_decode_split_k(fg):
     (256, 512, 640, 128, True, False),     # two full row chunks, g 128
     (64, 256, 4096, 64, False, False),     # one tile, K split 8 ways
     (64, 3072, 4096, 64, False, False),    # 12 tiles x 8-way K split
+    (256, 4096, 2048, 64, False, True),    # two row tiles, K split 4 ways
+    (200, 20480, 2048, 64, True, True),    # 160 tiles: 148 whole + a wave tail of 12
 ])
 def test_qgemm_decode_batches(fg, M, N, K, g, relu, resid):
-    """Decode-size GEMMs (M <= 256): ragged rows, row tiles, group sizes, deep K splits."""
+    """Decode-size GEMMs (M <= 256): ragged rows, row tiles, group sizes, deep K splits, the
+    wave tail."""
     got, exp = _case(fg, M, N, K, g, relu, resid, seed=3 * M + N + K)
     assert_close_rms(got, exp, what="decode qgemm")
 
