@@ -64,14 +64,39 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const uint4* __
 }
 
 // ------------------------------------------------------------------ KV append
+// n / d for 0 <= n < 2^31 by a multiply-high and a shift (Granlund and Montgomery, "Division
+// by invariant integers using multiplication", 1994): with l = ceil(log2 d) and
+// m = ceil(2^(31 + l) / d) < 2^32, n / d = (n m) >> (31 + l), because m d - 2^(31 + l) < d
+// keeps the error term n (m d - 2^(31 + l)) / (d 2^(31 + l)) below 1/d.  d = 1 is passed
+// through.  The append splits every 16-value chunk index into (row, chunk, sequence, token,
+// head): 64-bit divisions there cost more than the quantization itself.
+struct FastDiv {
+  uint32_t m;
+  int s;      // shift after the multiply-high: l - 1
+  int one;    // d == 1
+};
+FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f{0, 0, d == 1};
+  if (d > 1) {
+    int l = 0;
+    while ((uint64_t(1) << l) < d) ++l;
+    f.m = uint32_t(((uint64_t(1) << (31 + l)) + d - 1) / d);
+    f.s = l - 1;
+  }
+  return f;
+}
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+  return f.one ? n : (__umulhi(n, f.m) >> f.s);
+}
+
 // Rows r = b*T + t of k (blockIdx.y == 0) or v (== 1); h valid values per row, quantized in
 // chunks of 16 along the hidden dimension.  The group of head `head` lands at cache
-// position pos0 + t.
-template <int G, int U>
+// position pos0 + t.  FAST: fewer than 2^31 chunks, indices split with FastDiv.
+template <int G, int U, bool FAST>
 __global__ void __launch_bounds__(kThreads) kv_append_kernel(
     const __half* __restrict__ k, const __half* __restrict__ v, int64_t row_stride, int T, int h,
     int hd, int cap, int pos0, int64_t n_chunks, uint2* __restrict__ kc, uint2* __restrict__ vc,
-    __half2* __restrict__ kp, __half2* __restrict__ vp) {
+    __half2* __restrict__ kp, __half2* __restrict__ vp, FastDiv f_cpr, FastDiv f_T, FastDiv f_hd) {
   pdl_wait();  // the previous kernel in the stream has finished (see fg_launch)
   constexpr int TPG = G / 16;
   const __half* src = blockIdx.y == 0 ? k : v;
@@ -86,7 +111,7 @@ __global__ void __launch_bounds__(kThreads) kv_append_kernel(
     for (int u = 0; u < U; ++u) {
       const int64_t c = base + u * kThreads + threadIdx.x;
       if (c < n_chunks) {
-        const int64_t row = c / chunks_per_row;
+        const int64_t row = FAST ? int64_t(fdiv(uint32_t(c), f_cpr)) : c / chunks_per_row;
         const int cc = int(c - row * chunks_per_row);
         const uint4* p = reinterpret_cast<const uint4*>(src + row * row_stride + cc * 16);
         va[u] = ld_nc_v4(p);
@@ -101,12 +126,12 @@ __global__ void __launch_bounds__(kThreads) kv_append_kernel(
       const int64_t c = base + u * kThreads + threadIdx.x;
       GroupQ q = quantize_chunk16<TPG>(va[u], vb[u]);
       if (c < n_chunks) {
-        const int64_t row = c / chunks_per_row;
+        const int64_t row = FAST ? int64_t(fdiv(uint32_t(c), f_cpr)) : c / chunks_per_row;
         const int cc = int(c - row * chunks_per_row);
-        const int64_t b = row / T;
+        const int64_t b = FAST ? int64_t(fdiv(uint32_t(row), f_T)) : row / T;
         const int t = int(row - b * T);
         const int d = cc * 16;
-        const int head = d / hd;
+        const int head = FAST ? int(fdiv(uint32_t(d), f_hd)) : d / hd;
         const int dh = d - head * hd;
         const int64_t slot = (b * nh + head) * int64_t(cap) + (pos0 + t);
         dc[slot * (hd / 16) + dh / 16] = q.words;
@@ -322,12 +347,22 @@ int kv_append_impl(fg_kv_cache* c, const void* k, const void* v, int64_t row_str
   auto* vc = reinterpret_cast<uint2*>(c->v_codes);
   auto* kp = reinterpret_cast<__half2*>(c->k_params);
   auto* vp = reinterpret_cast<__half2*>(c->v_params);
-  if (G == 32)
-    FG_LAUNCH("kv append kernel", (small ? kv_append_kernel<32, 1> : kv_append_kernel<32, kUnroll>), dim3(grid), dim3(kThreads), size_t(0), s, K, V, row_stride, n_tokens, h, hd, c->capacity, c->len, chunks, kc, vc, kp, vp);
-  else if (G == 64)
-    FG_LAUNCH("kv append kernel", (small ? kv_append_kernel<64, 1> : kv_append_kernel<64, kUnroll>), dim3(grid), dim3(kThreads), size_t(0), s, K, V, row_stride, n_tokens, h, hd, c->capacity, c->len, chunks, kc, vc, kp, vp);
-  else
-    FG_LAUNCH("kv append kernel", (small ? kv_append_kernel<128, 1> : kv_append_kernel<128, kUnroll>), dim3(grid), dim3(kThreads), size_t(0), s, K, V, row_stride, n_tokens, h, hd, c->capacity, c->len, chunks, kc, vc, kp, vp);
+  const bool fast = chunks < (int64_t(1) << 31);
+  const FastDiv f_cpr = make_fastdiv(uint32_t(h / 16)), f_T = make_fastdiv(uint32_t(n_tokens)),
+                f_hd = make_fastdiv(uint32_t(hd));
+  using KernelT = void (*)(const __half*, const __half*, int64_t, int, int, int, int, int, int64_t, uint2*, uint2*,
+                           __half2*, __half2*, FastDiv, FastDiv, FastDiv);
+  // [group 32 / 64 / 128][one chunk per thread, kUnroll][64-bit, fast indices]
+  static const KernelT table[3][2][2] = {
+      {{kv_append_kernel<32, 1, false>, kv_append_kernel<32, 1, true>},
+       {kv_append_kernel<32, kUnroll, false>, kv_append_kernel<32, kUnroll, true>}},
+      {{kv_append_kernel<64, 1, false>, kv_append_kernel<64, 1, true>},
+       {kv_append_kernel<64, kUnroll, false>, kv_append_kernel<64, kUnroll, true>}},
+      {{kv_append_kernel<128, 1, false>, kv_append_kernel<128, 1, true>},
+       {kv_append_kernel<128, kUnroll, false>, kv_append_kernel<128, kUnroll, true>}}};
+  const KernelT kern = table[G == 32 ? 0 : (G == 64 ? 1 : 2)][small ? 0 : 1][fast ? 1 : 0];
+  FG_LAUNCH("kv append kernel", kern, dim3(grid), dim3(kThreads), size_t(0), s, K, V, row_stride, n_tokens, h, hd,
+            c->capacity, c->len, chunks, kc, vc, kp, vp, f_cpr, f_T, f_hd);
   c->len += n_tokens;
   return FG_OK;
 }
