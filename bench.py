@@ -803,6 +803,8 @@ def main():
                     help="kernel-only cases sized for ncu captures (inputs larger than L2, a few GB at most)")
     ap.add_argument("--mnk", default="", help="M,N,K of the qgemm_decode case")
     ap.add_argument("--rows", type=int, default=0, help="rows M of the gemm_prefill case (default B*L)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="sequences per GPU instead of the configuration's (small batches: the latency side)")
     ap.add_argument("--weights", choices=["4bit", "fp16", "offload"], default="4bit",
                     help="fp16: the same generation over uncompressed weights (compression contrast); "
                          "offload: 4-bit weights in pinned host memory, streamed layer by layer")
@@ -812,6 +814,8 @@ def main():
     if args.case != "generate":
         return kernel_case(args)
     c = use_config(args.config)
+    if args.batch:
+        c["batch"] = args.batch
     world, rank, local = replica_env()
     wdesc = {"4bit": "4-bit weights", "fp16": "fp16 (uncompressed) weights",
              "offload": "4-bit weights in pinned host memory (streamed per layer)"}[args.weights]
