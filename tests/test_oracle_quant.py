@@ -225,7 +225,7 @@ def test_storage_matches_readme_about_70_percent(g, expect_pct):
     assert nbytes == oracle.storage_bytes(rows * cols, g) == rows * cols // 2 + 4 * rows * cols // g
     saving = 100.0 * (1 - nbytes / (2 * rows * cols))
     assert saving == pytest.approx(expect_pct)
-    assert abs(saving - 70.0) < 4.0          # "around 70 %"
+    assert abs(saving - 70.0) < 4.0          # the README mirror states a saving of roughly 70 %
 
 
 # ----------------------------------------------------------------------------------------
