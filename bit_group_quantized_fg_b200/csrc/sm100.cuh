@@ -1,7 +1,7 @@
 // Thin wrappers over the sm_100a PTX used by the tensor-core kernels: mbarriers with
-// bounded waits, TMA tile loads (no multicast), tcgen05 MMA / TMEM alloc / ld / commit,
-// and the shared-memory matrix descriptors.  Written from the PTX ISA's descriptions of
-// these instructions.
+// bounded waits, TMA tile loads into the issuing CTA's own shared memory, tcgen05 MMA /
+// TMEM alloc / ld / commit, and the shared-memory matrix descriptors.  Written from the PTX
+// ISA's descriptions of these instructions.
 #pragma once
 
 #include <cuda.h>
