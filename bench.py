@@ -948,7 +948,7 @@ def main():
         "vs_baseline": None, "dtype": "f16", "data": "synthetic", "config": config,
         "prefill_ms": statistics.median(t[0] for t in r["timings"]),
         "decode_ms": statistics.median(t[1] for t in r["timings"]),
-        "roofline": {"kernel": f"tcgen05 GEMM of the prompt pass (M = {M_pf}; " +
+        "roofline": {"kernel": f"tcgen05 GEMM of the prompt pass on CTA pairs (M = {M_pf}; " +
                                ("4-bit weights expanded to fp16 once per layer)" if args.weights != "fp16"
                                 else "uncompressed fp16 weights)"), "bound": "tensor",
                      "achieved": achieved_tf, "peak": pk["tf_sust"], "unit": "TFLOP/s",

@@ -95,6 +95,10 @@ int ensure_smem_attr(Kernel kernel, int bytes, std::atomic<uint64_t>& done) {
 // fp16 tensor-core GEMM (measured break-even ~700 rows on B200).
 constexpr int64_t kExpandRows = 1024;
 
+// Row count from which an fp16 [K][N] GEMM runs 256 x 256 tiles on CTA pairs
+// (tcgen05 cta_group::2) instead of 128 x 256 tiles on single CTAs.
+constexpr int64_t kPairRows = 1024;
+
 // Device address of the flag that bounded device-side waits set when they give up.
 int* device_error_ptr();
 

@@ -21,7 +21,9 @@
 // rasterized in bands of row tiles (at most 64 MiB of X) so a band of X stays in L2 while
 // the weight streams past it.
 // With few tiles (decode batches) the K loop is split and fp32 partials are reduced by a
-// second kernel that applies the epilogue.
+// second kernel that applies the epilogue.  Prompt-pass fp16 [K][N] GEMMs (from kPairRows
+// rows) run on CTA pairs instead (gemm_pair.cu); this kernel keeps the decode batches, the
+// LM head and the smaller fp16 GEMMs.
 #include <algorithm>
 #include <cstring>
 #include <cudaTypedefs.h>
@@ -864,8 +866,12 @@ size_t qgemm_ws_bytes(int64_t M, int N, int K) {
   return w + splitk_ws_bytes(M, N, K);
 }
 
+int gemm_pair_launch(const void* X, int64_t M, int N, int K, const void* W, const void* bias, const void* R,
+                     int relu, void* Y, cudaStream_t s);
+
 // mode: 0 = 4-bit weight W grouped along N, 1 = fp16 [K][N] weight, 2 = fp16 [N][K] weight,
-// 3 = 4-bit weight grouped along K.
+// 3 = 4-bit weight grouped along K.  An fp16 [K][N] weight with many rows (the prompt pass)
+// runs on CTA pairs (gemm_pair.cu).
 int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, const void* wparams, int G,
               const void* bias, const void* R, int relu, void* Y, bool out_f32, void* ws, size_t ws_bytes,
               cudaStream_t s, bool w_ready, LnFuse* ln) {
@@ -962,7 +968,9 @@ int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, c
   {
     ProfScope ps(out_f32 ? PROF_LM_HEAD : (M > 256 ? PROF_GEMM : PROF_GEMM_DECODE), s, flops, bytes);
     int st;
-    if (mode == B_Q4) st = launch<B_Q4, false>(ta, tb, tp, a, s);
+    if (mode == B_F16_MN && !out_f32 && a.splits == 1 && a.tail_tiles == 0 && M >= kPairRows)
+      st = gemm_pair_launch(X, M, N, K, w, bias, R, relu, Y, s);   // 256 x 256 tiles on CTA pairs
+    else if (mode == B_Q4) st = launch<B_Q4, false>(ta, tb, tp, a, s);
     else if (mode == B_Q4K) st = launch<B_Q4K, false>(ta, tb, tp, a, s);
     else if (mode == B_F16_MN) st = launch<B_F16_MN, false>(ta, tb, tp, a, s);
     else st = out_f32 ? launch<B_F16_K, true>(ta, tb, tp, a, s) : launch<B_F16_K, false>(ta, tb, tp, a, s);
