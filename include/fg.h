@@ -148,7 +148,10 @@ int fg_kv_append(fg_kv_cache* cache, const void* k, const void* v, int64_t row_s
  * fg_dequantize of the weight (exact fp16; W->w16 itself when set), products accumulate
  * in fp32.  K % 64 == 0, N % 256 == 0, N % (4 * group) == 0, group in {32, 64, 128}.
  * `workspace` may be NULL when fg_qgemm_workspace_bytes(M, N, K) is 0; with M >= 1024 and
- * enough workspace the 4-bit weight is first expanded to fp16 inside it. */
+ * enough workspace the 4-bit weight is first expanded to fp16 inside it.  The workspace also
+ * holds fp32 partial results when the output tiles do not fill the GPU evenly: K-split
+ * partials for few tiles, or the partial tiles of the last wave when that wave is spread over
+ * every SM (fg_qgemm_workspace_bytes counts them; FG_ERR_WORKSPACE if it is smaller). */
 size_t fg_qgemm_workspace_bytes(int64_t M, int N, int K);
 int fg_qgemm(const void* X, int64_t M, const fg_qlinear* W, const void* R, int relu, void* Y,
              void* workspace, size_t ws_bytes, void* stream);
@@ -156,7 +159,8 @@ int fg_qgemm(const void* X, int64_t M, const fg_qlinear* W, const void* R, int r
 /* The same tensor-core GEMM over an uncompressed fp16 weight W [K][N] (N contiguous): the
  * "FlexGen" README mirror's benchmark table contrasts FlexGen with and without compression;
  * this is the uncompressed side.  Y[M][N] = [relu](X W + b) [+ R], fp32 accumulation.
- * K % 64 == 0, N % 256 == 0; workspace >= fg_gemm_f16_workspace_bytes(M, N, K). */
+ * K % 64 == 0, N % 256 == 0; workspace >= fg_gemm_f16_workspace_bytes(M, N, K) (fp32 partial
+ * results as for fg_qgemm; 0 for the prompt-size GEMMs, which run on CTA pairs). */
 size_t fg_gemm_f16_workspace_bytes(int64_t M, int N, int K);
 int fg_gemm_f16(const void* X, int64_t M, const void* W, int K, int N, const void* bias,
                 const void* R, int relu, void* Y, void* workspace, size_t ws_bytes, void* stream);
