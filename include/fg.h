@@ -160,7 +160,8 @@ int fg_qgemm(const void* X, int64_t M, const fg_qlinear* W, const void* R, int r
  * "FlexGen" README mirror's benchmark table contrasts FlexGen with and without compression;
  * this is the uncompressed side.  Y[M][N] = [relu](X W + b) [+ R], fp32 accumulation.
  * K % 64 == 0, N % 256 == 0; workspace >= fg_gemm_f16_workspace_bytes(M, N, K) (fp32 partial
- * results as for fg_qgemm; 0 for the prompt-size GEMMs, which run on CTA pairs). */
+ * results as for fg_qgemm when the output tiles do not fill the GPU; from 1024 rows with
+ * enough tiles the GEMM runs on CTA pairs and needs none). */
 size_t fg_gemm_f16_workspace_bytes(int64_t M, int N, int K);
 int fg_gemm_f16(const void* X, int64_t M, const void* W, int K, int N, const void* bias,
                 const void* R, int relu, void* Y, void* workspace, size_t ws_bytes, void* stream);
