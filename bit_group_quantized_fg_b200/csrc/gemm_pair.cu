@@ -11,7 +11,9 @@
 //     (32 KB per stage instead of the 48 KB one SM would need for a 128 x 256 tile alone),
 //   - the leader (rank 0) issues tcgen05.mma.cta_group::2 M256 N256 K16, which reads both
 //     CTAs' shared memory and accumulates each CTA's 128 rows in its own tensor memory,
-//   - each CTA's epilogue warps read their 128 rows and apply bias / ReLU / residual.
+//   - each CTA's epilogue warps read their 128 rows, apply bias / ReLU / residual, and write
+//     each 32 x 32 fp16 box through shared memory with one TMA store (about 1 % faster at the
+//     OPT-30B prompt shapes than 16-byte stores from registers, under the same power cap).
 // Per SM, every MMA of 128 x 256 x 16 now reads 8 KB of shared memory instead of 12 KB.
 //
 // Scheduling: one cluster per tile, two CTAs per SM (3 stages of 32 KB, one 256-column
@@ -57,7 +59,10 @@ constexpr int kABytes = 128 * PK * 2;         // 16 KB: this CTA's rows of X
 constexpr int kBBytes = PK * (PN / 2) * 2;    // 16 KB: this CTA's columns of W (two 64-column blocks)
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kThreads = 256;  // warp 0 loads, warp 1 MMA (leader) / drain, warps 4-7 epilogue
-constexpr int kSmem = kStages * kStageBytes + 1024 + 256;
+constexpr int kStageOut = 4 * 32 * 32 * 2;  // one 32 x 32 fp16 output box per epilogue warp
+// stages, barriers (padded to 1 KB so the output boxes stay 1 KB aligned), output boxes, and
+// the alignment slack of the dynamic shared-memory base
+constexpr int kSmem = kStages * kStageBytes + 1024 + kStageOut + 1024;
 static_assert(kSmem <= 232448, "shared memory budget");
 
 struct PairArgs {
@@ -83,11 +88,12 @@ __device__ __forceinline__ void pair_tile(const PairArgs& a, int t, int& m0, int
 
 __global__ void __launch_bounds__(kThreads, 2)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                     const PairArgs args, int* err) {
+                     const __grid_constant__ CUtensorMap tm_y, const PairArgs args, int* err) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base_u32 = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024 - (base_u32 & 1023)) & 1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint8_t* out_box = smem + kStages * kStageBytes + 1024;
   uint64_t* full = bars;                         // [kStages] (leader)
   uint64_t* empty = bars + kStages;              // [kStages]
   uint64_t* acc_full = bars + 2 * kStages;       // [2]
@@ -203,7 +209,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         tmem_ld_32x32b_x32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * PN + cc), r);
         tmem_ld_wait();
         const int n = n0 + cc;
-        if (!row_ok) continue;
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
@@ -225,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.f);
         }
-        if (args.R != nullptr) {
+        if (args.R != nullptr && row_ok) {
           const uint4* rp = reinterpret_cast<const uint4*>(args.R + int64_t(m) * args.N + n);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -239,7 +244,12 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
           }
         }
-        uint4* dst = reinterpret_cast<uint4*>(args.Y + int64_t(m) * args.N + n);
+        // the warp's 32 x 32 box goes out through shared memory as one TMA store (the tensor
+        // map clips rows past M).  Lane l holds row l; with the 64-byte swizzle its four 16-byte
+        // pieces land in distinct banks for every 8 consecutive lanes.
+        uint8_t* box = out_box + q * 2048;
+        if (lane == 0) bulk_wait_read0();  // this warp's previous box has left shared memory
+        __syncwarp();
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint4 o;
@@ -247,7 +257,13 @@ __global__ void __launch_bounds__(kThreads, 2)
           o.y = h2_as_u32(__floats2half2_rn(v[8 * j + 2], v[8 * j + 3]));
           o.z = h2_as_u32(__floats2half2_rn(v[8 * j + 4], v[8 * j + 5]));
           o.w = h2_as_u32(__floats2half2_rn(v[8 * j + 6], v[8 * j + 7]));
-          dst[j] = o;
+          *reinterpret_cast<uint4*>(box + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) = o;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && m < args.M) {
+          tma_store_2d(&tm_y, n, m, box);
+          bulk_commit();
         }
       }
       tc_fence_before();
@@ -255,6 +271,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (lane == 0) mbar_arrive_cluster(acc_empty_leader + uint32_t(acc) * 8u);
       if (++acc == kAccs) { acc = 0; acc_phase ^= 1; }
     }
+    if (lane == 0) bulk_wait0();  // every box written before the CTA exits
   }
 
   tc_fence_before();
@@ -289,11 +306,13 @@ int gemm_pair_launch(const void* X, int64_t M, int N, int K, const void* W, cons
   a.R = reinterpret_cast<const __half*>(R);
   a.relu = relu;
   a.Y = reinterpret_cast<__half*>(Y);
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, ty;
   FG_TRY(make_map_2d(&ta, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, uint64_t(K), uint64_t(M), uint64_t(K) * 2, PK, 128,
                      CU_TENSOR_MAP_SWIZZLE_128B));
   FG_TRY(make_map_2d(&tb, W, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, uint64_t(N), uint64_t(K), uint64_t(N) * 2, 64, PK,
                      CU_TENSOR_MAP_SWIZZLE_128B));
+  FG_TRY(make_map_2d(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, uint64_t(N), uint64_t(M), uint64_t(N) * 2, 32, 32,
+                     CU_TENSOR_MAP_SWIZZLE_64B));
   static std::atomic<uint64_t> attr_done{0};
   FG_TRY(ensure_smem_attr(gemm_pair_kernel, kSmem, attr_done));
   const int clusters = a.total;   // one cluster per tile (see the header)
@@ -312,7 +331,7 @@ int gemm_pair_launch(const void* X, int64_t M, int N, int K, const void* W, cons
   cfg.attrs = at;
   cfg.numAttrs = 2;
   count_launch();
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel, ta, tb, a, err);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel, ta, tb, ty, a, err);
   if (e != cudaSuccess) return cuda_fail(e, "tcgen05 pair gemm kernel");
   return FG_OK;
 }
