@@ -28,10 +28,10 @@
 // Barriers (same offsets in both CTAs):
 //   full[s]      leader only: the leader's producer arms it with both CTAs' bytes; each
 //                CTA's tile loads count their bytes on it (cta_group::2 loads).
-//   empty[s]     each CTA: the leader's commit (multicast to both) frees stage s.
-//   acc_full[a]  each CTA: the leader's commit (multicast) says accumulator a is complete.
+//   empty[s]     each CTA: the leader's commit (signalled to both CTAs) frees stage s.
+//   acc_full[a]  each CTA: the leader's commit (signalled to both) says accumulator a is complete.
 //   acc_empty[a] leader only: 8 arrivals (4 epilogue warps of each CTA) free accumulator a.
-//   drain        each CTA: the leader's last commit (multicast), before TMEM is freed.
+//   drain        each CTA: the leader's last commit (signalled to both), before TMEM is freed.
 // Every wait is bounded (about 2 s); a wait that gives up records an error code for the host
 // and the kernel winds down.
 #include <algorithm>
