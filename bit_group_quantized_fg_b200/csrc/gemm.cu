@@ -22,7 +22,9 @@
 // the weight streams past it.
 // With few tiles (decode batches) the K loop is split and fp32 partials are reduced by a
 // second kernel that applies the epilogue.  Prompt-pass fp16 [K][N] GEMMs (from kPairRows
-// rows) run on CTA pairs instead (gemm_pair.cu); this kernel keeps the decode batches, the
+// rows) run on CTA pairs instead (gemm_pair.cu), and so do 4-bit GEMMs grouped along N of
+// 129-256 rows (gemm_q4pair.cu: each CTA of a pair expands half of a 256-column weight
+// tile); this kernel keeps decode batches of up to 128 rows, weights grouped along K, the
 // LM head and the smaller fp16 GEMMs.
 #include <algorithm>
 #include <cstring>
@@ -845,8 +847,21 @@ int* device_error_ptr() {
 
 // Split-K partials of one GEMM, or the fp32 segments of its wave tail (0 when the tiles
 // alone fill the GPU evenly).
+size_t q4_pair_ws_bytes(int64_t M, int N, int K);
+
 size_t splitk_ws_bytes(int64_t M, int N, int K) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
+  if (M > BM && M <= 2 * BM && N % BN == 0 && K % BK == 0) {
+    // 4-bit weights at these batch sizes run on CTA pairs (gemm_q4pair.cu); the fp16 path
+    // still runs single CTAs, so the workspace covers both plans
+    const size_t q = q4_pair_ws_bytes(M, N, K);
+    const int m_tiles = int((M + BM - 1) / BM), n_tiles = N / BN;
+    const int sp = pick_splits(m_tiles * n_tiles, K / BK);
+    size_t one = 0;
+    if (sp > 1) one = size_t(sp) * size_t(M) * size_t(N) * sizeof(float);
+    else if (pick_tail(m_tiles * n_tiles, K / BK, N) > 0) one = size_t(num_sms()) * 2 * BM * BN * sizeof(float);
+    return std::max(q, one);
+  }
   const int m_tiles = int((M + BM - 1) / BM);
   const int n_tiles = (N + BN - 1) / BN;
   const int sp = pick_splits(m_tiles * n_tiles, K / BK);
@@ -868,10 +883,14 @@ size_t qgemm_ws_bytes(int64_t M, int N, int K) {
 
 int gemm_pair_launch(const void* X, int64_t M, int N, int K, const void* W, const void* bias, const void* R,
                      int relu, void* Y, cudaStream_t s);
+int gemm_q4_pair_launch(const void* X, int64_t M, int N, int K, const void* w, const void* wparams, int G,
+                        const void* bias, const void* R, int relu, void* Y, void* ws, size_t ws_bytes,
+                        cudaStream_t s, int* splits_out, float** partial_out);
 
 // mode: 0 = 4-bit weight W grouped along N, 1 = fp16 [K][N] weight, 2 = fp16 [N][K] weight,
 // 3 = 4-bit weight grouped along K.  An fp16 [K][N] weight with many rows (the prompt pass)
-// runs on CTA pairs (gemm_pair.cu).
+// runs on CTA pairs (gemm_pair.cu), a 4-bit weight grouped along N at 129-256 rows too
+// (gemm_q4pair.cu).
 int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, const void* wparams, int G,
               const void* bias, const void* R, int relu, void* Y, bool out_f32, void* ws, size_t ws_bytes,
               cudaStream_t s, bool w_ready, LnFuse* ln) {
@@ -896,6 +915,27 @@ int gemm_impl(int mode, const void* X, int64_t M, int N, int K, const void* w, c
       (bias && !aligned16(bias)) || (R && !aligned16(R)))
     return fail(FG_ERR_ALIGN, "pointers must be 16-byte aligned");
   if (M == 0) return FG_OK;
+
+  if (mode == B_Q4 && !out_f32 && M > BM && M <= 2 * BM) {
+    // 129-256 rows: 256 x 256 tiles on CTA pairs, each CTA expanding half the weight tile
+    const double flops = 2.0 * double(M) * N * K;
+    const double bytes = double(N) * K * (0.5 + 4.0 / G) + double(M) * K * 2.0 + double(M) * N * 2.0 +
+                         (R ? double(M) * N * 2.0 : 0.0);
+    ProfScope ps(PROF_GEMM_DECODE, s, flops, bytes);
+    int sp = 1;
+    float* part = nullptr;
+    FG_TRY(gemm_q4_pair_launch(X, M, N, K, w, wparams, G, bias, R, relu, Y, ws, ws_bytes, s, &sp, &part));
+    if (sp > 1) {
+      if (ln && ln->g && ln->b && ln->H && !relu && N % 8 == 0 && N <= 12288 && aligned16(ln->g) &&
+          aligned16(ln->b) && aligned16(ln->H)) {
+        FG_TRY(splitk_reduce_ln_launch(part, sp, M, N, bias, R, Y, ln->g, ln->b, ln->H, s));
+        ln->done = true;
+      } else {
+        FG_TRY(splitk_reduce_launch(part, sp, M, N, bias, R, relu, Y, s));
+      }
+    }
+    return FG_OK;
+  }
 
   GemmArgs a{};
   a.M = int(M);

@@ -287,6 +287,13 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t cta_mask
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
+// The same arrival with the default CTA-scope release: it orders the arriving thread's
+// earlier writes to its own CTA's shared memory, which is all that a pair MMA issued after the
+// barrier completes reads from that CTA (the writer fences them to the async proxy first).
+// Per 64-deep k-block of a 4-bit pair GEMM the cluster-scope form cost ~0.5 us.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
 
 }  // namespace sm100
 }  // namespace fg

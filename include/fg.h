@@ -151,7 +151,9 @@ int fg_kv_append(fg_kv_cache* cache, const void* k, const void* v, int64_t row_s
  * enough workspace the 4-bit weight is first expanded to fp16 inside it.  The workspace also
  * holds fp32 partial results when the output tiles do not fill the GPU evenly: K-split
  * partials for few tiles, or the partial tiles of the last wave when that wave is spread over
- * every SM (fg_qgemm_workspace_bytes counts them; FG_ERR_WORKSPACE if it is smaller). */
+ * every SM (fg_qgemm_workspace_bytes counts them; FG_ERR_WORKSPACE if it is smaller).  From
+ * 129 to 256 rows a weight grouped along N runs 256 x 256 tiles on pairs of SMs, with the
+ * same kinds of partials per pair of SMs. */
 size_t fg_qgemm_workspace_bytes(int64_t M, int N, int K);
 int fg_qgemm(const void* X, int64_t M, const fg_qlinear* W, const void* R, int relu, void* Y,
              void* workspace, size_t ws_bytes, void* stream);

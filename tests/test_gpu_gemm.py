@@ -123,6 +123,40 @@ def test_qgemm_large_decode_sampled(fg, M, N, K):
     assert_close_rms(got, exp, what="sampled decode GEMM")
 
 
+@pytest.mark.parametrize("M,N,K", [
+    (256, 21504, 7168),    # wave tail over the pairs (84 tiles on 74 pairs)
+    (256, 7168, 28672),    # K split in two
+    (144, 12288, 12288),   # every tile's k-blocks spread over the pairs
+])
+def test_qgemm_pair_repeatable(fg, M, N, K):
+    """From 129 to 256 rows each SM of a pair expands half of every weight tile and hands it
+    to the pair's MMA through a barrier of the other SM.  A hand-off that let the MMA read a
+    half-tile before it was written would make repeated launches differ: 16 launches must be
+    bitwise identical, and sampled outputs match the oracle."""
+    import torch
+    from fg_synth import gpu as sg
+    x = torch.empty((M, K), dtype=torch.float16, device="cuda")
+    sg.fill(x, 9, 1, "normal", 1.0)
+    w = torch.empty((K, N), dtype=torch.float16, device="cuda")
+    sg.fill(w, 9, 2, "normal", 0.02)
+    b = torch.empty((N,), dtype=torch.float16, device="cuda")
+    sg.fill(b, 9, 3, "normal", 0.5)
+    lin = fg.DeviceQLinear.from_fp16(w, b, 64)
+    del w
+    ws = torch.empty((max(fg.fg_qgemm_workspace_bytes(M, N, K), 16),), dtype=torch.uint8, device="cuda")
+    y0 = fg.fg_qgemm(x, lin, workspace=ws)
+    outs = [fg.fg_qgemm(x, lin, workspace=ws) for _ in range(15)]
+    torch.cuda.synchronize()
+    assert all(torch.equal(y0, y) for y in outs)
+    rng = np.random.default_rng(N)
+    rows = np.concatenate([[0, M - 1], rng.integers(0, M, 4)])
+    cols = np.concatenate([[0, N - 1], rng.integers(0, N, 10)])
+    sub, pos = oracle_weight_groups(9, 2, K, N, 64, cols)
+    xr = fg_synth.values(9, 1, (rows[:, None] * K + np.arange(K)[None, :]).ravel(), "normal", 1.0).reshape(-1, K)
+    exp = oracle.qlinear(xr, sub)[:, pos]
+    assert_close_rms(to_np(y0)[rows][:, cols], exp, what="pair decode GEMM")
+
+
 def test_qgemm_prefill_size_sampled(fg):
     """Config-2 prefill QKV shape (M 32768, N 12288, K 4096) on sampled outputs."""
     M, N, K = 32768, 12288, 4096
